@@ -1,0 +1,118 @@
+"""Pins of the oracle's GEMM, routing, SwiGLU and combine: an integer GEMM
+that is exact (so the fp64 oracle must equal an int64 matmul), tiny GEMMs with
+hand-computed sums, a brute-force routing order, and closed forms."""
+import numpy as np
+
+from oracle import formats as F
+from oracle import gemm as G
+from oracle import moe as M
+from oracle import quant as Q
+
+
+def _codes_with_unit_scales(rng, rows, cols):
+    codes = rng.integers(0, 16, (rows, cols)).astype(np.uint8)
+    sf = np.full((rows, cols // 16), 0x38, dtype=np.uint8)  # E4M3 1.0
+    return F.pack_nibbles(codes), sf, codes
+
+
+def test_gemm_integer_special_case_equals_int_matmul():
+    """With every scale 1.0 and g = 1, 2*val(code) is an integer in
+    {0, +-1, +-2, +-3, +-4, +-6, +-8, +-12}; C*4 is then an integer matmul."""
+    rng = np.random.default_rng(0)
+    M_, N_, K_ = 48, 40, 320
+    a_p, a_sf, a_c = _codes_with_unit_scales(rng, M_, K_)
+    b_p, b_sf, b_c = _codes_with_unit_scales(rng, N_, K_)
+    C, _ = G.nvfp4_gemm_ref(a_p, a_sf, np.float32(1), b_p, b_sf, np.float32(1))
+    two_a = {0: 0, 1: 1, 2: 2, 3: 3, 4: 4, 5: 6, 6: 8, 7: 12}
+    ia = np.vectorize(lambda c: (-1 if c & 8 else 1) * two_a[c & 7])(a_c).astype(np.int64)
+    ib = np.vectorize(lambda c: (-1 if c & 8 else 1) * two_a[c & 7])(b_c).astype(np.int64)
+    assert np.array_equal(C * 4, (ia @ ib.T).astype(np.float64))
+
+
+def test_gemm_hand_computed_1x1x64():
+    # a: 64 x 1.5 (code 3) under sf 2.0 (0x40), g_a = 0.5
+    # b: 32 x 2.0 (code 4) then 32 x -0.5 (code 9) under sf 1.0, g_b = 4
+    # C = (0.5*4) * sum(1.5*2 * b) = 2 * 3 * (32*2 - 32*0.5) = 2*3*48 = 288
+    a = F.pack_nibbles(np.full((1, 64), 3, dtype=np.uint8))
+    b = F.pack_nibbles(np.array([[4] * 32 + [9] * 32], dtype=np.uint8))
+    C, bound = G.nvfp4_gemm_ref(a, np.full((1, 4), 0x40, np.uint8), np.float32(0.5), b, np.full((1, 4), 0x38, np.uint8), np.float32(4))
+    assert C[0, 0] == 288.0
+    assert bound[0, 0] == 2 * 3 * (32 * 2 + 32 * 0.5)
+
+
+def test_gemm_hand_computed_2x2x64_mixed_scales():
+    # row/col codes chosen so each output is a short hand sum
+    a = np.zeros((2, 64), np.uint8)
+    a[0, 0] = 7  # 6
+    a[1, 16] = 2  # 1
+    a[1, 63] = 13  # -3
+    b = np.zeros((2, 64), np.uint8)
+    b[0, 0] = 1  # 0.5
+    b[0, 16] = 5  # 3
+    b[1, 63] = 6  # 4
+    a_sf = np.array([[0x38, 0x40, 0x38, 0x30], [0x38, 0x48, 0x38, 0x30]], np.uint8)  # 1,2,1,.5 / 1,4,1,.5
+    b_sf = np.array([[0x38, 0x38, 0x38, 0x38], [0x38, 0x38, 0x38, 0x58]], np.uint8)  # 1,1,1,1 / 1,1,1,16
+    C, _ = G.nvfp4_gemm_ref(F.pack_nibbles(a), a_sf, np.float32(1), F.pack_nibbles(b), b_sf, np.float32(1))
+    # C00 = 6*0.5 = 3 ; C01 = 0 ; C10 = (1*4)*(3*1) = 12 ; C11 = (-3*0.5)*(4*16) = -96
+    assert C.tolist() == [[3.0, 0.0], [12.0, -96.0]]
+
+
+def test_route_matches_brute_force_order():
+    rng = np.random.default_rng(1)
+    T, k, E = 37, 3, 7
+    ids = np.stack([rng.choice(E, k, replace=False) for _ in range(T)])
+    counts, offsets, perm, inv = M.route(ids, E)
+    brute = sorted(((ids[t, s], t, s) for t in range(T) for s in range(k)))
+    assert perm.tolist() == [t * k + s for (_, t, s) in brute]
+    assert counts.tolist() == [sum(1 for (e, _, _) in brute if e == x) for x in range(E)]
+    assert offsets[0] == 0 and offsets[-1] == T * k
+    for t in range(T):
+        for s in range(k):
+            assert perm[inv[t, s]] == t * k + s
+
+
+def test_route_rejects_bad_ids():
+    import pytest
+
+    with pytest.raises(ValueError):
+        M.route(np.array([[0, 5]]), 5)
+
+
+def test_silu_closed_forms():
+    z = np.linspace(-30, 30, 601)
+    s = M.silu(z)
+    assert M.silu(np.array([0.0]))[0] == 0.0
+    np.testing.assert_allclose(s - M.silu(-z), z, rtol=0, atol=1e-12)  # z*sig(z) + z*sig(-z) = z
+    assert abs(M.silu(np.array([1.0]))[0] - 1.0 / (1.0 + np.exp(-1.0))) < 1e-16
+
+
+def test_combine_hand_example():
+    y = np.array([[1.0, 2.0], [10.0, 20.0], [100.0, 200.0]])
+    inv = np.array([[2, 0], [1, 2]])
+    w = np.array([[0.5, 2.0], [1.0, -1.0]])
+    out, bits = M.combine_ref(y, inv, w)
+    assert out.tolist() == [[52.0, 104.0], [-90.0, -180.0]]
+    assert np.array_equal(F.bf16_bits_to_f32(bits), out.astype(np.float32))
+
+
+def test_w13_interleave_layout():
+    w1 = np.arange(32 * 2).reshape(32, 2)
+    w3 = 1000 + np.arange(32 * 2).reshape(32, 2)
+    w13 = M.interleave_w13(w1, w3)
+    assert w13[0:16].tolist() == w1[0:16].tolist()
+    assert w13[16:32].tolist() == w3[0:16].tolist()
+    assert w13[32:48].tolist() == w1[16:32].tolist()
+    a, b = M.deinterleave_w13(w13)
+    assert np.array_equal(a, w1) and np.array_equal(b, w3)
+
+
+def test_expert_ffn_requantizes_h_with_static_scale():
+    rng = np.random.default_rng(2)
+    x = rng.standard_normal((5, 64))
+    w1, w3 = rng.standard_normal((32, 64)) * 0.1, rng.standard_normal((32, 64)) * 0.1
+    w2 = rng.standard_normal((64, 32)) * 0.1
+    r = M.expert_ffn_ref(x, w1, w3, w2, np.float32(0.01))
+    np.testing.assert_allclose(r["h"], (r["gate"] / (1 + np.exp(-r["gate"]))) * r["up"], rtol=1e-15)
+    c2, s2, _ = Q.nvfp4_quantize(r["h"].astype(np.float32), g=np.float32(0.01))
+    assert np.array_equal(c2, r["h_codes"]) and np.array_equal(s2, r["h_sf"])
+    np.testing.assert_allclose(r["y"], r["h_dq"] @ w2.T, rtol=1e-15)

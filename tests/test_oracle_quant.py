@@ -1,0 +1,222 @@
+"""Pins of the oracle's quantizers and remap: exhaustive round trips of every
+representable block, brute-force optimality of the chosen scale and codes,
+closed-form error bounds, and the pages' "lossless remap" invariant checked
+over every exponent pair."""
+import numpy as np
+import pytest
+
+from oracle import formats as F
+from oracle import quant as Q
+from oracle.layouts import mma_sf_index, sf_from_mma, sf_to_mma
+
+
+def _nv_block(codes16, sf, g):
+    return (F.e2m1_decode(codes16) * F.e4m3_decode(np.uint8(sf)) * g).astype(np.float32)
+
+
+def test_nv_round_trip_every_code_and_scale():
+    """Every block val(code)*dec(sf)*g whose largest magnitude is 6 (so the
+    block amax pins sf) quantizes back to its own codes and scale, for all 16
+    codes in every position and all 126 positive finite E4M3 scales."""
+    g = np.float32(2.0**-4)
+    rng = np.random.default_rng(0)
+    rows, sfs = [], []
+    for sf in range(1, 0x7F):
+        for rep in range(2):
+            c = rng.integers(0, 16, size=16).astype(np.uint8)
+            c[rng.integers(0, 16)] = 7 if rep == 0 else 15  # +-6 sets amax
+            c[:16] = c if rep == 0 else np.roll(np.arange(16, dtype=np.uint8), sf % 16)
+            if not np.any((c & 7) == 7):
+                c[0] = 7
+            rows.append(c)
+            sfs.append(sf)
+    codes = np.stack(rows)
+    x = np.stack([_nv_block(c, s, g) for c, s in zip(codes, sfs)])
+    packed, sf_out, g_out = Q.nvfp4_quantize(x, g=g)
+    assert np.array_equal(sf_out[:, 0], np.array(sfs, dtype=np.uint8))
+    got = F.unpack_nibbles(packed)
+    # +0 and -0 are both exact for a zero element; compare magnitudes and the
+    # sign of every nonzero element
+    assert np.array_equal(got & 7, codes & 7)
+    nz = (codes & 7) != 0
+    assert np.array_equal(got[nz] & 8, codes[nz] & 8)
+
+
+def test_nv_scale_is_nearest_e4m3_and_codes_nearest_values():
+    """Brute force over all 127 E4M3 values and all 16 codes: sf is the E4M3
+    value nearest to amax_b/(6g) (as computed in fp32), and each code's
+    dequantized value is the nearest representable value to x under that
+    block scale (within the one fp32 rounding of x*(1/s))."""
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal((64, 256)).astype(np.float32)
+    x[rng.random(x.shape) < 0.01] *= 30
+    packed, sf, g = Q.nvfp4_quantize(x)
+    xb = x.reshape(64, 16, 16)
+    amax_b = np.abs(xb).max(axis=2).astype(np.float32)
+    q = (amax_b / np.float32(np.float32(6) * g)).astype(np.float64)
+    dist = np.abs(q[..., None] - F.E4M3_VALUES[None, None, :])
+    best = dist.min(axis=2)
+    assert np.all(np.abs(q - F.e4m3_decode(sf)) == best)
+    s = (F.e4m3_decode(sf) * g).astype(np.float64)
+    codes = F.unpack_nibbles(packed).reshape(64, 16, 16)
+    deq = F.e2m1_decode(codes) * s[..., None]
+    allv = np.concatenate([F.E2M1_MAGNITUDES, -F.E2M1_MAGNITUDES])
+    cand = np.abs(xb[..., None].astype(np.float64) - allv * s[..., None, None])
+    err = np.abs(xb - deq)
+    slack = np.abs(xb).astype(np.float64) * 2.0**-22
+    assert np.all(err <= cand.min(axis=-1) + slack)
+
+
+def test_nv_global_scale_closed_form():
+    x = np.array([[0.0] * 15 + [-2688.0]], dtype=np.float32)
+    assert Q.nv_global_scale(x) == np.float32(1.0)
+    packed, sf, g = Q.nvfp4_quantize(x)
+    assert g == 1.0 and sf[0, 0] == 0x7E  # 448
+    assert F.unpack_nibbles(packed)[0, 15] == 15  # -6
+
+
+def test_nv_error_bound():
+    """|x - x_hat| <= half the E2M1 grid step at |x|/s, times s (saturation
+    adds at most 0.375 s, inside the top bin's half step of 1)."""
+    rng = np.random.default_rng(2)
+    x = (rng.standard_normal((32, 512)) * rng.exponential(1.0, (32, 1))).astype(np.float32)
+    packed, sf, g = Q.nvfp4_quantize(x)
+    xh = Q.nvfp4_dequantize(packed, sf, g)
+    s = np.repeat(F.e4m3_decode(sf) * g, 16, axis=1)
+    a = np.abs(x) / s
+    half_step = np.where(a < 2, 0.25, np.where(a < 4, 0.5, 1.0))
+    assert np.all(np.abs(x - xh) <= half_step * s * (1 + 1e-6))
+
+
+def test_nv_zero_tensor_and_zero_block():
+    x = np.zeros((2, 32), dtype=np.float32)
+    x[1, :] = -0.0
+    packed, sf, g = Q.nvfp4_quantize(x)
+    assert g == 0 and np.all(sf == 0)
+    assert np.all(F.unpack_nibbles(packed)[0] == 0) and np.all(F.unpack_nibbles(packed)[1] == 8)
+    y = np.zeros((1, 32), dtype=np.float32)
+    y[0, 16:] = 1.0
+    packed, sf, g = Q.nvfp4_quantize(y)
+    assert sf[0, 0] == 0 and np.all(F.unpack_nibbles(packed)[0, :16] == 0)
+
+
+def test_nv_static_scale_saturates():
+    x = np.full((1, 16), 100.0, dtype=np.float32)
+    packed, sf, g = Q.nvfp4_quantize(x, g=np.float32(1e-3))  # far too small a g
+    assert sf[0, 0] == 0x7E and np.all(F.unpack_nibbles(packed) == 7)
+
+
+def test_mx_round_trip_every_code_and_scale():
+    rng = np.random.default_rng(3)
+    rows, scales = [], []
+    for c in range(0, 255):
+        X = c - 127
+        if X > 125 or X < -125:  # 6 * 2^X must be a finite normal fp32
+            continue
+        codes = rng.integers(0, 16, size=32).astype(np.uint8)
+        codes[rng.integers(0, 32)] = 7 if c % 2 else 14  # magnitude 6 or 4 pins X
+        rows.append(codes)
+        scales.append(c)
+    codes = np.stack(rows)
+    x = (F.e2m1_decode(codes) * F.ue8m0_decode(np.array(scales))[:, None]).astype(np.float32)
+    packed, sc = Q.mxfp4_quantize(x)
+    assert np.array_equal(sc[:, 0], np.array(scales, dtype=np.uint8))
+    got = F.unpack_nibbles(packed)
+    assert np.array_equal(got & 7, codes & 7)
+    nz = (codes & 7) != 0
+    assert np.array_equal(got[nz] & 8, codes[nz] & 8)
+
+
+def test_mx_scale_closed_form_and_nearest_codes():
+    rng = np.random.default_rng(4)
+    x = (rng.standard_normal((16, 256)) * np.exp2(rng.integers(-20, 20, (16, 1)))).astype(np.float32)
+    packed, sc = Q.mxfp4_quantize(x)
+    xb = x.reshape(16, 8, 32).astype(np.float64)
+    amax = np.abs(xb).max(axis=2)
+    scale = np.ldexp(1.0, sc.astype(np.int64) - 127)
+    ratio = amax / scale
+    assert np.all((ratio >= 4) & (ratio < 8))  # X = floor(log2 amax) - 2
+    codes = F.unpack_nibbles(packed).reshape(16, 8, 32)
+    deq = F.e2m1_decode(codes) * scale[..., None]
+    allv = np.concatenate([F.E2M1_MAGNITUDES, -F.E2M1_MAGNITUDES])
+    cand = np.abs(xb[..., None] - allv * scale[..., None, None]).min(axis=-1)
+    assert np.all(np.abs(xb - deq) <= cand)  # scaling by 2^-X is exact
+
+
+def test_mx_zero_block_and_tiny_values():
+    x = np.zeros((1, 64), dtype=np.float32)
+    x[0, 32] = np.float32(2.0**-140)  # subnormal: X clamps to -127
+    packed, sc = Q.mxfp4_quantize(x)
+    assert sc[0, 0] == 0 and sc[0, 1] == 0
+    # 2^-140 * 2^127 = 2^-13 rounds to zero in E2M1
+    assert np.all(F.unpack_nibbles(packed)[0] & 7 == 0)
+
+
+@pytest.mark.parametrize("span", list(range(0, 18)))
+def test_remap_lossless_for_every_exponent_pair(span):
+    """The pages' claim (remap keeps every dequantized weight): enumerate a
+    reference exponent and every other exponent within `span` octaves below it;
+    dequant(MX) must equal dequant(NV) exactly in fp64, codes untouched."""
+    for e_top in (-100, -3, 0, 7, 100):
+        e_low = e_top - span
+        if e_low < -127:
+            continue
+        codes = np.zeros((2, 32), dtype=np.uint8)
+        codes[0, :] = np.arange(32) % 16
+        codes[1, :] = (np.arange(32) * 7) % 16
+        codes[:, 0] = 7
+        scales = np.array([[e_top + 127], [e_low + 127]], dtype=np.uint8)
+        packed = F.pack_nibbles(codes)
+        nv_sf, g = Q.mx_to_nv(packed, scales, 1)
+        mx = Q.mxfp4_dequantize(packed, scales)
+        nv = Q.nvfp4_dequantize(packed, nv_sf, g[0])
+        assert np.array_equal(mx, nv)
+        assert g[0] == np.float32(np.ldexp(1.0, e_top - 8))
+
+
+def test_remap_span_18_is_range_error():
+    codes = np.full((2, 32), 1, dtype=np.uint8)
+    scales = np.array([[127 + 10], [127 + 10 - 18]], dtype=np.uint8)
+    with pytest.raises(Q.RemapRangeError):
+        Q.mx_to_nv(F.pack_nibbles(codes), scales, 1)
+
+
+def test_remap_dead_blocks_get_zero_scale_and_do_not_set_range():
+    codes = np.zeros((2, 32), dtype=np.uint8)
+    codes[0, 3] = 5
+    codes[1, :] = 8  # all -0: a dead block, its exponent is ignored
+    scales = np.array([[127 + 50], [0]], dtype=np.uint8)
+    nv_sf, g = Q.mx_to_nv(F.pack_nibbles(codes), scales, 1)
+    assert nv_sf[1, 0] == 0 and nv_sf[1, 1] == 0
+    assert nv_sf[0, 0] == nv_sf[0, 1] == ((8 + 7) << 3)
+
+
+def test_remap_per_tensor_globals():
+    rng = np.random.default_rng(5)
+    w = (rng.standard_normal((4 * 8, 128)) * 0.02).astype(np.float32)
+    w[:8] *= 100  # tensor 0 has a different range
+    packed, sc = Q.mxfp4_quantize(w)
+    nv_sf, g = Q.mx_to_nv(packed, sc, 4)
+    for t in range(4):
+        sl = slice(8 * t, 8 * t + 8)
+        assert np.array_equal(Q.mxfp4_dequantize(packed[sl], sc[sl]), Q.nvfp4_dequantize(packed[sl], nv_sf[sl], g[t]))
+    assert g[0] > g[1]
+
+
+def test_e4m3_power_of_two_encoding():
+    for k in range(-9, 9):
+        b = Q.e4m3_power_of_two(k)
+        assert F.e4m3_decode(b) == 2.0**k
+
+
+def test_mma_layout_permutation():
+    rows, cols = 200, 192
+    idx = mma_sf_index(rows, cols)
+    flat = idx.reshape(-1)
+    assert len(np.unique(flat)) == flat.size  # a permutation (into the padded buffer)
+    # hand-worked positions: row 33, block 5 -> slab 0, k-step 1, line 1, column group 1, byte 1
+    assert idx[33, 5] == 1 * 512 + 1 * 16 + 1 * 4 + 1
+    # row 130 (slab 1, line 2, group 0), block 11 (k-step 2, byte 3): (1*3 + 2)*512 + 2*16 + 0 + 3
+    assert idx[130, 11] == 5 * 512 + 32 + 3
+    sf = np.random.default_rng(6).integers(0, 256, (rows, cols // 16)).astype(np.uint8)
+    assert np.array_equal(sf_from_mma(sf_to_mma(sf), rows, cols), sf)
