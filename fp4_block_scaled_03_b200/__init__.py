@@ -1,0 +1,272 @@
+"""Python binding of libfp4.so (NVFP4 / MXFP4 W4A4 MoE expert path, sm_100a).
+
+Argument marshalling only: every computation runs in the library's CUDA
+kernels.  PyTorch supplies device memory and the current stream.  The
+library is loaded from this package directory; importing the package on a
+machine without the built library raises immediately, and there is no CPU
+fallback anywhere.
+
+The functions with the C names (``fp4_quantize``, ``fp4_gemm`` ...) take
+tensors for the C pointers and raise ``Fp4Error`` on a non-OK status; the
+``quantize_nv`` / ``gemm`` / ``moe_layer`` helpers also allocate the outputs.
+"""
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfp4.so")
+
+FP4_NV, FP4_MX = 0, 1
+FP4_OUT_F32, FP4_OUT_BF16 = 0, 1
+FP4_STATIC_GLOBAL_SCALE = 0x1
+FP4_SCALE_LAYOUT_TILED = 0x2
+FP4_DEBUG_DUMP_H = 0x4
+
+STATUS = {
+    0: "FP4_OK",
+    1: "FP4_ERR_INVALID_ARG",
+    2: "FP4_ERR_ALIGNMENT",
+    3: "FP4_ERR_UNSUPPORTED_SHAPE",
+    4: "FP4_ERR_RANGE",
+    5: "FP4_ERR_BAD_EXPERT",
+    6: "FP4_ERR_WORKSPACE",
+    7: "FP4_ERR_DEVICE_TIMEOUT",
+    8: "FP4_ERR_CUDA",
+}
+
+
+class Fp4Error(RuntimeError):
+    def __init__(self, code, where):
+        self.code = code
+        super().__init__(f"{where}: {STATUS.get(code, code)}")
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libfp4.so is not built ({LIB_PATH}); run python -m fp4_block_scaled_03_b200.build")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_I32 = ctypes.c_int32
+_U32 = ctypes.c_uint32
+_SZ = ctypes.c_size_t
+
+
+class MoeWeights(ctypes.Structure):
+    _fields_ = [
+        ("w13_codes", _P),
+        ("w13_sf", _P),
+        ("w13_g", _P),
+        ("w2_codes", _P),
+        ("w2_sf", _P),
+        ("w2_g", _P),
+        ("h_g", _P),
+    ]
+
+
+_SIGS = {
+    "fp4_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "fp4_sf_tiled_bytes": (_SZ, [_I64, _I64]),
+    "fp4_quantize_workspace_size": (_SZ, []),
+    "fp4_quantize": (ctypes.c_int, [ctypes.c_int, _P, _I64, _I64, _I64, _P, _P, _P, _U32, _P, _SZ, _P]),
+    "fp4_mx_to_nv": (ctypes.c_int, [_P, _P, _I64, _I64, _I64, _P, _P, _U32, _P]),
+    "fp4_gemm": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, ctypes.c_int, _I64, _I64, _I64, _U32, _P]),
+    "fp4_moe_workspace_size": (_SZ, [_I64, _I32, _I64, _I64, _I32]),
+    "fp4_moe_grouped_gemm": (
+        ctypes.c_int,
+        [_P, _P, _P, _I64, _I32, ctypes.POINTER(MoeWeights), _I64, _I64, _I32, _P, _P, _SZ, _U32, _P, _P],
+    ),
+    "fp4_moe_route_scratch_bytes": (_SZ, [_I64, _I32]),
+    "fp4_moe_route": (ctypes.c_int, [_P, _I64, _I32, _I32, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "fp4_moe_gather": (ctypes.c_int, [_P, _P, _I64, _I32, _I64, _I32, _P, _P, _P, _P, _P, _I64, _P]),
+    "fp4_moe_w13": (
+        ctypes.c_int,
+        [_P, _P, _P, ctypes.POINTER(MoeWeights), _I64, _I64, _I32, _P, _P, _I64, _P, _P, _U32, _P, _P],
+    ),
+    "fp4_moe_w2": (
+        ctypes.c_int,
+        [_P, _P, ctypes.POINTER(MoeWeights), _I64, _I64, _I32, _P, _P, _P, _P, _P, _I64, _P, _P],
+    ),
+    "fp4_moe_combine": (ctypes.c_int, [_P, _P, _I64, _I32, _I64, _P, _P]),
+    "fp4_get_device_status": (ctypes.c_int, [_P]),
+    "fp4_set_wait_limit_ns": (None, [ctypes.c_uint64]),
+}
+
+for _name, (_res, _args) in _SIGS.items():
+    _f = getattr(lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+EXPORTED = sorted(_SIGS)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream():
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _check(code, where):
+    if code != 0:
+        raise Fp4Error(code, where)
+
+
+# ---- C-named entry points (tensors in, status checked) ----------------------
+
+def fp4_quantize(fmt, x, rows, cols, ld, codes, scales, global_scale, flags, workspace, ws_bytes):
+    _check(lib.fp4_quantize(fmt, _ptr(x), rows, cols, ld, _ptr(codes), _ptr(scales), _ptr(global_scale), flags,
+                            _ptr(workspace), ws_bytes, _stream()), "fp4_quantize")
+
+
+def fp4_mx_to_nv(codes, mx_scales, rows, cols, num_tensors, nv_scales, nv_global, flags=0):
+    _check(lib.fp4_mx_to_nv(_ptr(codes), _ptr(mx_scales), rows, cols, num_tensors, _ptr(nv_scales),
+                            _ptr(nv_global), flags, _stream()), "fp4_mx_to_nv")
+
+
+def fp4_gemm(a_codes, a_sf, a_g, b_codes, b_sf, b_g, c, c_dtype, M, N, K, flags=0):
+    _check(lib.fp4_gemm(_ptr(a_codes), _ptr(a_sf), _ptr(a_g), _ptr(b_codes), _ptr(b_sf), _ptr(b_g), _ptr(c),
+                        c_dtype, M, N, K, flags, _stream()), "fp4_gemm")
+
+
+def fp4_moe_route(expert_ids, T, topk, E, counts, offsets, tile_offsets, perm, inv, scratch):
+    _check(lib.fp4_moe_route(_ptr(expert_ids), T, topk, E, _ptr(counts), _ptr(offsets), _ptr(tile_offsets),
+                             _ptr(perm), _ptr(inv), _ptr(scratch), scratch.numel() * scratch.element_size(),
+                             _stream()), "fp4_moe_route")
+
+
+def fp4_moe_gather(x_codes, x_sf, T, topk, H, E, offsets, tile_offsets, perm, a_codes, a_sf, rows_cap):
+    _check(lib.fp4_moe_gather(_ptr(x_codes), _ptr(x_sf), T, topk, H, E, _ptr(offsets), _ptr(tile_offsets),
+                              _ptr(perm), _ptr(a_codes), _ptr(a_sf), rows_cap, _stream()), "fp4_moe_gather")
+
+
+def fp4_moe_w13(a_codes, a_sf, a_g, w, H, I, E, counts, tile_offsets, rows_cap, h_codes, h_sf, flags=0, h_dump=None):
+    _check(lib.fp4_moe_w13(_ptr(a_codes), _ptr(a_sf), _ptr(a_g), ctypes.byref(w.c_struct()), H, I, E, _ptr(counts),
+                           _ptr(tile_offsets), rows_cap, _ptr(h_codes), _ptr(h_sf), flags, _ptr(h_dump), _stream()),
+           "fp4_moe_w13")
+
+
+def fp4_moe_w2(h_codes, h_sf, w, H, I, E, counts, offsets, tile_offsets, perm, topk_weights, rows_cap, y):
+    _check(lib.fp4_moe_w2(_ptr(h_codes), _ptr(h_sf), ctypes.byref(w.c_struct()), H, I, E, _ptr(counts),
+                          _ptr(offsets), _ptr(tile_offsets), _ptr(perm), _ptr(topk_weights), rows_cap, _ptr(y),
+                          _stream()), "fp4_moe_w2")
+
+
+def fp4_moe_combine(y, inv, T, topk, H, out):
+    _check(lib.fp4_moe_combine(_ptr(y), _ptr(inv), T, topk, H, _ptr(out), _stream()), "fp4_moe_combine")
+
+
+def fp4_moe_grouped_gemm(tokens, expert_ids, topk_weights, T, topk, w, H, I, E, out, workspace, flags=0,
+                         h_dump=None):
+    _check(lib.fp4_moe_grouped_gemm(_ptr(tokens), _ptr(expert_ids), _ptr(topk_weights), T, topk,
+                                    ctypes.byref(w.c_struct()), H, I, E, _ptr(out), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), flags, _ptr(h_dump), _stream()),
+           "fp4_moe_grouped_gemm")
+
+
+def fp4_get_device_status():
+    return lib.fp4_get_device_status(_stream())
+
+
+def fp4_set_wait_limit_ns(ns):
+    lib.fp4_set_wait_limit_ns(int(ns))
+
+
+def fp4_sf_tiled_bytes(rows, cols):
+    return lib.fp4_sf_tiled_bytes(rows, cols)
+
+
+def fp4_moe_workspace_size(T, topk, H, I, E):
+    return lib.fp4_moe_workspace_size(T, topk, H, I, E)
+
+
+def fp4_moe_route_scratch_bytes(R, E):
+    return lib.fp4_moe_route_scratch_bytes(R, E)
+
+
+# ---- allocating helpers -------------------------------------------------------
+
+def _u8(n, dev):
+    return torch.empty(int(n), dtype=torch.uint8, device=dev)
+
+
+def quantize_nv(x, g=None, tiled=False):
+    """bf16 [rows, cols] -> (codes u8 [rows, cols/2], scales u8, g fp32[1])."""
+    rows, cols = x.shape
+    dev = x.device
+    codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
+    scales = _u8(fp4_sf_tiled_bytes(rows, cols), dev) if tiled else torch.empty((rows, cols // 16), dtype=torch.uint8, device=dev)
+    flags = FP4_SCALE_LAYOUT_TILED if tiled else 0
+    if g is not None:
+        gs = g.to(device=dev, dtype=torch.float32).reshape(1).clone()
+        flags |= FP4_STATIC_GLOBAL_SCALE
+        ws = None
+        ws_bytes = 0
+    else:
+        gs = torch.empty(1, dtype=torch.float32, device=dev)
+        ws_bytes = lib.fp4_quantize_workspace_size()
+        ws = _u8(ws_bytes, dev)
+    fp4_quantize(FP4_NV, x, rows, cols, x.stride(0), codes, scales, gs, flags, ws, ws_bytes)
+    return codes, scales, gs
+
+
+def quantize_mx(x):
+    rows, cols = x.shape
+    dev = x.device
+    codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((rows, cols // 32), dtype=torch.uint8, device=dev)
+    fp4_quantize(FP4_MX, x, rows, cols, x.stride(0), codes, scales, None, 0, None, 0)
+    return codes, scales
+
+
+def mx_to_nv(codes, mx_scales, num_tensors):
+    total_rows, half = codes.shape
+    rows, cols = total_rows // num_tensors, half * 2
+    nv = torch.empty((total_rows, cols // 16), dtype=torch.uint8, device=codes.device)
+    g = torch.empty(num_tensors, dtype=torch.float32, device=codes.device)
+    fp4_mx_to_nv(codes, mx_scales, rows, cols, num_tensors, nv, g)
+    return nv, g
+
+
+def gemm(a_codes, a_sf, a_g, b_codes, b_sf, b_g, M, N, K, out_dtype=torch.float32):
+    c = torch.empty((M, N), dtype=out_dtype, device=a_codes.device)
+    fp4_gemm(a_codes, a_sf, a_g, b_codes, b_sf, b_g, c, FP4_OUT_F32 if out_dtype == torch.float32 else FP4_OUT_BF16,
+             M, N, K)
+    return c
+
+
+class MoeWeightSet:
+    """Device tensors of one layer's NVFP4 expert weights (see fp4.h)."""
+
+    def __init__(self, w13_codes, w13_sf, w13_g, w2_codes, w2_sf, w2_g, h_g):
+        self.w13_codes, self.w13_sf, self.w13_g = w13_codes, w13_sf, w13_g
+        self.w2_codes, self.w2_sf, self.w2_g = w2_codes, w2_sf, w2_g
+        self.h_g = h_g
+        self._c = MoeWeights(*[_ptr(t) for t in (w13_codes, w13_sf, w13_g, w2_codes, w2_sf, w2_g, h_g)])
+
+    def c_struct(self):
+        return self._c
+
+
+def moe_rows_cap(T, topk, E):
+    return ((T * topk + 127 * E + 127) // 128) * 128
+
+
+def moe_layer(x, expert_ids, topk_weights, w, H, I, E, workspace=None, out=None, h_dump=None):
+    T, topk = expert_ids.shape
+    dev = x.device
+    if workspace is None:
+        workspace = _u8(fp4_moe_workspace_size(T, topk, H, I, E), dev)
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    flags = FP4_DEBUG_DUMP_H if h_dump is not None else 0
+    fp4_moe_grouped_gemm(x, expert_ids, topk_weights, T, topk, w, H, I, E, out, workspace, flags, h_dump)
+    return out

@@ -1,0 +1,525 @@
+// Block-scaled FP4 x FP4 GEMM on the sm_100a 5th-generation tensor core.
+//
+// "DeepSeek-V4.1-Flash-NVFP4", §二: the W4A4 product runs on 4-bit E2M1
+// operands with one scale per 16 elements multiplied back in the fp32
+// accumulator.  On B200 that is one instruction, tcgen05.mma
+// kind::mxf4nvf4.block_scale (E4M3 scale per 16 K-elements, fp32
+// accumulation in tensor memory), so the kernel only stages operands:
+//
+//   warp 0      TMA producer: per K stage, a 128 x 256 A tile and a BN x 256
+//               B tile (packed codes, 128-byte swizzle) plus their scale tiles
+//               (bulk copies of the tiled scale layout) into a ring of shared
+//               memory stages, completing on the stage's "full" mbarrier.
+//   warp 1      allocates tensor memory; one lane copies each stage's scale
+//               tiles shared -> TMEM (tcgen05.cp) and issues 4 MMAs of
+//               K = 64, then commits to the stage's "empty" barrier; after
+//               the last K stage it commits to "acc_full".
+//   warps 2-5   epilogue: tcgen05.ld of the 128 x BN fp32 accumulator (each
+//               thread one row), then the fused output step for the caller:
+//                 dense    alpha * acc -> fp32 or bf16
+//                 w13      SwiGLU over interleaved 16-column gate/up groups,
+//                          then NVFP4 re-quantization of h with a static
+//                          per-expert scale (codes + tiled scales)
+//                 w2       routing weight * alpha * acc -> fp32 rows
+//               and arrives on "acc_empty".
+//
+// The grid is persistent (at most one CTA per SM); every role walks the same
+// tile sequence.  Grouped (MoE) tiles are (128-row tile of one expert's
+// padded rows) x (BN columns of that expert's weights).  Every mbarrier wait
+// is bounded; on expiry the CTA records FP4_ERR_DEVICE_TIMEOUT, lets its
+// in-flight copies and MMAs finish, frees tensor memory and returns.
+#include <mutex>
+
+#include "common.cuh"
+
+namespace fp4 {
+namespace {
+
+constexpr int BM = 128;        // rows per tile (MMA M)
+constexpr int BK_BYTES = 128;  // one 128-byte swizzle row = 256 FP4 elements per stage
+constexpr int kThreads = 192;
+
+enum Epi { EPI_F32 = 0, EPI_BF16 = 1, EPI_W13 = 2, EPI_W2 = 3 };
+
+template <int BN>
+struct Cfg {
+  static constexpr int kStages = 4;
+  static constexpr int A_BYTES = BM * BK_BYTES;
+  static constexpr int B_BYTES = BN * BK_BYTES;
+  static constexpr int HALVES = (BN + 127) / 128;  // 128-row scale slabs of B per tile
+  static constexpr int SFA_BYTES = 4 * 512;
+  static constexpr int SFB_BYTES = HALVES * 4 * 512;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int ACC_COL = 0;
+  static constexpr int SFA_COL = 256;                 // 4 K-words x 4 columns
+  static constexpr int SFB_COL = 256 + 16;            // 4 K-words x 4*HALVES columns
+  static constexpr int SMEM_BYTES = kStages * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+  static_assert(BN % 32 == 0 && BN <= 256, "BN");
+  static_assert(SFB_COL + 16 * HALVES <= TMEM_COLS, "tmem");
+};
+
+struct Params {
+  int M, N, K;       // dense: A rows M; grouped: N and K per expert
+  int n_tiles;       // ceil(N / BN)
+  int m_tiles;       // dense only
+  int k_stages;      // ceil(K / 256)
+  int kw;            // K / 64 (scale words per row)
+  const uint8_t *a_sf;
+  const uint8_t *b_sf;
+  int64_t b_sf_rows;  // rows covered by b's tiled scale buffer (padded to 128)
+  // dense
+  const float *a_g;
+  const float *b_g;
+  void *c;
+  // grouped
+  int E;
+  const int32_t *counts;
+  const int32_t *offsets;
+  const int32_t *tile_offsets;
+  const float *w_g;  // per-expert weight tensor scale
+  const float *h_g;  // per-expert h scale
+  uint8_t *h_codes;
+  uint8_t *h_sf;
+  float *h_dump;
+  int I;
+  const int32_t *perm;
+  const float *topk_w;
+  float *y;
+  unsigned int *status;
+  uint64_t wait_limit;
+};
+
+struct TileInfo {
+  int a_row0;     // first A row (tensor-map row coordinate)
+  int a_slab;     // 128-row slab index of A's scales
+  int b_row0;     // first B row
+  int n0;         // first output column within the expert / matrix
+  int e;          // expert (grouped) or 0
+  int rows_valid; // rows of this tile that hold data
+  int out_row0;   // grouped w2: first routed row of the tile (unpadded)
+};
+
+__device__ __forceinline__ int upper_bound_i32(const int32_t *a, int n, int v) {
+  int lo = 0, hi = n;  // first index with a[i] > v
+  while (lo < hi) {
+    int mid = (lo + hi) >> 1;
+    if (a[mid] <= v) lo = mid + 1; else hi = mid;
+  }
+  return lo;
+}
+
+template <int BN, bool kGrouped>
+__device__ __forceinline__ TileInfo tile_info(const Params &p, int t) {
+  TileInfo ti;
+  const int mt = t / p.n_tiles, nt = t - (t / p.n_tiles) * p.n_tiles;
+  ti.n0 = nt * BN;
+  ti.a_row0 = mt * BM;
+  ti.a_slab = mt;
+  if (kGrouped) {
+    const int e = upper_bound_i32(p.tile_offsets, p.E + 1, mt) - 1;
+    const int lm = mt - p.tile_offsets[e];
+    ti.e = e;
+    ti.b_row0 = e * p.N + nt * BN;
+    const int cnt = p.counts[e];
+    ti.rows_valid = min(BM, cnt - lm * BM);
+    ti.out_row0 = p.offsets[e] + lm * BM;
+  } else {
+    ti.e = 0;
+    ti.b_row0 = nt * BN;
+    ti.rows_valid = min(BM, p.M - mt * BM);
+    ti.out_row0 = mt * BM;
+  }
+  return ti;
+}
+
+__device__ __forceinline__ float silu_f32(float z) {
+  return __fdiv_rn(z, __fadd_rn(1.0f, expf(-z)));
+}
+
+template <int BN, int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const Params p) {
+  using C = Cfg<BN>;
+  constexpr bool kGrouped = (EPI == EPI_W13 || EPI == EPI_W2);
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *smA = smem;
+  uint8_t *smB = smA + C::kStages * C::A_BYTES;
+  uint8_t *smSFA = smB + C::kStages * C::B_BYTES;
+  uint8_t *smSFB = smSFA + C::kStages * C::SFA_BYTES;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smSFB + C::kStages * C::SFB_BYTES);
+  uint64_t *full = bars;
+  uint64_t *empty = bars + C::kStages;
+  uint64_t *acc_full = bars + 2 * C::kStages;
+  uint64_t *acc_empty = acc_full + 1;
+  uint64_t *drain = acc_full + 2;
+  __shared__ uint32_t s_tmem_base;
+  __shared__ volatile int s_abort;
+  __shared__ int s_total;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 4);
+    mbar_init(drain, 1);
+    fence_barrier_init();
+    s_abort = 0;
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+    s_total = kGrouped ? p.tile_offsets[p.E] * p.n_tiles : p.m_tiles * p.n_tiles;
+  }
+  if (warp == 1) {
+    tmem_alloc(&s_tmem_base, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem_base;
+  const int total = s_total;
+  const uint64_t lim = p.wait_limit;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued[C::kStages];
+      uint32_t issued_par[C::kStages];
+      for (int s = 0; s < C::kStages; ++s) issued[s] = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < total; t += gridDim.x) {
+        const TileInfo ti = tile_info<BN, kGrouped>(p, t);
+        const int b_slab0 = ti.b_row0 / 128;
+        for (int kt = 0; kt < p.k_stages; ++kt) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, &s_abort, p.status, lim)) { ok = false; break; }
+          const int nk = min(4, p.kw - kt * 4);
+          const uint32_t sf_bytes = (uint32_t)nk * 512u;
+          int halves = 0;
+          for (int h = 0; h < C::HALVES; ++h)
+            if ((int64_t)(b_slab0 + h) * 128 < p.b_sf_rows) ++halves;
+          const uint32_t bytes = C::A_BYTES + C::B_BYTES + sf_bytes * (1 + halves);
+          mbar_arrive_expect_tx(&full[stage], bytes);
+          tma_load_2d(smA + stage * C::A_BYTES, &tmA, &full[stage], kt * BK_BYTES, ti.a_row0);
+          tma_load_2d(smB + stage * C::B_BYTES, &tmB, &full[stage], kt * BK_BYTES, ti.b_row0);
+          bulk_load(smSFA + stage * C::SFA_BYTES, p.a_sf + ((int64_t)ti.a_slab * p.kw + kt * 4) * 512, sf_bytes,
+                    &full[stage]);
+          for (int h = 0; h < halves; ++h)
+            bulk_load(smSFB + stage * C::SFB_BYTES + h * 4 * 512,
+                      p.b_sf + ((int64_t)(b_slab0 + h) * p.kw + kt * 4) * 512, sf_bytes, &full[stage]);
+          issued[stage] = 1;
+          issued_par[stage] = phase;
+          if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {  // let copies already in flight land before the CTA exits
+        for (int s = 0; s < C::kStages; ++s)
+          if (issued[s]) mbar_drain(&full[s], issued_par[s], 1000000000ull);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_mxf4nvf4(BM, BN);
+      int stage = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true, any_mma = false;
+      const uint32_t t_acc = tmem + C::ACC_COL;
+      const uint32_t t_sfa = tmem + C::SFA_COL;
+      const uint32_t t_sfb = tmem + C::SFB_COL;
+      for (int t = blockIdx.x; ok && t < total; t += gridDim.x) {
+        if (!mbar_wait(acc_empty, acc_phase ^ 1u, &s_abort, p.status, lim)) { ok = false; break; }
+        tc_fence_after();
+        for (int kt = 0; kt < p.k_stages; ++kt) {
+          if (!mbar_wait(&full[stage], phase, &s_abort, p.status, lim)) { ok = false; break; }
+          tc_fence_after();
+          const int nk = min(4, p.kw - kt * 4);
+          const uint32_t a_base = smem_u32(smA + stage * C::A_BYTES);
+          const uint32_t b_base = smem_u32(smB + stage * C::B_BYTES);
+          const uint32_t sfa_base = smem_u32(smSFA + stage * C::SFA_BYTES);
+          const uint32_t sfb_base = smem_u32(smSFB + stage * C::SFB_BYTES);
+          for (int j = 0; j < nk; ++j) {
+            tmem_cp_sf(t_sfa + j * 4, smem_desc(sfa_base + j * 512, 0, 128, 0));
+#pragma unroll
+            for (int h = 0; h < C::HALVES; ++h)
+              tmem_cp_sf(t_sfb + j * 4 * C::HALVES + h * 4, smem_desc(sfb_base + (h * 4 + j) * 512, 0, 128, 0));
+          }
+          for (int j = 0; j < nk; ++j) {
+            const uint64_t ad = smem_desc(a_base + j * 32, 16, 1024, 2);
+            const uint64_t bd = smem_desc(b_base + j * 32, 16, 1024, 2);
+            mma_nvf4(t_acc, ad, bd, idesc, t_sfa + j * 4, t_sfb + j * 4 * C::HALVES, (kt > 0 || j > 0) ? 1u : 0u);
+          }
+          any_mma = true;
+          tc_commit(&empty[stage]);
+          if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit(acc_full);
+        acc_phase ^= 1u;
+      }
+      if (!ok && any_mma) {  // wait for issued MMAs / copies before freeing TMEM
+        tc_commit(drain);
+        mbar_drain(drain, 0, 1000000000ull);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int row = q * 32 + lane;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+      const TileInfo ti = tile_info<BN, kGrouped>(p, t);
+      if (!mbar_wait(acc_full, acc_phase, &s_abort, p.status, lim)) break;
+      tc_fence_after();
+      const bool row_ok = row < ti.rows_valid;
+      float alpha;
+      if (EPI == EPI_F32 || EPI == EPI_BF16) alpha = __fmul_rn(*p.a_g, *p.b_g);
+      else if (EPI == EPI_W13) alpha = __fmul_rn(*p.a_g, p.w_g[ti.e]);
+      else alpha = __fmul_rn(p.h_g[ti.e], p.w_g[ti.e]);
+      float wrow = 1.0f;
+      if (EPI == EPI_W2 && row_ok && p.topk_w) wrow = p.topk_w[p.perm[ti.out_row0 + row]];
+      const float scale = (EPI == EPI_W2) ? __fmul_rn(alpha, wrow) : alpha;
+      float hg = 0.f;
+      if (EPI == EPI_W13) hg = p.h_g[ti.e];
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        float v[32];
+        __syncwarp();
+        tmem_ld32(tmem + C::ACC_COL + ((uint32_t)(q * 32) << 16) + c * 32, v);
+        const int col0 = ti.n0 + c * 32;
+        if (!row_ok || col0 >= p.N) {
+          // nothing to store for this row / column block
+        } else if (EPI == EPI_F32) {
+          float *dst = static_cast<float *>(p.c) + (int64_t)(ti.out_row0 + row) * p.N + col0;
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            if (col0 + i < p.N)
+              *reinterpret_cast<float4 *>(dst + i) =
+                  make_float4(__fmul_rn(v[i], scale), __fmul_rn(v[i + 1], scale), __fmul_rn(v[i + 2], scale),
+                              __fmul_rn(v[i + 3], scale));
+          }
+        } else if (EPI == EPI_BF16) {
+          __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.c) + (int64_t)(ti.out_row0 + row) * p.N + col0;
+#pragma unroll
+          for (int i = 0; i < 32; i += 8) {
+            if (col0 + i < p.N) {
+              __nv_bfloat162 b[4];
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                b[j] = __floats2bfloat162_rn(__fmul_rn(v[i + 2 * j], scale), __fmul_rn(v[i + 2 * j + 1], scale));
+              *reinterpret_cast<uint4 *>(dst + i) = *reinterpret_cast<uint4 *>(b);
+            }
+          }
+        } else if (EPI == EPI_W13) {
+          // columns col0..col0+15 are gate, col0+16..col0+31 are up, for
+          // intermediate columns hc..hc+15 with hc = col0 / 2
+          float h[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float gte = __fmul_rn(v[i], scale);
+            const float up = __fmul_rn(v[16 + i], scale);
+            h[i] = __fmul_rn(silu_f32(gte), up);
+          }
+          const int hc = col0 / 2;
+          const int64_t prow = (int64_t)ti.a_row0 + row;  // padded row
+          uint32_t lo, hi;
+          const uint32_t sf = nvfp4_block16(h, hg, &lo, &hi);
+          *reinterpret_cast<uint2 *>(p.h_codes + prow * (p.I / 2) + hc / 2) = make_uint2(lo, hi);
+          p.h_sf[sf_tiled_offset(prow, hc / 16, p.I / 64)] = (uint8_t)sf;
+          if (p.h_dump) {
+            float4 *d = reinterpret_cast<float4 *>(p.h_dump + prow * p.I + hc);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) d[i] = make_float4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
+          }
+        } else {  // EPI_W2
+          float *dst = p.y + (int64_t)(ti.out_row0 + row) * p.N + col0;
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4 *>(dst + i) =
+                make_float4(__fmul_rn(v[i], scale), __fmul_rn(v[i + 1], scale), __fmul_rn(v[i + 2], scale),
+                            __fmul_rn(v[i + 3], scale));
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
+      acc_phase ^= 1u;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// Packed-code matrix [rows][row_bytes] as a 2-D uint8 tensor map with a
+// 128-byte x box_rows box and 128-byte swizzle (zero fill out of bounds).
+bool make_code_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t row_bytes, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {row_bytes, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms;
+}
+
+template <int BN, int EPI>
+fp4_status launch(const CUtensorMap &ta, const CUtensorMap &tb, const Params &p, int grid, cudaStream_t s) {
+  using C = Cfg<BN>;
+  auto kern = fp4_gemm_kernel<BN, EPI>;
+  FP4_HOST_CHECK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
+  kern<<<grid, kThreads, C::SMEM_BYTES, s>>>(ta, tb, p);
+  FP4_HOST_CHECK(cudaGetLastError());
+  return FP4_OK;
+}
+
+bool al16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr int kBN = 256;
+
+}  // namespace
+}  // namespace fp4
+
+using namespace fp4;
+
+extern "C" {
+
+fp4_status fp4_gemm(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_g, const uint8_t *b_codes,
+                    const uint8_t *b_sf, const float *b_g, void *c, fp4_out_dtype c_dtype, int64_t M, int64_t N,
+                    int64_t K, uint32_t flags, fp4_stream_t stream) {
+  (void)flags;
+  if (!a_codes || !a_sf || !a_g || !b_codes || !b_sf || !b_g || !c) return FP4_ERR_INVALID_ARG;
+  if (c_dtype != FP4_OUT_F32 && c_dtype != FP4_OUT_BF16) return FP4_ERR_INVALID_ARG;
+  if (M < 1 || N < 1 || K < 64 || K % 64 || N % 8) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (M > (1LL << 30) || N > (1LL << 30) || K > (1LL << 30)) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (!al16(a_codes) || !al16(b_codes) || !al16(a_sf) || !al16(b_sf) || !al16(c)) return FP4_ERR_ALIGNMENT;
+  const DeviceCtx *ctx = device_ctx();
+  if (!ctx) return FP4_ERR_CUDA;
+  CUtensorMap ta, tb;
+  if (!make_code_map(&ta, a_codes, (uint64_t)M, (uint64_t)K / 2, BM)) return FP4_ERR_CUDA;
+  if (!make_code_map(&tb, b_codes, (uint64_t)N, (uint64_t)K / 2, kBN)) return FP4_ERR_CUDA;
+  Params p = {};
+  p.M = (int)M; p.N = (int)N; p.K = (int)K;
+  p.n_tiles = (int)((N + kBN - 1) / kBN);
+  p.m_tiles = (int)((M + BM - 1) / BM);
+  p.k_stages = (int)((K + 255) / 256);
+  p.kw = (int)(K / 64);
+  p.a_sf = a_sf; p.b_sf = b_sf;
+  p.b_sf_rows = ((N + 127) / 128) * 128;
+  p.a_g = a_g; p.b_g = b_g; p.c = c;
+  p.status = ctx->status;
+  p.wait_limit = ctx->wait_limit_ns;
+  const int64_t tiles = (int64_t)p.m_tiles * p.n_tiles;
+  if (tiles > 2147483647LL) return FP4_ERR_UNSUPPORTED_SHAPE;
+  const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (c_dtype == FP4_OUT_F32) return launch<kBN, EPI_F32>(ta, tb, p, grid, s);
+  return launch<kBN, EPI_BF16>(ta, tb, p, grid, s);
+}
+
+fp4_status fp4_moe_w13(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_g, const fp4_moe_weights *w,
+                       int64_t H, int64_t I, int32_t E, const int32_t *counts, const int32_t *tile_offsets,
+                       int64_t rows_cap, uint8_t *h_codes, uint8_t *h_sf, uint32_t flags, float *h_dump,
+                       fp4_stream_t stream) {
+  if (!a_codes || !a_sf || !a_g || !w || !w->w13_codes || !w->w13_sf || !w->w13_g || !w->h_g || !counts ||
+      !tile_offsets || !h_codes || !h_sf)
+    return FP4_ERR_INVALID_ARG;
+  if ((flags & FP4_DEBUG_DUMP_H) && !h_dump) return FP4_ERR_INVALID_ARG;
+  if (H < 256 || H % 256 || I < 256 || I % 256 || E < 1 || E > 4096 || rows_cap < 1) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if ((int64_t)E * 2 * I > (1LL << 31) - 1 || rows_cap > (1LL << 31) - 1) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (!al16(a_codes) || !al16(a_sf) || !al16(w->w13_codes) || !al16(w->w13_sf) || !al16(h_codes) || !al16(h_sf) ||
+      (h_dump && !al16(h_dump)))
+    return FP4_ERR_ALIGNMENT;
+  const DeviceCtx *ctx = device_ctx();
+  if (!ctx) return FP4_ERR_CUDA;
+  CUtensorMap ta, tb;
+  if (!make_code_map(&ta, a_codes, (uint64_t)rows_cap, (uint64_t)H / 2, BM)) return FP4_ERR_CUDA;
+  if (!make_code_map(&tb, w->w13_codes, (uint64_t)E * 2 * I, (uint64_t)H / 2, kBN)) return FP4_ERR_CUDA;
+  Params p = {};
+  p.N = (int)(2 * I); p.K = (int)H;
+  p.n_tiles = (int)(2 * I / kBN);
+  p.k_stages = (int)(H / 256);
+  p.kw = (int)(H / 64);
+  p.a_sf = a_sf; p.b_sf = w->w13_sf;
+  p.b_sf_rows = (int64_t)E * 2 * I;
+  p.a_g = a_g;
+  p.E = E; p.counts = counts; p.tile_offsets = tile_offsets;
+  p.w_g = w->w13_g; p.h_g = w->h_g;
+  p.h_codes = h_codes; p.h_sf = h_sf; p.I = (int)I;
+  p.h_dump = (flags & FP4_DEBUG_DUMP_H) ? h_dump : nullptr;
+  p.status = ctx->status;
+  p.wait_limit = ctx->wait_limit_ns;
+  return launch<kBN, EPI_W13>(ta, tb, p, sm_count(), reinterpret_cast<cudaStream_t>(stream));
+}
+
+fp4_status fp4_moe_w2(const uint8_t *h_codes, const uint8_t *h_sf, const fp4_moe_weights *w, int64_t H, int64_t I,
+                      int32_t E, const int32_t *counts, const int32_t *offsets, const int32_t *tile_offsets,
+                      const int32_t *perm, const float *topk_weights, int64_t rows_cap, float *y,
+                      fp4_stream_t stream) {
+  if (!h_codes || !h_sf || !w || !w->w2_codes || !w->w2_sf || !w->w2_g || !w->h_g || !counts || !offsets ||
+      !tile_offsets || !perm || !y)
+    return FP4_ERR_INVALID_ARG;
+  if (H < 256 || H % 256 || I < 256 || I % 256 || E < 1 || E > 4096 || rows_cap < 1) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if ((int64_t)E * H > (1LL << 31) - 1 || rows_cap > (1LL << 31) - 1) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (!al16(h_codes) || !al16(h_sf) || !al16(w->w2_codes) || !al16(w->w2_sf) || !al16(y)) return FP4_ERR_ALIGNMENT;
+  const DeviceCtx *ctx = device_ctx();
+  if (!ctx) return FP4_ERR_CUDA;
+  CUtensorMap ta, tb;
+  if (!make_code_map(&ta, h_codes, (uint64_t)rows_cap, (uint64_t)I / 2, BM)) return FP4_ERR_CUDA;
+  if (!make_code_map(&tb, w->w2_codes, (uint64_t)E * H, (uint64_t)I / 2, kBN)) return FP4_ERR_CUDA;
+  Params p = {};
+  p.N = (int)H; p.K = (int)I;
+  p.n_tiles = (int)(H / kBN);
+  p.k_stages = (int)(I / 256);
+  p.kw = (int)(I / 64);
+  p.a_sf = h_sf; p.b_sf = w->w2_sf;
+  p.b_sf_rows = (int64_t)E * H;
+  p.E = E; p.counts = counts; p.offsets = offsets; p.tile_offsets = tile_offsets;
+  p.w_g = w->w2_g; p.h_g = w->h_g;
+  p.perm = perm; p.topk_w = topk_weights; p.y = y;
+  p.status = ctx->status;
+  p.wait_limit = ctx->wait_limit_ns;
+  return launch<kBN, EPI_W2>(ta, tb, p, sm_count(), reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,92 @@
+// The routed-expert MoE layer as one call: quantize x -> route -> gather ->
+// grouped w13 (+SwiGLU +NVFP4 re-quantize) -> grouped w2 -> combine.
+//
+// "DeepSeek-V4 FP4 QAT", §3.1 (tokens go to their top-k experts; outputs are
+// summed), "DeepSeek-V4 architecture", §5.1 (SwiGLU feed-forward experts),
+// "DeepSeek-V4.1-Flash-NVFP4", §一 point 3 and §三 (W4A4 routed experts:
+// w1/w3/w2 and their activations all in NVFP4).  Every stage is one of the
+// library's own kernels on the caller's stream; the caller's workspace holds
+// every intermediate.
+#include "common.cuh"
+
+namespace {
+
+struct MoeLayout {
+  size_t header, x_codes, x_sf, counts, offsets, tile_offsets, perm, inv, scratch, a_codes, a_sf, h_codes, h_sf, y;
+  size_t total;
+  int64_t rows_cap;
+};
+
+size_t up256(size_t v) { return (v + 255) & ~size_t(255); }
+
+MoeLayout moe_layout(int64_t T, int32_t topk, int64_t H, int64_t I, int32_t E) {
+  MoeLayout L;
+  const int64_t R = T * topk;
+  L.rows_cap = ((R + 127LL * E + 127) / 128) * 128;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t at = off;
+    off += up256(bytes);
+    return at;
+  };
+  L.header = take(512);  // [0,256) quantize workspace, [256,260) g_x
+  L.x_codes = take((size_t)(T * H / 2));
+  L.x_sf = take((size_t)(T * H / 16));
+  L.counts = take((size_t)E * 4);
+  L.offsets = take((size_t)(E + 1) * 4);
+  L.tile_offsets = take((size_t)(E + 1) * 4);
+  L.perm = take((size_t)R * 4);
+  L.inv = take((size_t)R * 4);
+  L.scratch = take(fp4_moe_route_scratch_bytes(R, E));
+  L.a_codes = take((size_t)(L.rows_cap * H / 2));
+  L.a_sf = take(fp4_sf_tiled_bytes(L.rows_cap, H));
+  L.h_codes = take((size_t)(L.rows_cap * I / 2));
+  L.h_sf = take(fp4_sf_tiled_bytes(L.rows_cap, I));
+  L.y = take((size_t)R * (size_t)H * 4);
+  L.total = off;
+  return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t fp4_moe_workspace_size(int64_t T, int32_t topk, int64_t H, int64_t I, int32_t E) {
+  if (T < 0 || topk < 1 || H <= 0 || I <= 0 || E < 1) return 0;
+  return moe_layout(T, topk, H, I, E).total;
+}
+
+fp4_status fp4_moe_grouped_gemm(const void *tokens_bf16, const int32_t *expert_ids, const float *topk_weights,
+                                int64_t T, int32_t topk, const fp4_moe_weights *w, int64_t H, int64_t I, int32_t E,
+                                void *out_bf16, void *workspace, size_t ws_bytes, uint32_t flags, float *h_dump,
+                                fp4_stream_t stream) {
+  if (!tokens_bf16 || !expert_ids || !w || !out_bf16 || !workspace) return FP4_ERR_INVALID_ARG;
+  if (T < 0 || topk < 1 || topk > 16 || E < 1 || E > 4096) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (H < 256 || H % 256 || I < 256 || I % 256) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return FP4_ERR_ALIGNMENT;
+  const MoeLayout L = moe_layout(T, topk, H, I, E);
+  if (ws_bytes < L.total) return FP4_ERR_WORKSPACE;
+  if ((flags & FP4_DEBUG_DUMP_H) && !h_dump) return FP4_ERR_INVALID_ARG;
+  if (T == 0) return FP4_OK;
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  float *g_x = reinterpret_cast<float *>(ws + L.header + 256);
+  auto I32 = [&](size_t off) { return reinterpret_cast<int32_t *>(ws + off); };
+  fp4_status st;
+  st = fp4_quantize(FP4_NV, tokens_bf16, T, H, H, ws + L.x_codes, ws + L.x_sf, g_x, 0, ws + L.header, 256, stream);
+  if (st != FP4_OK) return st;
+  st = fp4_moe_route(expert_ids, T, topk, E, I32(L.counts), I32(L.offsets), I32(L.tile_offsets), I32(L.perm),
+                     I32(L.inv), ws + L.scratch, fp4_moe_route_scratch_bytes(T * topk, E), stream);
+  if (st != FP4_OK) return st;
+  st = fp4_moe_gather(ws + L.x_codes, ws + L.x_sf, T, topk, H, E, I32(L.offsets), I32(L.tile_offsets), I32(L.perm),
+                      ws + L.a_codes, ws + L.a_sf, L.rows_cap, stream);
+  if (st != FP4_OK) return st;
+  st = fp4_moe_w13(ws + L.a_codes, ws + L.a_sf, g_x, w, H, I, E, I32(L.counts), I32(L.tile_offsets), L.rows_cap,
+                   ws + L.h_codes, ws + L.h_sf, flags & FP4_DEBUG_DUMP_H, h_dump, stream);
+  if (st != FP4_OK) return st;
+  st = fp4_moe_w2(ws + L.h_codes, ws + L.h_sf, w, H, I, E, I32(L.counts), I32(L.offsets), I32(L.tile_offsets),
+                  I32(L.perm), topk_weights, L.rows_cap, reinterpret_cast<float *>(ws + L.y), stream);
+  if (st != FP4_OK) return st;
+  return fp4_moe_combine(reinterpret_cast<const float *>(ws + L.y), I32(L.inv), T, topk, H, out_bf16, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,278 @@
+// NVFP4 / MXFP4 quantizers and the MXFP4 -> NVFP4 scale remap.
+//
+// "DeepSeek-V4.1-Flash-NVFP4", §二: E2M1 elements (0, 0.5, 1, 1.5, 2, 3, 4, 6
+// with a sign), two per byte; NVFP4 = one block scale per 16 elements that
+// brings the block into [-6, 6], under a tensor-level scale.  §三: MXFP4 =
+// one UE8M0 scale per 32 elements.  §一 point 2 and §六: the MX scales
+// re-expressed as NVFP4 scales without changing any dequantized value.
+//
+// Kernels are HBM-bound: 16-byte vector loads and stores, one thread per
+// scale block, grid sized to a multiple of the SM count.
+#include "common.cuh"
+
+namespace fp4 {
+namespace {
+
+constexpr int kThreads = 256;
+
+int grid_for(int64_t work_items, int per_cta = kThreads) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int64_t need = (work_items + per_cta - 1) / per_cta;
+  int64_t cap = (int64_t)sms * 8;  // 8 resident CTAs of 256 threads per SM
+  return (int)(need < cap ? (need < 1 ? 1 : need) : cap);
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---- pass 1 of dynamic NVFP4: tensor amax ---------------------------------
+// |x| of a bf16 is its bit pattern with the sign cleared; for non-negative
+// values the integer order of the patterns is the numeric order, so the max
+// is an integer max.  The result is stored as fp32 bits (bf16 << 16).
+__global__ void __launch_bounds__(kThreads) amax_bf16_kernel(const uint16_t *__restrict__ x, int64_t rows,
+                                                             int64_t cols, int64_t ld,
+                                                             unsigned int *__restrict__ amax_bits) {
+  const int64_t vec_per_row = cols / 8;
+  const int64_t total = rows * vec_per_row;
+  uint32_t m = 0;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = i / vec_per_row, c = (i - r * vec_per_row) * 8;
+    const uint4 v = __ldcs(reinterpret_cast<const uint4 *>(x + r * ld + c));
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      m = max(m, w[j] & 0x7FFFu);
+      m = max(m, (w[j] >> 16) & 0x7FFFu);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+  __shared__ uint32_t red[kThreads / 32];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    m = threadIdx.x < kThreads / 32 ? red[threadIdx.x] : 0u;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (threadIdx.x == 0 && m) atomicMax(amax_bits, m << 16);
+  }
+}
+
+// ---- NVFP4 quantize: one thread per 16-element block -----------------------
+template <bool kTiled>
+__global__ void __launch_bounds__(kThreads) nvfp4_quantize_kernel(
+    const uint16_t *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, uint8_t *__restrict__ codes,
+    uint8_t *__restrict__ scales, const unsigned int *__restrict__ amax_bits, float *__restrict__ g_out,
+    const float *__restrict__ g_in) {
+  float g;
+  if (g_in) {
+    g = *g_in;
+  } else {
+    g = __fdiv_rn(__uint_as_float(*amax_bits), 2688.0f);  // amax / (448 * 6)
+    if (blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
+  }
+  const int64_t nb = cols / 16;
+  const int64_t total = rows * nb;
+  const int64_t n_ksteps = cols / 64;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = i / nb, b = i - r * nb;
+    const uint4 *src = reinterpret_cast<const uint4 *>(x + r * ld + b * 16);
+    const uint4 v0 = __ldcs(src), v1 = __ldcs(src + 1);
+    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    float f[16];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      f[2 * j] = bf16_bits_to_f32(w[j] & 0xFFFFu);
+      f[2 * j + 1] = bf16_bits_to_f32(w[j] >> 16);
+    }
+    uint32_t lo, hi;
+    const uint32_t sf = nvfp4_block16(f, g, &lo, &hi);
+    *reinterpret_cast<uint2 *>(codes + r * (cols / 2) + b * 8) = make_uint2(lo, hi);
+    if (kTiled)
+      scales[sf_tiled_offset(r, b, n_ksteps)] = (uint8_t)sf;
+    else
+      scales[i] = (uint8_t)sf;
+  }
+}
+
+// ---- MXFP4 quantize: one thread per 32-element block -----------------------
+__global__ void __launch_bounds__(kThreads) mxfp4_quantize_kernel(const uint16_t *__restrict__ x, int64_t rows,
+                                                                  int64_t cols, int64_t ld,
+                                                                  uint8_t *__restrict__ codes,
+                                                                  uint8_t *__restrict__ scales) {
+  const int64_t nb = cols / 32;
+  const int64_t total = rows * nb;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = i / nb, b = i - r * nb;
+    const uint4 *src = reinterpret_cast<const uint4 *>(x + r * ld + b * 32);
+    uint32_t w[16];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint4 v = __ldcs(src + q);
+      w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
+    }
+    uint32_t amax = 0;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) amax = max(amax, max(w[j] & 0x7FFFu, (w[j] >> 16) & 0x7FFFu));
+    // floor(log2 amax) from the bf16 pattern: exponent field, or for a
+    // subnormal (m * 2^-133) the index of m's top bit.
+    int X = 0;
+    uint32_t scale = 0;
+    if (amax) {
+      const int e = (int)(amax >> 7);
+      const int fl = e ? e - 127 : (31 - __clz((int)(amax & 0x7Fu))) - 133;
+      X = min(max(fl - 2, -127), 127);
+      scale = (uint32_t)(X + 127);
+    }
+    const float p = __uint_as_float((uint32_t)(127 - X) << 23);  // 2^-X, X in [-127, 126]
+    float f[32];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      f[2 * j] = __fmul_rn(bf16_bits_to_f32(w[j] & 0xFFFFu), p);
+      f[2 * j + 1] = __fmul_rn(bf16_bits_to_f32(w[j] >> 16), p);
+    }
+    const uint4 out = make_uint4(pack8_e2m1(f), pack8_e2m1(f + 8), pack8_e2m1(f + 16), pack8_e2m1(f + 24));
+    *reinterpret_cast<uint4 *>(codes + r * (cols / 2) + b * 16) = out;
+    scales[i] = (uint8_t)scale;
+  }
+}
+
+// ---- MXFP4 -> NVFP4 remap: one CTA per tensor ------------------------------
+// A block is live if any of its 32 codes has a nonzero magnitude (bits 0-2).
+__device__ __forceinline__ bool block_live(const uint4 c) {
+  const uint32_t m = 0x77777777u;
+  return ((c.x | c.y | c.z | c.w) & m) != 0;
+}
+
+__device__ __forceinline__ float pow2_f32(int e) {  // exact 2^e, e in [-149, 127]
+  if (e >= -126) return __uint_as_float((uint32_t)(e + 127) << 23);
+  return __uint_as_float(1u << (e + 149));
+}
+
+__global__ void __launch_bounds__(kThreads) mx_to_nv_kernel(const uint8_t *__restrict__ codes,
+                                                            const uint8_t *__restrict__ mx, int64_t rows,
+                                                            int64_t cols, uint8_t *__restrict__ nv,
+                                                            float *__restrict__ nv_global) {
+  const int64_t t = blockIdx.x;
+  const int64_t nb = rows * (cols / 32);
+  const uint8_t *cb = codes + t * rows * (cols / 2);
+  const uint8_t *sb = mx + t * nb;
+  uint8_t *ob = nv + t * rows * (cols / 16);
+  int emax = -1000, emin = 1000, bad = 0;
+  for (int64_t i = threadIdx.x; i < nb; i += blockDim.x) {
+    const uint4 c = *reinterpret_cast<const uint4 *>(cb + i * 16);
+    if (block_live(c)) {
+      const int s = sb[i];
+      if (s == 255) bad = 1;
+      emax = max(emax, s - 127);
+      emin = min(emin, s - 127);
+    }
+  }
+  __shared__ int s_max[kThreads], s_min[kThreads], s_bad[kThreads];
+  s_max[threadIdx.x] = emax;
+  s_min[threadIdx.x] = emin;
+  s_bad[threadIdx.x] = bad;
+  __syncthreads();
+  for (int o = kThreads / 2; o > 0; o >>= 1) {
+    if (threadIdx.x < o) {
+      s_max[threadIdx.x] = max(s_max[threadIdx.x], s_max[threadIdx.x + o]);
+      s_min[threadIdx.x] = min(s_min[threadIdx.x], s_min[threadIdx.x + o]);
+      s_bad[threadIdx.x] |= s_bad[threadIdx.x + o];
+    }
+    __syncthreads();
+  }
+  emax = s_max[0];
+  emin = s_min[0];
+  bad = s_bad[0];
+  const bool any_live = emax > -1000;
+  if (bad || (any_live && emax - emin > 17)) {
+    if (threadIdx.x == 0) nv_global[t] = __uint_as_float(0x7FC00000u);  // NaN marks a refused tensor
+    return;
+  }
+  if (threadIdx.x == 0) nv_global[t] = any_live ? pow2_f32(emax - 8) : 0.0f;
+  for (int64_t i = threadIdx.x; i < nb; i += blockDim.x) {
+    const uint4 c = *reinterpret_cast<const uint4 *>(cb + i * 16);
+    uint32_t code = 0;
+    if (block_live(c)) {
+      const int k = ((int)sb[i] - 127) - emax + 8;  // in [-9, 8]
+      code = k >= -6 ? (uint32_t)((k + 7) << 3) : (1u << (k + 9));
+    }
+    *reinterpret_cast<uint16_t *>(ob + 2 * i) = (uint16_t)(code | (code << 8));
+  }
+}
+
+}  // namespace
+}  // namespace fp4
+
+using namespace fp4;
+
+extern "C" {
+
+fp4_status fp4_quantize(fp4_format fmt, const void *x_bf16, int64_t rows, int64_t cols, int64_t ld, uint8_t *codes,
+                        uint8_t *scales, float *global_scale, uint32_t flags, void *workspace, size_t ws_bytes,
+                        fp4_stream_t stream) {
+  if (!x_bf16 || !codes || !scales || rows < 0 || cols <= 0 || ld < cols) return FP4_ERR_INVALID_ARG;
+  if (fmt != FP4_NV && fmt != FP4_MX) return FP4_ERR_INVALID_ARG;
+  if (!aligned16(x_bf16) || !aligned16(codes) || (ld * 2) % 16) return FP4_ERR_ALIGNMENT;
+  const DeviceCtx *ctx = device_ctx();
+  if (!ctx) return FP4_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (rows == 0) return FP4_OK;
+  const uint16_t *x = static_cast<const uint16_t *>(x_bf16);
+  if (fmt == FP4_MX) {
+    if (cols % 32) return FP4_ERR_UNSUPPORTED_SHAPE;
+    mxfp4_quantize_kernel<<<grid_for(rows * (cols / 32)), kThreads, 0, s>>>(x, rows, cols, ld, codes, scales);
+    FP4_HOST_CHECK(cudaGetLastError());
+    return FP4_OK;
+  }
+  const bool tiled = flags & FP4_SCALE_LAYOUT_TILED;
+  if (cols % 16 || (tiled && cols % 64)) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (!global_scale) return FP4_ERR_INVALID_ARG;
+  const bool stat = flags & FP4_STATIC_GLOBAL_SCALE;
+  unsigned int *amax = nullptr;
+  if (!stat) {
+    if (!workspace) return FP4_ERR_INVALID_ARG;
+    if (ws_bytes < fp4_quantize_workspace_size()) return FP4_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return FP4_ERR_ALIGNMENT;
+    amax = static_cast<unsigned int *>(workspace);
+    FP4_HOST_CHECK(cudaMemsetAsync(amax, 0, sizeof(unsigned int), s));
+    amax_bf16_kernel<<<grid_for(rows * (cols / 8)), kThreads, 0, s>>>(x, rows, cols, ld, amax);
+    FP4_HOST_CHECK(cudaGetLastError());
+  }
+  const int grid = grid_for(rows * (cols / 16));
+  const float *g_in = stat ? global_scale : nullptr;
+  if (tiled)
+    nvfp4_quantize_kernel<true><<<grid, kThreads, 0, s>>>(x, rows, cols, ld, codes, scales, amax, global_scale, g_in);
+  else
+    nvfp4_quantize_kernel<false><<<grid, kThreads, 0, s>>>(x, rows, cols, ld, codes, scales, amax, global_scale, g_in);
+  FP4_HOST_CHECK(cudaGetLastError());
+  return FP4_OK;
+}
+
+fp4_status fp4_mx_to_nv(const uint8_t *codes, const uint8_t *mx_scales, int64_t rows, int64_t cols,
+                        int64_t num_tensors, uint8_t *nv_scales, float *nv_global, uint32_t flags,
+                        fp4_stream_t stream) {
+  (void)flags;
+  if (!codes || !mx_scales || !nv_scales || !nv_global || rows <= 0 || cols <= 0 || num_tensors <= 0)
+    return FP4_ERR_INVALID_ARG;
+  if (cols % 32) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(codes) || (reinterpret_cast<uintptr_t>(nv_scales) & 1u)) return FP4_ERR_ALIGNMENT;
+  if (num_tensors > 2147483647) return FP4_ERR_UNSUPPORTED_SHAPE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  mx_to_nv_kernel<<<(unsigned)num_tensors, kThreads, 0, s>>>(codes, mx_scales, rows, cols, nv_scales, nv_global);
+  FP4_HOST_CHECK(cudaGetLastError());
+  // offline step: report refused tensors (NaN globals) synchronously
+  FP4_HOST_CHECK(cudaStreamSynchronize(s));
+  fp4_status st = FP4_OK;
+  float host[256];
+  for (int64_t i0 = 0; i0 < num_tensors; i0 += 256) {
+    const int64_t n = num_tensors - i0 < 256 ? num_tensors - i0 : 256;
+    FP4_HOST_CHECK(cudaMemcpy(host, nv_global + i0, sizeof(float) * (size_t)n, cudaMemcpyDeviceToHost));
+    for (int64_t i = 0; i < n; ++i)
+      if (host[i] != host[i]) st = FP4_ERR_RANGE;
+  }
+  return st;
+}
+
+}  // extern "C"

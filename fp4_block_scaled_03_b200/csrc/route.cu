@@ -1,0 +1,274 @@
+// Routing permute, gather into expert tiles, and the fixed-order combine.
+//
+// "DeepSeek-V4 FP4 QAT", §3.1 (each token is sent to its top-k experts and
+// the expert outputs are summed) and "DeepSeek-V4 architecture", §2.1 (384
+// routed experts, 6 active per token).  Routed rows are put in (expert,
+// token, slot) order -- a stable counting sort of the flattened expert ids --
+// so each expert's rows are contiguous; each expert's block of rows is padded
+// to a multiple of 128 (the GEMM's M tile).
+#include "common.cuh"
+
+namespace fp4 {
+namespace {
+
+constexpr int kChunk = 1024;  // flat slots per routing chunk (one warp each)
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+// Pass 1: per-chunk histogram (one warp per chunk, in slot order).
+__global__ void route_count_kernel(const int32_t *__restrict__ ids, int64_t R, int32_t E,
+                                   int32_t *__restrict__ chunk_counts, unsigned int *__restrict__ status) {
+  extern __shared__ int32_t cnt[];  // [E]
+  const int lane = threadIdx.x;
+  for (int e = lane; e < E; e += 32) cnt[e] = 0;
+  __syncwarp();
+  const int64_t base = (int64_t)blockIdx.x * kChunk;
+  for (int step = 0; step < kChunk / 32; ++step) {
+    const int64_t f = base + step * 32 + lane;
+    int id = -1;
+    if (f < R) {
+      id = ids[f];
+      if (id < 0 || id >= E) {
+        record_status(status, FP4_ERR_BAD_EXPERT);
+        id = -1;
+      }
+    }
+    const uint32_t grp = __match_any_sync(0xffffffffu, id);
+    if (id >= 0 && (grp & lanemask_lt()) == 0) cnt[id] += __popc(grp);  // group leader
+    __syncwarp();
+  }
+  for (int e = lane; e < E; e += 32) chunk_counts[(int64_t)blockIdx.x * E + e] = cnt[e];
+}
+
+// Pass 2 (one CTA): per-expert totals, exclusive prefixes over experts (rows
+// and 128-row tiles), and each chunk's starting row for each expert.
+__global__ void route_scan_kernel(int32_t *__restrict__ chunk_counts, int nchunks, int32_t E,
+                                  int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
+                                  int32_t *__restrict__ tile_offsets) {
+  extern __shared__ int32_t sm[];  // [2 * blockDim.x]
+  int32_t *s_rows = sm, *s_tiles = sm + blockDim.x;
+  const int per = (E + blockDim.x - 1) / blockDim.x;
+  const int e0 = threadIdx.x * per;
+  int32_t local_rows = 0, local_tiles = 0;
+  for (int e = e0; e < e0 + per && e < E; ++e) {
+    int32_t run = 0;
+    for (int c = 0; c < nchunks; ++c) {
+      int32_t v = chunk_counts[(int64_t)c * E + e];
+      chunk_counts[(int64_t)c * E + e] = run;  // exclusive within the expert
+      run += v;
+    }
+    counts[e] = run;
+    local_rows += run;
+    local_tiles += (run + 127) / 128;
+  }
+  s_rows[threadIdx.x] = local_rows;
+  s_tiles[threadIdx.x] = local_tiles;
+  __syncthreads();
+  // inclusive Hillis-Steele scan over threads
+  for (int o = 1; o < (int)blockDim.x; o <<= 1) {
+    int32_t a = threadIdx.x >= (unsigned)o ? s_rows[threadIdx.x - o] : 0;
+    int32_t b = threadIdx.x >= (unsigned)o ? s_tiles[threadIdx.x - o] : 0;
+    __syncthreads();
+    s_rows[threadIdx.x] += a;
+    s_tiles[threadIdx.x] += b;
+    __syncthreads();
+  }
+  int32_t row_base = s_rows[threadIdx.x] - local_rows;
+  int32_t tile_base = s_tiles[threadIdx.x] - local_tiles;
+  for (int e = e0; e < e0 + per && e < E; ++e) {
+    offsets[e] = row_base;
+    tile_offsets[e] = tile_base;
+    for (int c = 0; c < nchunks; ++c) chunk_counts[(int64_t)c * E + e] += row_base;
+    row_base += counts[e];
+    tile_base += (counts[e] + 127) / 128;
+  }
+  if (threadIdx.x == blockDim.x - 1) {
+    offsets[E] = s_rows[threadIdx.x];
+    tile_offsets[E] = s_tiles[threadIdx.x];
+  }
+}
+
+// Pass 3: stable scatter.  Within a chunk, slots are visited in order; a
+// slot's row is its expert's running position.
+__global__ void route_scatter_kernel(const int32_t *__restrict__ ids, int64_t R, int32_t E,
+                                     const int32_t *__restrict__ chunk_base, int32_t *__restrict__ perm,
+                                     int32_t *__restrict__ inv) {
+  extern __shared__ int32_t run[];  // [E]
+  const int lane = threadIdx.x;
+  for (int e = lane; e < E; e += 32) run[e] = chunk_base[(int64_t)blockIdx.x * E + e];
+  __syncwarp();
+  const int64_t base = (int64_t)blockIdx.x * kChunk;
+  for (int step = 0; step < kChunk / 32; ++step) {
+    const int64_t f = base + step * 32 + lane;
+    int id = -1;
+    if (f < R) {
+      id = ids[f];
+      if (id < 0 || id >= E) id = -1;
+    }
+    const uint32_t grp = __match_any_sync(0xffffffffu, id);
+    int32_t pos = -1;
+    if (id >= 0) pos = run[id] + __popc(grp & lanemask_lt());
+    __syncwarp();
+    if (id >= 0 && (grp & lanemask_lt()) == 0) run[id] += __popc(grp);
+    __syncwarp();
+    if (f < R) {
+      inv[f] = pos;
+      if (pos >= 0) perm[pos] = (int32_t)f;
+    }
+  }
+}
+
+__device__ __forceinline__ int find_expert(const int32_t *__restrict__ offsets, int E, int32_t r) {
+  // largest e with offsets[e] <= r < offsets[e+1]  (upper_bound(offsets, r) - 1)
+  int lo = 0, hi = E;  // offsets[lo] <= r < offsets[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (offsets[mid] <= r) lo = mid; else hi = mid;
+  }
+  return lo;
+}
+
+// One warp per routed row: copy the token's packed codes (16-byte vectors)
+// and its scale words into the padded expert-row position (tiled scales).
+__global__ void gather_kernel(const uint8_t *__restrict__ x_codes, const uint8_t *__restrict__ x_sf, int64_t R,
+                              int32_t topk, int64_t H, int32_t E, const int32_t *__restrict__ offsets,
+                              const int32_t *__restrict__ tile_offsets, const int32_t *__restrict__ perm,
+                              uint8_t *__restrict__ a_codes, uint8_t *__restrict__ a_sf) {
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
+  const int lane = threadIdx.x & 31;
+  const int32_t nvalid = offsets[E];
+  const int64_t nvec = H / 32;      // 16-byte vectors of codes per row
+  const int64_t nwords = H / 64;    // 4-byte scale words per row (= K steps)
+  for (int64_t r = blockIdx.x * (int64_t)(blockDim.x / 32) + (threadIdx.x >> 5); r < nvalid; r += warps) {
+    const int e = find_expert(offsets, E, (int32_t)r);
+    const int64_t dst = (int64_t)tile_offsets[e] * 128 + (r - offsets[e]);
+    const int64_t t = perm[r] / topk;
+    const uint4 *src = reinterpret_cast<const uint4 *>(x_codes + t * (H / 2));
+    uint4 *out = reinterpret_cast<uint4 *>(a_codes + dst * (H / 2));
+    for (int64_t v = lane; v < nvec; v += 32) out[v] = src[v];
+    const uint32_t *ssrc = reinterpret_cast<const uint32_t *>(x_sf + t * (H / 16));
+    const int64_t line = ((dst >> 7) * nwords) * 512 + (dst & 31) * 16 + ((dst >> 5) & 3) * 4;
+    for (int64_t w = lane; w < nwords; w += 32)
+      *reinterpret_cast<uint32_t *>(a_sf + line + w * 512) = ssrc[w];
+  }
+}
+
+// out[t, c..c+7] = bf16(sum_s y[inv[t,s], c..c+7]), fp32 adds in slot order.
+__global__ void combine_kernel(const float *__restrict__ y, const int32_t *__restrict__ inv, int64_t T,
+                               int32_t topk, int64_t H, __nv_bfloat16 *__restrict__ out) {
+  const int64_t per_row = H / 8;
+  const int64_t total = T * per_row;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = i / per_row, c = (i - t * per_row) * 8;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int s = 0; s < topk; ++s) {
+      const int32_t r = inv[t * topk + s];
+      if (r < 0) continue;
+      const float4 *p = reinterpret_cast<const float4 *>(y + (int64_t)r * H + c);
+      const float4 a = __ldcs(p), b = __ldcs(p + 1);
+      acc[0] = __fadd_rn(acc[0], a.x); acc[1] = __fadd_rn(acc[1], a.y);
+      acc[2] = __fadd_rn(acc[2], a.z); acc[3] = __fadd_rn(acc[3], a.w);
+      acc[4] = __fadd_rn(acc[4], b.x); acc[5] = __fadd_rn(acc[5], b.y);
+      acc[6] = __fadd_rn(acc[6], b.z); acc[7] = __fadd_rn(acc[7], b.w);
+    }
+    uint4 o;
+    __nv_bfloat162 h0 = __floats2bfloat162_rn(acc[0], acc[1]), h1 = __floats2bfloat162_rn(acc[2], acc[3]);
+    __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[4], acc[5]), h3 = __floats2bfloat162_rn(acc[6], acc[7]);
+    o.x = *reinterpret_cast<uint32_t *>(&h0); o.y = *reinterpret_cast<uint32_t *>(&h1);
+    o.z = *reinterpret_cast<uint32_t *>(&h2); o.w = *reinterpret_cast<uint32_t *>(&h3);
+    *reinterpret_cast<uint4 *>(out + t * H + c) = o;
+  }
+}
+
+int sm_count() {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms;
+}
+
+bool al16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+}  // namespace fp4
+
+using namespace fp4;
+
+extern "C" {
+
+size_t fp4_moe_route_scratch_bytes(int64_t R, int32_t E) {
+  const int64_t nchunks = (R + kChunk - 1) / kChunk;
+  return (size_t)((nchunks < 1 ? 1 : nchunks) * (int64_t)E * 4);
+}
+
+fp4_status fp4_moe_route(const int32_t *expert_ids, int64_t T, int32_t topk, int32_t E, int32_t *counts,
+                         int32_t *offsets, int32_t *tile_offsets, int32_t *perm, int32_t *inv, void *scratch,
+                         size_t scratch_bytes, fp4_stream_t stream) {
+  if (!expert_ids || !counts || !offsets || !tile_offsets || !perm || !inv || !scratch) return FP4_ERR_INVALID_ARG;
+  if (T < 0 || topk < 1 || topk > 16 || E < 1 || E > 4096) return FP4_ERR_UNSUPPORTED_SHAPE;
+  const int64_t R = T * topk;
+  if (R > 2147483647LL / 2) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (scratch_bytes < fp4_moe_route_scratch_bytes(R, E)) return FP4_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(scratch) & 3u)) return FP4_ERR_ALIGNMENT;
+  const DeviceCtx *ctx = device_ctx();
+  if (!ctx) return FP4_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int nchunks = (int)((R + kChunk - 1) / kChunk);
+  int32_t *cc = static_cast<int32_t *>(scratch);
+  const size_t esm = (size_t)E * 4;
+  if (nchunks > 0) {
+    route_count_kernel<<<nchunks, 32, esm, s>>>(expert_ids, R, E, cc, ctx->status);
+    FP4_HOST_CHECK(cudaGetLastError());
+  }
+  route_scan_kernel<<<1, 1024, 2 * 1024 * 4, s>>>(cc, nchunks, E, counts, offsets, tile_offsets);
+  FP4_HOST_CHECK(cudaGetLastError());
+  if (nchunks > 0) {
+    route_scatter_kernel<<<nchunks, 32, esm, s>>>(expert_ids, R, E, cc, perm, inv);
+    FP4_HOST_CHECK(cudaGetLastError());
+  }
+  return FP4_OK;
+}
+
+fp4_status fp4_moe_gather(const uint8_t *x_codes, const uint8_t *x_sf, int64_t T, int32_t topk, int64_t H,
+                          int32_t E, const int32_t *offsets, const int32_t *tile_offsets, const int32_t *perm,
+                          uint8_t *a_codes, uint8_t *a_sf, int64_t rows_cap, fp4_stream_t stream) {
+  if (!x_codes || !x_sf || !offsets || !tile_offsets || !perm || !a_codes || !a_sf) return FP4_ERR_INVALID_ARG;
+  if (T < 0 || topk < 1 || topk > 16 || E < 1 || E > 4096 || H <= 0 || H % 64) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (rows_cap < T * topk + 127LL * E) return FP4_ERR_WORKSPACE;
+  if (!al16(x_codes) || !al16(a_codes) || (reinterpret_cast<uintptr_t>(x_sf) & 3u) ||
+      (reinterpret_cast<uintptr_t>(a_sf) & 3u))
+    return FP4_ERR_ALIGNMENT;
+  const int64_t R = T * topk;
+  if (R == 0) return FP4_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t warps_needed = R;
+  int64_t grid = (warps_needed + 7) / 8;
+  const int64_t cap = (int64_t)sm_count() * 8;
+  if (grid > cap) grid = cap;
+  gather_kernel<<<(unsigned)grid, 256, 0, s>>>(x_codes, x_sf, R, topk, H, E, offsets, tile_offsets, perm, a_codes,
+                                                a_sf);
+  FP4_HOST_CHECK(cudaGetLastError());
+  return FP4_OK;
+}
+
+fp4_status fp4_moe_combine(const float *y, const int32_t *inv, int64_t T, int32_t topk, int64_t H, void *out_bf16,
+                           fp4_stream_t stream) {
+  if (!y || !inv || !out_bf16) return FP4_ERR_INVALID_ARG;
+  if (T < 0 || topk < 1 || topk > 16 || H <= 0 || H % 8) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (!al16(y) || !al16(out_bf16)) return FP4_ERR_ALIGNMENT;
+  if (T == 0) return FP4_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t total = T * (H / 8);
+  int64_t grid = (total + 255) / 256;
+  const int64_t cap = (int64_t)sm_count() * 8;
+  if (grid > cap) grid = cap;
+  combine_kernel<<<(unsigned)grid, 256, 0, s>>>(y, inv, T, topk, H, static_cast<__nv_bfloat16 *>(out_bf16));
+  FP4_HOST_CHECK(cudaGetLastError());
+  return FP4_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,255 @@
+/*
+ * fp4.h -- C ABI of libfp4.so: the NVFP4 / MXFP4 W4A4 hot path for the
+ * routed-expert projections of a mixture-of-experts layer, on NVIDIA B200
+ * (sm_100a).
+ *
+ * Sources (by page title and section):
+ *   [NVFP4]  "DeepSeek-V4.1-Flash-NVFP4" model-card digest:
+ *            §二 E2M1 values {0,0.5,1,1.5,2,3,4,6} with a sign bit, two codes
+ *                per byte, NVFP4 = one block scale per 16 elements under a
+ *                tensor-level scale, W4A4 GEMM with per-block scale correction
+ *                in the accumulator;
+ *            §一 / §六 lossless MXFP4 -> NVFP4 scale remap;
+ *            §三 routed experts w1/w2/w3 quantized, MXFP4 = one UE8M0 scale
+ *                per 32 elements.
+ *   [ARCH]   "DeepSeek-V4 architecture": §2.1 (384 experts, 6 active),
+ *            §5.1 (SwiGLU feed-forward), §6.3 (1x32 MX tiles).
+ *   [QAT]    "DeepSeek-V4 FP4 QAT": §2.1 (E4M3 max 448), §3.1 (MoE forward:
+ *            top-k experts per token, outputs summed).
+ *
+ * Conventions for every entry point
+ *   - All pointers are DEVICE pointers unless marked "host".  The caller owns
+ *     and allocates every buffer, including the workspace; the library
+ *     allocates nothing and keeps only a per-device status word and a cache
+ *     of driver entry points.
+ *   - Calls are asynchronous on `stream` (0 = legacy default stream) unless
+ *     stated otherwise.
+ *   - Argument errors (null pointers, misalignment, unsupported shapes, a
+ *     too-small workspace) are detected on the host and returned before any
+ *     launch.  Errors found on the device (expert id out of range, a
+ *     pipeline wait that timed out) are recorded in the per-device status
+ *     word; read (and clear) it with fp4_get_device_status().
+ *   - Inputs must be finite; NaN/Inf handling is unspecified.
+ *   - Matrices are row-major.  FP4 operands are packed two codes per byte,
+ *     element 2j in the low nibble of byte j.
+ *   - Block scales come in two layouts:
+ *       canonical: uint8 [rows][cols/16] row-major;
+ *       tiled ("MMA layout"): the tensor-core operand layout.  For each slab
+ *         of 128 rows and each 64-column K step, a 512-byte tile of 32 lines
+ *         x 16 bytes; line i holds rows i, i+32, i+64, i+96 (4 bytes each:
+ *         the scales of that row's four 16-element blocks).  Tiles are K-step
+ *         major within a slab:
+ *           byte(r, kb) = ((r/128)*(cols/64) + kb/4)*512 + (r%32)*16
+ *                         + ((r/32)%4)*4 + kb%4
+ *         Its size is fp4_sf_tiled_bytes(rows, cols) (rows padded to 128).
+ */
+#ifndef FP4_H_
+#define FP4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *fp4_stream_t; /* same object as cudaStream_t */
+
+typedef enum {
+  FP4_OK = 0,
+  FP4_ERR_INVALID_ARG = 1,       /* null pointer, bad enum, negative size */
+  FP4_ERR_ALIGNMENT = 2,         /* pointer or leading dimension not 16-byte aligned */
+  FP4_ERR_UNSUPPORTED_SHAPE = 3, /* a size outside what the kernels accept */
+  FP4_ERR_RANGE = 4,             /* MX->NV remap: exponent span > 17 octaves, or UE8M0 NaN */
+  FP4_ERR_BAD_EXPERT = 5,        /* device: expert id outside [0, E) */
+  FP4_ERR_WORKSPACE = 6,         /* workspace too small */
+  FP4_ERR_DEVICE_TIMEOUT = 7,    /* device: a bounded pipeline wait expired */
+  FP4_ERR_CUDA = 8               /* a CUDA runtime/driver call failed */
+} fp4_status;
+
+typedef enum { FP4_NV = 0, FP4_MX = 1 } fp4_format;
+
+typedef enum { FP4_OUT_F32 = 0, FP4_OUT_BF16 = 1 } fp4_out_dtype;
+
+/* flags */
+#define FP4_STATIC_GLOBAL_SCALE 0x1u /* fp4_quantize(NV): *global_scale is an input */
+#define FP4_SCALE_LAYOUT_TILED 0x2u  /* fp4_quantize(NV): write scales in the tiled layout */
+#define FP4_DEBUG_DUMP_H 0x4u        /* MoE w13 stage: also write fp32 h */
+
+/* Human-readable name of a status code (static string). */
+const char *fp4_status_string(fp4_status s);
+
+/* Size in bytes of a tiled scale buffer for a [rows, cols] FP4 matrix
+ * (cols % 64 == 0): ceil(rows/128)*128 * cols/16. */
+size_t fp4_sf_tiled_bytes(int64_t rows, int64_t cols);
+
+/* Workspace bytes fp4_quantize needs (dynamic NVFP4 amax): 256. */
+size_t fp4_quantize_workspace_size(void);
+
+/*
+ * fp4_quantize -- bf16 [rows, cols] (row stride `ld` elements) -> packed E2M1
+ * codes uint8 [rows, cols/2] + block scales.  [NVFP4 §二; NVFP4 §三 for MX]
+ *
+ * FP4_NV (cols % 16 == 0; cols % 64 == 0 with FP4_SCALE_LAYOUT_TILED):
+ *   g = amax(tensor)/2688 (fp32) unless FP4_STATIC_GLOBAL_SCALE, in which case
+ *   *global_scale (device fp32) is read as g.  Per 16-element block:
+ *   sf = E4M3_RNE(amax_b / (6 g)); s = dec(sf)*g; code = E2M1_RNE(x * (1/s))
+ *   (0 when s == 0); every step one fp32 RN operation in that order.
+ *   scales: E4M3 bytes, canonical [rows][cols/16] or tiled.
+ *   global_scale: device fp32[1]; output g (dynamic) or input (static).
+ *   workspace: >= fp4_quantize_workspace_size() bytes, 16-byte aligned
+ *   (dynamic mode only; may be NULL with FP4_STATIC_GLOBAL_SCALE).
+ * FP4_MX (cols % 32 == 0): per 32-element block X = clamp(floor(log2 amax)-2,
+ *   -127, 127), scale byte X+127 (0 for an all-zero block), code =
+ *   E2M1_RNE(x * 2^-X).  scales: UE8M0 [rows][cols/32].  global_scale,
+ *   workspace and flags are ignored.
+ * Alignment: x, codes, workspace 16-byte aligned; ld*2 % 16 == 0.
+ */
+fp4_status fp4_quantize(fp4_format fmt, const void *x_bf16, int64_t rows, int64_t cols, int64_t ld,
+                        uint8_t *codes, uint8_t *scales, float *global_scale, uint32_t flags,
+                        void *workspace, size_t ws_bytes, fp4_stream_t stream);
+
+/*
+ * fp4_mx_to_nv -- lossless MXFP4 -> NVFP4 scale remap [NVFP4 §一 point 2, §六].
+ * `num_tensors` tensors of [rows, cols] each, stored back to back (codes
+ * uint8 [num_tensors*rows][cols/2], mx_scales UE8M0 [..][cols/32]).  Per
+ * tensor: e_max = the largest MX exponent among blocks holding a nonzero
+ * magnitude code; nv_global[t] = 2^(e_max-8); each such block's E4M3 scale
+ * is 2^(e - e_max + 8), written to both of its 16-element halves
+ * (nv_scales canonical [..][cols/16]); blocks of zeros get scale 0.  Codes
+ * are not touched (they are identical in both formats).
+ * A tensor whose live exponents span more than 17 octaves (or holds a UE8M0
+ * NaN byte) cannot be remapped exactly: its scales are left untouched and its
+ * nv_global is set to NaN.  This call is an offline weight-preparation step
+ * and is SYNCHRONOUS: it waits for the stream and returns FP4_ERR_RANGE if any
+ * tensor was refused.
+ */
+fp4_status fp4_mx_to_nv(const uint8_t *codes, const uint8_t *mx_scales, int64_t rows, int64_t cols,
+                        int64_t num_tensors, uint8_t *nv_scales, float *nv_global, uint32_t flags,
+                        fp4_stream_t stream);
+
+/*
+ * fp4_gemm -- C[M,N] = (g_a*g_b) * A_dq[M,K] . B_dq[N,K]^T  [NVFP4 §二]
+ * A and B are NVFP4, K-major (row-major [M,K] and [N,K]); a_sf/b_sf are
+ * TILED scale buffers (fp4_sf_tiled_bytes(M,K) / (N,K)); a_g/b_g device fp32[1].
+ * c: row-major [M,N], fp32 or bf16 (RNE).  fp32 accumulation in tensor memory.
+ * Shapes: M,N >= 1; K % 64 == 0; N % 8 == 0.  Codes 16-byte aligned.
+ */
+fp4_status fp4_gemm(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_g,
+                    const uint8_t *b_codes, const uint8_t *b_sf, const float *b_g, void *c,
+                    fp4_out_dtype c_dtype, int64_t M, int64_t N, int64_t K, uint32_t flags,
+                    fp4_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * MoE routed-expert layer [QAT §3.1; ARCH §2.1, §5.1; NVFP4 §三]
+ *
+ * Weights (all NVFP4, prepared offline with fp4_quantize / fp4_mx_to_nv):
+ *   w13_codes  uint8 [E][2I][H/2]   gate (w1) and up (w3) rows interleaved in
+ *                                   groups of 16: rows 32j..32j+15 = w1 rows
+ *                                   16j..16j+15, rows 32j+16..32j+31 = w3 rows
+ *                                   16j..16j+15
+ *   w13_sf     tiled scales of the [E*2I, H] matrix
+ *   w13_g      fp32 [E]  tensor scale of each expert's w13
+ *   w2_codes   uint8 [E][H][I/2];  w2_sf tiled scales of [E*H, I];  w2_g fp32 [E]
+ *   h_g        fp32 [E]  static NVFP4 tensor scale used to re-quantize each
+ *                        expert's intermediate h (calibrated by the caller)
+ * Per routed row (token t, slot s, expert e = expert_ids[t,s]):
+ *   h = silu(a_g*g13[e] * x_q.W1_e^T) * (a_g*g13[e] * x_q.W3_e^T)   (fp32)
+ *   h_q = NVFP4(h; g = h_g[e])
+ *   y = w[t,s] * (h_g[e]*g2[e]) * h_q.W2_e^T                           (fp32)
+ *   out[t] = bf16_RNE( sum over s = 0..k-1, in that order, of y(t,s) )
+ * Routed rows are ordered by (expert, token, slot) and padded per expert to
+ * a multiple of 128 rows.
+ * Shapes: H % 256 == 0, I % 256 == 0, 1 <= topk <= 16, 1 <= E <= 4096.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  const uint8_t *w13_codes;
+  const uint8_t *w13_sf;
+  const float *w13_g;
+  const uint8_t *w2_codes;
+  const uint8_t *w2_sf;
+  const float *w2_g;
+  const float *h_g;
+} fp4_moe_weights;
+
+/* Workspace bytes for fp4_moe_grouped_gemm at these sizes (256-byte aligned
+ * sub-buffers: header, quantized x, routing tables, gathered rows, h, y). */
+size_t fp4_moe_workspace_size(int64_t T, int32_t topk, int64_t H, int64_t I, int32_t E);
+
+/*
+ * fp4_moe_grouped_gemm -- the whole routed-expert layer in one call:
+ * dynamic NVFP4 quantize of x -> routing permute -> gather -> grouped w13 GEMM
+ * with SwiGLU and NVFP4 re-quantize in its epilogue -> grouped w2 GEMM with
+ * the top-k weight -> fixed-order combine to bf16.
+ *   tokens_bf16  [T][H];  expert_ids int32 [T][topk];
+ *   topk_weights fp32 [T][topk] or NULL (weights 1.0);  out_bf16 [T][H].
+ *   workspace >= fp4_moe_workspace_size(...), 256-byte aligned.
+ *   flags: FP4_DEBUG_DUMP_H needs h_dump (fp32, rows = padded routed rows,
+ *   I columns); otherwise h_dump may be NULL.
+ * Expert ids outside [0,E) set FP4_ERR_BAD_EXPERT in the device status; such
+ * slots contribute nothing.
+ */
+fp4_status fp4_moe_grouped_gemm(const void *tokens_bf16, const int32_t *expert_ids,
+                                const float *topk_weights, int64_t T, int32_t topk,
+                                const fp4_moe_weights *w, int64_t H, int64_t I, int32_t E,
+                                void *out_bf16, void *workspace, size_t ws_bytes, uint32_t flags,
+                                float *h_dump, fp4_stream_t stream);
+
+/* ---- the layer's stages, each callable on its own ------------------------ */
+
+/* Routing tables written by fp4_moe_route (all device int32):
+ *   counts[E]          rows per expert
+ *   offsets[E+1]       exclusive prefix of counts (row index in routed order)
+ *   tile_offsets[E+1]  exclusive prefix of ceil(counts/128) (128-row tiles);
+ *                      expert e's padded rows start at 128*tile_offsets[e]
+ *   perm[T*topk]       routed row -> flat slot index t*topk+s
+ *   inv[T*topk]        flat slot index -> routed row (-1 for a bad expert id)
+ * `scratch` needs fp4_moe_route_scratch_bytes(T*topk, E) bytes. */
+size_t fp4_moe_route_scratch_bytes(int64_t R, int32_t E);
+fp4_status fp4_moe_route(const int32_t *expert_ids, int64_t T, int32_t topk, int32_t E,
+                         int32_t *counts, int32_t *offsets, int32_t *tile_offsets, int32_t *perm,
+                         int32_t *inv, void *scratch, size_t scratch_bytes, fp4_stream_t stream);
+
+/* Gather token rows into expert-contiguous, 128-padded rows: a_codes
+ * [rows_cap][H/2], a_sf tiled for [rows_cap, H]; x_sf canonical [T][H/16].
+ * rows_cap >= 128*tile_offsets[E] (T*topk + 127*E always suffices). */
+fp4_status fp4_moe_gather(const uint8_t *x_codes, const uint8_t *x_sf, int64_t T, int32_t topk,
+                          int64_t H, int32_t E, const int32_t *offsets, const int32_t *tile_offsets,
+                          const int32_t *perm, uint8_t *a_codes, uint8_t *a_sf, int64_t rows_cap,
+                          fp4_stream_t stream);
+
+/* Grouped w13 GEMM + SwiGLU + NVFP4 re-quantize of h with h_g[e]:
+ * a = gathered rows (codes [rows_cap][H/2], tiled sf), a_g = fp32[1] tensor
+ * scale of x; writes h_codes [rows_cap][I/2] and tiled h_sf for [rows_cap, I]
+ * (only rows that hold a routed row are written). h_dump (FP4_DEBUG_DUMP_H):
+ * fp32 [rows_cap][I]. */
+fp4_status fp4_moe_w13(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_g,
+                       const fp4_moe_weights *w, int64_t H, int64_t I, int32_t E,
+                       const int32_t *counts, const int32_t *tile_offsets, int64_t rows_cap,
+                       uint8_t *h_codes, uint8_t *h_sf, uint32_t flags, float *h_dump,
+                       fp4_stream_t stream);
+
+/* Grouped w2 GEMM: y[offsets[e]+i] = w[perm[row]] * h_g[e]*w2_g[e] * (h . W2_e^T)
+ * y: fp32 [T*topk][H] in routed order; topk_weights may be NULL. */
+fp4_status fp4_moe_w2(const uint8_t *h_codes, const uint8_t *h_sf, const fp4_moe_weights *w,
+                      int64_t H, int64_t I, int32_t E, const int32_t *counts,
+                      const int32_t *offsets, const int32_t *tile_offsets, const int32_t *perm,
+                      const float *topk_weights, int64_t rows_cap, float *y, fp4_stream_t stream);
+
+/* out[t] = bf16_RNE(sum_{s=0..k-1} y[inv[t*k+s]]) (fp32 adds in slot order;
+ * inv < 0 contributes nothing). */
+fp4_status fp4_moe_combine(const float *y, const int32_t *inv, int64_t T, int32_t topk, int64_t H,
+                           void *out_bf16, fp4_stream_t stream);
+
+/* Synchronize `stream`, then read and clear this device's status word
+ * (FP4_OK if no device-side error was recorded since the last read). */
+fp4_status fp4_get_device_status(fp4_stream_t stream);
+
+/* Test hook: the pipeline-wait limit, in nanoseconds, used by kernels launched
+ * after this call on this device (default 2e9).  0 restores the default. */
+void fp4_set_wait_limit_ns(uint64_t ns);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FP4_H_ */

@@ -1,0 +1,39 @@
+"""Small helpers shared by the GPU parity tests (host conversions only)."""
+import numpy as np
+import torch
+
+
+def f32(x_bf16):
+    """bf16 torch tensor -> exact fp32 numpy array."""
+    return x_bf16.float().cpu().numpy()
+
+
+def np_u8(t):
+    return t.cpu().numpy().astype(np.uint8)
+
+
+def f32_bits_equal(a, b):
+    a = np.asarray(a, dtype=np.float32).reshape(-1)
+    b = np.asarray(b, dtype=np.float32).reshape(-1)
+    return np.array_equal(a.view(np.uint32), b.view(np.uint32))
+
+
+def bf16_bits(t):
+    return t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def bf16_ulps_apart(bits_a, bits_b):
+    """Distance in representable bf16 steps between two bit patterns (same
+    sign assumed for nonzero values; zeros of either sign are equal)."""
+    a = np.asarray(bits_a, dtype=np.int64)
+    b = np.asarray(bits_b, dtype=np.int64)
+
+    def ordered(x):
+        mag = x & 0x7FFF
+        return np.where(x & 0x8000, -mag, mag)
+
+    return np.abs(ordered(a) - ordered(b))
+
+
+def tiled_const(nbytes, value, device="cuda"):
+    return torch.full((int(nbytes),), value, dtype=torch.uint8, device=device)

@@ -1,0 +1,97 @@
+"""The C-ABI library loads, exports every entry point include/fp4.h declares,
+and rejects bad arguments on the host before touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    text = open(os.path.join(ROOT, "include", "fp4.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fp4_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_api():
+    syms = _declared_symbols()
+    for name in ["fp4_quantize", "fp4_mx_to_nv", "fp4_gemm", "fp4_moe_grouped_gemm", "fp4_moe_route",
+                 "fp4_moe_gather", "fp4_moe_w13", "fp4_moe_w2", "fp4_moe_combine", "fp4_get_device_status"]:
+        assert name in syms
+
+
+def test_library_exports_every_declared_symbol():
+    import fp4_block_scaled_03_b200 as fp4
+
+    lib = ctypes.CDLL(fp4.LIB_PATH)
+    missing = [s for s in _declared_symbols() if not hasattr(lib, s)]
+    assert not missing, missing
+    # the binding wraps exactly the declared entry points
+    assert sorted(fp4.EXPORTED) == _declared_symbols()
+
+
+def test_status_strings_and_sizes():
+    import fp4_block_scaled_03_b200 as fp4
+
+    for code, name in fp4.STATUS.items():
+        assert fp4.lib.fp4_status_string(code).decode() == name
+    assert fp4.fp4_sf_tiled_bytes(1, 64) == 128 * 4
+    assert fp4.fp4_sf_tiled_bytes(129, 128) == 256 * 8
+    assert fp4.fp4_sf_tiled_bytes(10, 32) == 0  # cols must be a multiple of 64
+    assert fp4.lib.fp4_quantize_workspace_size() == 256
+    # workspace grows with every dimension
+    a = fp4.fp4_moe_workspace_size(64, 6, 7168, 2048, 384)
+    assert a > 0 and fp4.fp4_moe_workspace_size(128, 6, 7168, 2048, 384) > a
+    assert fp4.fp4_moe_route_scratch_bytes(98304, 384) == 96 * 384 * 4
+
+
+def _fake(addr):
+    return ctypes.c_void_p(addr)
+
+
+def test_host_validation_without_gpu():
+    """Every call below fails its host checks, so nothing reaches CUDA."""
+    import fp4_block_scaled_03_b200 as fp4
+
+    L = fp4.lib
+    A = 0x10000  # 16-byte aligned fake address, never dereferenced
+    # null pointers
+    assert L.fp4_quantize(0, None, 4, 64, 64, A, A, A, 0, A, 256, None) == 1
+    # misaligned input
+    assert L.fp4_quantize(0, A + 2, 4, 64, 64, A, A, A, 0, A, 256, None) == 2
+    # bad format enum
+    assert L.fp4_quantize(7, A, 4, 64, 64, A, A, A, 0, A, 256, None) == 1
+    # GEMM: K not a multiple of 64, N not a multiple of 8, misaligned C
+    assert L.fp4_gemm(A, A, A, A, A, A, A, 0, 128, 256, 100, 0, None) == 3
+    assert L.fp4_gemm(A, A, A, A, A, A, A, 0, 128, 250, 512, 0, None) == 3
+    assert L.fp4_gemm(A, A, A, A, A, A, A + 4, 0, 128, 256, 512, 0, None) == 2
+    # routing: topk out of range, too little scratch
+    assert L.fp4_moe_route(A, 4, 0, 8, A, A, A, A, A, A, 1 << 20, None) == 3
+    assert L.fp4_moe_route(A, 4096, 6, 384, A, A, A, A, A, A, 16, None) == 6
+    # MoE layer: H not a multiple of 256, workspace too small, misaligned workspace
+    w = fp4.MoeWeights(A, A, A, A, A, A, A)
+    assert L.fp4_moe_grouped_gemm(A, A, None, 8, 2, ctypes.byref(w), 100, 256, 4, A, A, 1 << 30, 0, None, None) == 3
+    assert L.fp4_moe_grouped_gemm(A, A, None, 8, 2, ctypes.byref(w), 256, 256, 4, A, A, 64, 0, None, None) == 6
+    assert L.fp4_moe_grouped_gemm(A, A, None, 8, 2, ctypes.byref(w), 256, 256, 4, A, A + 16, 1 << 30, 0, None, None) == 2
+    # debug dump requested without a buffer
+    assert L.fp4_moe_grouped_gemm(A, A, None, 8, 2, ctypes.byref(w), 256, 256, 4, A, A, 1 << 30, 4, None, None) == 1
+    # gather: rows_cap too small for the worst-case padding
+    assert L.fp4_moe_gather(A, A, 8, 2, 256, 4, A, A, A, A, A, 16, None) == 6
+    # MX->NV: cols not a multiple of 32
+    assert L.fp4_mx_to_nv(A, A, 4, 48, 1, A, A, 0, None) == 3
+
+
+def test_package_fails_loudly_without_library(tmp_path, monkeypatch):
+    """Importing the binding from a copy without libfp4.so raises (no fallback)."""
+    import importlib.util
+    import shutil
+
+    pkg = tmp_path / "fp4copy"
+    pkg.mkdir()
+    shutil.copy(os.path.join(ROOT, "fp4_block_scaled_03_b200", "__init__.py"), pkg / "__init__.py")
+    spec = importlib.util.spec_from_file_location("fp4copy", pkg / "__init__.py")
+    mod = importlib.util.module_from_spec(spec)
+    with pytest.raises(ImportError):
+        spec.loader.exec_module(mod)

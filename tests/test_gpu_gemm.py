@@ -1,0 +1,103 @@
+"""Dense block-scaled GEMM on tcgen05 against the oracle.
+
+fp32 output: |C - C_ref| <= 1e-4 * (|A_dq| |B_dq|^T)_ij elementwise.
+bf16 output: within 1 bf16 ulp of RNE_bf16(C_ref) (where cancellation makes
+the fp32 accumulation bound exceed an ulp, that bound plus one ulp).
+The integer special case (all scales 1, g = 1) must be bit-exact."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import formats as F
+from oracle import gemm as G
+from oracle import quant as Q
+from tests._util import bf16_bits, bf16_ulps_apart, f32, tiled_const
+
+pytestmark = pytest.mark.gpu
+
+
+def _lib():
+    import fp4_block_scaled_03_b200 as fp4
+
+    return fp4
+
+
+def _int_val(codes):
+    two = np.array([0, 1, 2, 3, 4, 6, 8, 12], dtype=np.int64)
+    c = F.unpack_nibbles(codes)
+    return np.where(c & 8, -two[c & 7], two[c & 7])
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 256, 256), (200, 264, 320), (1, 8, 64), (300, 520, 1088)])
+def test_integer_gemm_bit_exact(M, N, K):
+    fp4 = _lib()
+    a = synth.random_codes((M, K // 2), seed=M + 1, device="cuda")
+    b = synth.random_codes((N, K // 2), seed=N + 2, device="cuda")
+    one = torch.ones(1, dtype=torch.float32, device="cuda")
+    a_sf = tiled_const(fp4.fp4_sf_tiled_bytes(M, K), 0x38)
+    b_sf = tiled_const(fp4.fp4_sf_tiled_bytes(N, K), 0x38)
+    c = fp4.gemm(a, a_sf, one, b, b_sf, one, M, N, K).cpu().numpy()
+    ref = (_int_val(a.cpu().numpy()) @ _int_val(b.cpu().numpy()).T).astype(np.float64) / 4.0
+    assert np.array_equal(c.astype(np.float64), ref)
+
+
+def _quantized_operands(M, N, K, seed, w_sigma=0.02, w_frac=0.01, w_factor=50.0):
+    fp4 = _lib()
+    a_bf = synth.activations_bf16((M, K), seed=seed, device="cuda")
+    b_bf = synth.weights_bf16((N, K), w_sigma, w_frac, w_factor, seed=seed + 1, device="cuda")
+    a_c, a_sf, a_g = fp4.quantize_nv(a_bf, tiled=True)
+    b_c, b_sf, b_g = fp4.quantize_nv(b_bf, tiled=True)
+    ra = Q.nvfp4_quantize(f32(a_bf))
+    rb = Q.nvfp4_quantize(f32(b_bf))
+    return (a_c, a_sf, a_g, b_c, b_sf, b_g), ra, rb
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 256, 512), (333, 136, 1088), (64, 512, 4096)])
+def test_gemm_fp32_within_bound(M, N, K):
+    ops, ra, rb = _quantized_operands(M, N, K, seed=M * 3 + K)
+    c = _lib().gemm(*ops, M, N, K).cpu().numpy().astype(np.float64)
+    C, bound = G.nvfp4_gemm_ref(*ra, *rb)
+    err = np.abs(c - C)
+    assert np.all(err <= G.FP32_REL_TOL * bound), float((err / np.maximum(bound, 1e-300)).max())
+
+
+def _check_bf16(c_bits, C, bound):
+    ref_bits = F.f64_to_bf16_rne(C)
+    ulps = bf16_ulps_apart(c_bits, ref_bits)
+    ok = ulps <= 1
+    got = F.bf16_bits_to_f32(c_bits).astype(np.float64)
+    ok |= np.abs(got - C) <= G.FP32_REL_TOL * bound + G.bf16_ulp(got)
+    return ok
+
+
+@pytest.mark.parametrize("M,N,K", [(256, 512, 1024), (77, 264, 576)])
+def test_gemm_bf16_within_one_ulp(M, N, K):
+    ops, ra, rb = _quantized_operands(M, N, K, seed=K + N)
+    c = _lib().gemm(*ops, M, N, K, out_dtype=torch.bfloat16)
+    C, bound = G.nvfp4_gemm_ref(*ra, *rb)
+    ok = _check_bf16(bf16_bits(c), C, bound)
+    assert ok.all(), int((~ok).sum())
+
+
+def test_gemm_4096_cubed_bf16_sampled():
+    """The dense expert-sized GEMM in the bench's launch configuration:
+    activations quantized on device, weights N(0,0.02) + 0.5% x30, bf16 out;
+    a block of rows and columns checked against the fp64 oracle."""
+    M = N = K = 4096
+    fp4 = _lib()
+    a_bf = synth.activations_bf16((M, K), seed=0, device="cuda")
+    b_bf = synth.weights_bf16((N, K), 0.02, 0.005, 30.0, seed=1, device="cuda")
+    a_c, a_sf, a_g = fp4.quantize_nv(a_bf, tiled=True)
+    b_c, b_sf, b_g = fp4.quantize_nv(b_bf, tiled=True)
+    c = fp4.gemm(a_c, a_sf, a_g, b_c, b_sf, b_g, M, N, K, out_dtype=torch.bfloat16)
+    rows = np.sort(np.random.default_rng(1).choice(M, 96, replace=False))
+    cols = np.sort(np.random.default_rng(2).choice(N, 160, replace=False))
+    af, bf = f32(a_bf), f32(b_bf)
+    ga, gb = Q.nv_global_scale(af), Q.nv_global_scale(bf)
+    ra = Q.nvfp4_quantize(af[rows], g=ga)
+    rb = Q.nvfp4_quantize(bf[cols], g=gb)
+    C, bound = G.nvfp4_gemm_ref(*ra, *rb)
+    cb = bf16_bits(c)[np.ix_(rows, cols)]
+    ok = _check_bf16(cb, C, bound)
+    assert ok.all(), int((~ok).sum())

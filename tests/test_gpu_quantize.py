@@ -1,0 +1,140 @@
+"""GPU quantizers and the MX->NV remap against the oracle: codes, scales and
+global scales must match bit for bit."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import formats as F
+from oracle import layouts as LY
+from oracle import quant as Q
+from tests._util import f32, f32_bits_equal, np_u8
+
+pytestmark = pytest.mark.gpu
+
+
+def _lib():
+    import fp4_block_scaled_03_b200 as fp4
+
+    return fp4
+
+
+@pytest.mark.parametrize("rows,cols", [(1, 16), (3, 48), (128, 512), (200, 1024), (1000, 7168)])
+def test_nv_dynamic_canonical_bit_exact(rows, cols):
+    x = synth.activations_bf16((rows, cols), seed=rows * 7 + cols, device="cuda")
+    codes, sf, g = _lib().quantize_nv(x)
+    rc, rs, rg = Q.nvfp4_quantize(f32(x))
+    assert f32_bits_equal(g.cpu().numpy(), [rg])
+    assert np.array_equal(np_u8(sf), rs)
+    assert np.array_equal(np_u8(codes), rc)
+
+
+@pytest.mark.parametrize("rows,cols", [(5, 64), (130, 256), (257, 4096)])
+def test_nv_tiled_layout_bit_exact(rows, cols):
+    x = synth.weights_bf16((rows, cols), 0.02, 0.005, 30.0, seed=11 + rows, device="cuda")
+    codes, sf_t, g = _lib().quantize_nv(x, tiled=True)
+    rc, rs, rg = Q.nvfp4_quantize(f32(x))
+    assert f32_bits_equal(g.cpu().numpy(), [rg])
+    assert np.array_equal(np_u8(codes), rc)
+    assert np.array_equal(LY.sf_from_mma(np_u8(sf_t), rows, cols), rs)
+
+
+def test_nv_static_scale_and_exact_ties():
+    """Blocks whose scale is a power of two put x*(1/s) exactly on every E2M1
+    rounding tie (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5) and on +-0 and tiny
+    negatives; the device must take the same decisions as the oracle."""
+    ties = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, -0.25, -0.75, -1.25, -1.75, -2.5, -3.5, -5.0, -0.0]
+    rows = []
+    for j in range(-8, 9):
+        blk = np.array([6.0] + ties, dtype=np.float64) * 2.0**j
+        rows.append(blk)
+        blk2 = blk.copy()
+        blk2[1:4] = [-1e-3 * 2.0**j, 7.0 * 2.0**j, 1.0e-30]  # tiny negative, saturation, tiny positive
+        rows.append(blk2)
+    x_np = np.stack(rows).astype(np.float32)
+    x = torch.from_numpy(x_np).to(torch.bfloat16).cuda()
+    g = torch.tensor([1.0], dtype=torch.float32)
+    codes, sf, _ = _lib().quantize_nv(x, g=g)
+    rc, rs, _ = Q.nvfp4_quantize(f32(x), g=np.float32(1.0))
+    assert np.array_equal(np_u8(sf), rs)
+    assert np.array_equal(np_u8(codes), rc)
+    # and the tie decisions are the reading's (ties to the even code)
+    dq = F.e2m1_decode(F.unpack_nibbles(rc))[0::2, 1:8]
+    assert np.allclose(dq[8], [0.0, 1.0, 1.0, 2.0, 2.0, 4.0, 4.0])  # j = 0 row
+
+
+def test_nv_zero_tensor():
+    x = torch.zeros((4, 64), dtype=torch.bfloat16, device="cuda")
+    x[1] = -0.0
+    codes, sf, g = _lib().quantize_nv(x)
+    rc, rs, rg = Q.nvfp4_quantize(f32(x))
+    assert g.item() == 0.0 and rg == 0
+    assert np.array_equal(np_u8(sf), rs) and np.array_equal(np_u8(codes), rc)
+
+
+def test_nv_full_size_sampled_rows():
+    """Pro-shaped activation [16384, 7168] in the launch the bench times:
+    dynamic g over the whole tensor, then sampled rows checked exactly."""
+    T, H = 16384, 7168
+    x = synth.activations_bf16((T, H), seed=3, device="cuda")
+    codes, sf, g = _lib().quantize_nv(x)
+    xf = f32(x)
+    rg = Q.nv_global_scale(xf)
+    assert f32_bits_equal(g.cpu().numpy(), [rg])
+    rows = np.random.default_rng(0).choice(T, 48, replace=False)
+    rows = np.concatenate([rows, [0, T - 1]])
+    rc, rs, _ = Q.nvfp4_quantize(xf[rows], g=rg)
+    assert np.array_equal(np_u8(codes[torch.from_numpy(rows).cuda()]), rc)
+    assert np.array_equal(np_u8(sf[torch.from_numpy(rows).cuda()]), rs)
+
+
+@pytest.mark.parametrize("rows,cols", [(1, 32), (5, 96), (256, 4096)])
+def test_mx_bit_exact(rows, cols):
+    x = synth.weights_bf16((rows, cols), 0.02, 0.005, 30.0, seed=rows + cols, device="cuda")
+    codes, sc = _lib().quantize_mx(x)
+    rc, rs = Q.mxfp4_quantize(f32(x))
+    assert np.array_equal(np_u8(sc), rs)
+    assert np.array_equal(np_u8(codes), rc)
+
+
+def test_mx_extreme_exponents():
+    base = synth.activations_bf16((8, 64), seed=5, device="cuda").float()
+    scale = torch.tensor([2.0**-130, 2.0**-126, 2.0**-100, 1.0, 2.0**60, 2.0**120, 2.0**126, 0.0],
+                         device="cuda")[:, None]
+    x = (base * scale).to(torch.bfloat16)
+    codes, sc = _lib().quantize_mx(x)
+    rc, rs = Q.mxfp4_quantize(f32(x))
+    assert np.array_equal(np_u8(sc), rs)
+    assert np.array_equal(np_u8(codes), rc)
+
+
+def test_remap_bit_exact_and_lossless():
+    nt, rows, cols = 4, 64, 256
+    w = synth.weights_bf16((nt * rows, cols), 0.02, 0.005, 30.0, seed=9, device="cuda")
+    w[: rows] *= 64  # tensor 0 has its own range
+    codes, sc = _lib().quantize_mx(w)
+    nv, g = _lib().mx_to_nv(codes, sc, nt)
+    rc, rs = Q.mxfp4_quantize(f32(w))
+    rnv, rg = Q.mx_to_nv(rc, rs, nt)
+    assert np.array_equal(np_u8(nv), rnv)
+    assert f32_bits_equal(g.cpu().numpy(), rg)
+    for t in range(nt):
+        sl = slice(t * rows, (t + 1) * rows)
+        assert np.array_equal(Q.mxfp4_dequantize(rc[sl], rs[sl]), Q.nvfp4_dequantize(rc[sl], np_u8(nv)[sl], rg[t]))
+
+
+def test_remap_refuses_wide_span():
+    fp4 = _lib()
+    rows, cols = 4, 64
+    codes = torch.full((2 * rows, cols // 2), 0x11, dtype=torch.uint8, device="cuda")
+    sc = torch.full((2 * rows, cols // 32), 127, dtype=torch.uint8, device="cuda")
+    sc[rows + 1, 0] = 127 - 18  # tensor 1 spans 18 octaves
+    nv = torch.full((2 * rows, cols // 16), 0xAB, dtype=torch.uint8, device="cuda")
+    g = torch.empty(2, dtype=torch.float32, device="cuda")
+    with pytest.raises(fp4.Fp4Error) as ei:
+        fp4.fp4_mx_to_nv(codes, sc, rows, cols, 2, nv, g)
+    assert ei.value.code == 4
+    gh = g.cpu().numpy()
+    assert gh[0] == np.float32(2.0**-8) and np.isnan(gh[1])
+    assert torch.all(nv[rows:] == 0xAB)  # the refused tensor's scales are untouched
+    assert fp4.fp4_get_device_status() == 0
