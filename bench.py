@@ -1,0 +1,616 @@
+"""Benchmark of the NVFP4 W4A4 routed-expert hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload pro|flash|decode|dense4096|quant]
+                    [--impl fp4|reference]
+
+A step is one pass of the whole hot path over one synthetic batch: dynamic
+NVFP4 quantize of the activations -> routing permute -> gather -> grouped
+w13 GEMM with SwiGLU + NVFP4 re-quantize -> grouped w2 GEMM -> combine
+(workloads pro / flash / decode), one quantize + dense GEMM (dense4096), or
+one activation quantize (quant).  Inputs are resident in HBM before timing;
+weights (9.5 GB for pro) and activations exceed the 126 MB L2, so no flush
+is needed between steps.  Per-kernel times come from CUDA events recorded
+between the stages on the launching stream.  `e2e` repeats the measurement
+through the public C-ABI call with the step's inputs copied from pinned host
+memory and the output copied back inside the timed region.
+
+With --gpus N (torchrun), every rank runs an independent replica on its own
+batch (the layer shards by expert only through an all-to-all exchange, which
+this build does not have): weak scaling, time = max over ranks.
+
+--impl reference times the CPU oracle (oracle/, fp64 numpy) on a bounded
+sample of the same workload, on this host's cores.
+"""
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOADS = {
+    # name: (T, H, I, E, k, zipf, w_sigma, description)
+    "pro": (16384, 7168, 2048, 384, 6, 1.1, 0.01,
+            "Pro-shaped MoE layer: hidden 7168, 384 experts, I 2048, top-6, Zipf 1.1, 16384 prefill tokens"),
+    "flash": (4096, 4096, 2048, 256, 6, 0.0, 0.02,
+              "Flash-shaped MoE layer: hidden 4096, 256 experts, I 2048, top-6 uniform, 4096 tokens, MX weights remapped"),
+    "decode": (64, 7168, 2048, 384, 6, 1.1, 0.01, "Pro-shaped MoE layer at 64 decode tokens (weight-read bound)"),
+}
+
+METRIC = "NVFP4 W4A4 grouped-MoE GEMM TFLOPS (% FP4 peak); quantize GB/s (% HBM)"
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sus=d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                    src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.rows = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append([x.strip() for x in line.split(",")])
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm = []
+        mx = None
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in self.rows:
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+                for i, n in enumerate(names):
+                    if r[5 + i].lower().startswith("active"):
+                        reasons.add(n)
+            except Exception:
+                pass
+        sm_sorted = sorted(sm)
+        loaded = [s for s in sm_sorted if mx and s > 0.5 * mx] or sm_sorted
+        med = loaded[len(loaded) // 2] if loaded else None
+        return {"sm_mhz": med, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+def setup_dist(args):
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+class MoeBench:
+    def __init__(self, name, seed):
+        import torch
+
+        import fp4_block_scaled_03_b200 as fp4
+        import synth
+
+        self.fp4 = fp4
+        T, H, I, E, k, zipf, sigma, desc = WORKLOADS[name]
+        self.T, self.H, self.I, self.E, self.k, self.desc, self.name = T, H, I, E, k, desc, name
+        dev = "cuda"
+        self.x = synth.activations_bf16((T, H), seed=seed, device=dev)
+        self.ids, self.w, self.counts = synth.router(T, E, k, seed=seed + 1, zipf_s=zipf, device=dev)
+        self.w13_codes = torch.empty((E * 2 * I, H // 2), dtype=torch.uint8, device=dev)
+        self.w2_codes = torch.empty((E * H, I // 2), dtype=torch.uint8, device=dev)
+        self.w13_sf = torch.empty(fp4.fp4_sf_tiled_bytes(E * 2 * I, H), dtype=torch.uint8, device=dev)
+        self.w2_sf = torch.empty(fp4.fp4_sf_tiled_bytes(E * H, I), dtype=torch.uint8, device=dev)
+        self.w13_g = torch.empty(E, dtype=torch.float32, device=dev)
+        self.w2_g = torch.empty(E, dtype=torch.float32, device=dev)
+        s13, s2 = fp4.fp4_sf_tiled_bytes(2 * I, H), fp4.fp4_sf_tiled_bytes(H, I)
+        for e in range(E):
+            for (rows, cols, codes, sf, g, sfb, off) in ((2 * I, H, self.w13_codes, self.w13_sf, self.w13_g, s13, 2),
+                                                          (H, I, self.w2_codes, self.w2_sf, self.w2_g, s2, 3)):
+                wb = synth.weights_bf16((rows, cols), sigma, 0.005, 30.0, seed=seed + 1000 * off + e, device=dev)
+                sl = slice(e * rows, (e + 1) * rows)
+                if name == "flash":  # MXFP4 weights remapped losslessly to NVFP4
+                    mc, ms = fp4.quantize_mx(wb)
+                    nv, gg = fp4.mx_to_nv(mc, ms, 1, tiled=True)
+                    codes[sl] = mc
+                    sf[e * sfb:(e + 1) * sfb] = nv
+                    g[e] = gg[0]
+                else:
+                    cc, ss, gg = fp4.quantize_nv(wb, tiled=True)
+                    codes[sl] = cc
+                    sf[e * sfb:(e + 1) * sfb] = ss
+                    g[e] = gg[0]
+                del wb
+        self.h_g = torch.ones(E, dtype=torch.float32, device=dev)
+        self.R = T * k
+        self.cap = fp4.moe_rows_cap(T, k, E)
+        self._alloc()
+        self.calibrate()
+
+    def _alloc(self):
+        import torch
+
+        fp4, T, H, I, E, k, R, cap = self.fp4, self.T, self.H, self.I, self.E, self.k, self.R, self.cap
+        d = "cuda"
+        u8 = lambda n: torch.empty(int(n), dtype=torch.uint8, device=d)  # noqa: E731
+        i32 = lambda n: torch.empty(int(n), dtype=torch.int32, device=d)  # noqa: E731
+        self.xc = torch.empty((T, H // 2), dtype=torch.uint8, device=d)
+        self.xs = torch.empty((T, H // 16), dtype=torch.uint8, device=d)
+        self.xg = torch.empty(1, dtype=torch.float32, device=d)
+        self.qws = u8(256)
+        self.counts_d, self.offs, self.toffs = i32(E), i32(E + 1), i32(E + 1)
+        self.perm, self.inv = i32(R), i32(R)
+        self.scratch = u8(fp4.fp4_moe_route_scratch_bytes(R, E))
+        self.a_c = torch.empty((cap, H // 2), dtype=torch.uint8, device=d)
+        self.a_s = u8(fp4.fp4_sf_tiled_bytes(cap, H))
+        self.h_c = torch.empty((cap, I // 2), dtype=torch.uint8, device=d)
+        self.h_s = u8(fp4.fp4_sf_tiled_bytes(cap, I))
+        self.y = torch.empty((R, H), dtype=torch.float32, device=d)
+        self.out = torch.empty((T, H), dtype=torch.bfloat16, device=d)
+        self.wset = fp4.MoeWeightSet(self.w13_codes, self.w13_sf, self.w13_g, self.w2_codes, self.w2_sf, self.w2_g,
+                                     self.h_g)
+
+    def calibrate(self):
+        """h_g[e] = max|h| over expert e's rows of this batch / 2688 (once)."""
+        import torch
+
+        fp4 = self.fp4
+        dump = torch.zeros((self.cap, self.I), dtype=torch.float32, device="cuda")
+        self.step(events=None, dump=dump)
+        torch.cuda.synchronize()
+        toffs = self.toffs.cpu().tolist()
+        counts = self.counts_d.cpu().tolist()
+        rowmax = dump.abs().amax(dim=1)
+        hg = torch.ones(self.E, dtype=torch.float32, device="cuda")
+        for e in range(self.E):
+            if counts[e]:
+                a = rowmax[toffs[e] * 128: toffs[e] * 128 + counts[e]].max()
+                hg[e] = torch.clamp(a / 2688.0, min=1e-30)
+        self.h_g.copy_(hg)
+        del dump
+        assert fp4.fp4_get_device_status() == 0
+
+    def step(self, events=None, dump=None):
+        fp4 = self.fp4
+        T, H, I, E, k, cap = self.T, self.H, self.I, self.E, self.k, self.cap
+        ev = (lambda i: events[i].record()) if events else (lambda i: None)
+        ev(0)
+        fp4.fp4_quantize(fp4.FP4_NV, self.x, T, H, H, self.xc, self.xs, self.xg, 0, self.qws, 256)
+        ev(1)
+        fp4.fp4_moe_route(self.ids, T, k, E, self.counts_d, self.offs, self.toffs, self.perm, self.inv, self.scratch)
+        ev(2)
+        fp4.fp4_moe_gather(self.xc, self.xs, T, k, H, E, self.offs, self.toffs, self.perm, self.a_c, self.a_s, cap)
+        ev(3)
+        fp4.fp4_moe_w13(self.a_c, self.a_s, self.xg, self.wset, H, I, E, self.counts_d, self.toffs, cap, self.h_c,
+                        self.h_s, fp4.FP4_DEBUG_DUMP_H if dump is not None else 0, dump)
+        ev(4)
+        fp4.fp4_moe_w2(self.h_c, self.h_s, self.wset, H, I, E, self.counts_d, self.offs, self.toffs, self.perm, self.w,
+                       cap, self.y)
+        ev(5)
+        fp4.fp4_moe_combine(self.y, self.inv, T, k, H, self.out)
+        ev(6)
+
+    LAUNCHES_PER_STEP = 9  # amax, quantize, 3 routing, gather, w13, w2, combine
+
+    def flops(self):
+        return 2.0 * 3.0 * self.H * self.I * self.R
+
+    def touched_weight_bytes(self):
+        n = int((self.counts > 0).sum().item())
+        return n * 3 * self.H * self.I * 0.5625
+
+
+# ---------------------------------------------------------------------------
+def run_moe(args, world, rank, peaks):
+    import torch
+
+    fp4 = __import__("fp4_block_scaled_03_b200")
+    b = MoeBench(args.workload, seed=rank * 7919)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        b.step()
+    torch.cuda.synchronize()
+    nst = 7
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nst)] for _ in range(args.steps)]
+    sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        b.step(events=evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop() if sampler else None
+    assert fp4.fp4_get_device_status() == 0
+    ms_total = t0.elapsed_time(t1)
+    ms = max_over_ranks(ms_total / args.steps, world)
+    stage = [0.0] * (nst - 1)
+    for i in range(args.steps):
+        for j in range(nst - 1):
+            stage[j] += evs[i][j].elapsed_time(evs[i][j + 1]) / args.steps
+    flops = b.flops()
+    value = world * flops / (ms * 1e-3) / 1e12
+    fp4_peak = 4.0 * peaks["bf16_sus"]
+    # dominant kernel: the grouped w13 GEMM (2/3 of the layer's FLOPs)
+    w13_flops = 2.0 * 2 * b.I * b.H * b.R
+    w13_tf = w13_flops / (stage[3] * 1e-3) / 1e12
+    w2_tf = (2.0 * b.I * b.H * b.R) / (stage[4] * 1e-3) / 1e12
+    q_bytes = b.T * b.H * 2.5625
+    q_gbs = q_bytes / (stage[0] * 1e-3) / 1e9
+
+    # e2e through the public call: pinned host inputs in, output out, per step
+    x_h = b.x.cpu().pin_memory()
+    ids_h = b.ids.cpu().pin_memory()
+    w_h = b.w.cpu().pin_memory()
+    out_h = torch.empty((b.T, b.H), dtype=torch.bfloat16).pin_memory()
+    x_d, ids_d, w_d = torch.empty_like(b.x), torch.empty_like(b.ids), torch.empty_like(b.w)
+    ws = torch.empty(fp4.fp4_moe_workspace_size(b.T, b.k, b.H, b.I, b.E), dtype=torch.uint8, device="cuda")
+
+    def e2e_step():
+        x_d.copy_(x_h, non_blocking=True)
+        ids_d.copy_(ids_h, non_blocking=True)
+        w_d.copy_(w_h, non_blocking=True)
+        fp4.fp4_moe_grouped_gemm(x_d, ids_d, w_d, b.T, b.k, b.wset, b.H, b.I, b.E, b.out, ws)
+        out_h.copy_(b.out, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+    h2d = b.T * b.H * 2 + b.R * 4 + b.R * 4
+    d2h = b.T * b.H * 2
+    del ws
+
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "nvfp4 (e2m1 x e2m1, e4m3/16 scales, fp32 accumulate)",
+        "data": "synthetic (seeded): bf16 N(0,1) activations, N(0,sigma)+0.5% x30 outlier weights, Gaussian router"
+                " logits + Zipf popularity",
+        "config": {"workload": b.desc, "tokens": b.T, "hidden": b.H, "intermediate": b.I, "experts": b.E,
+                   "topk": b.k, "routed_rows": b.R, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (weights %.2f GB)" % (b.E * 3 * b.H * b.I * 0.5625 / 1e9),
+                   "experts_touched": int((b.counts > 0).sum().item())},
+        "roofline": {"bound": "tensor", "kernel": "fp4_gemm_kernel<256, w13> (grouped w13 + SwiGLU + requant)",
+                     "achieved": round(w13_tf, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
+                     "frac": round(w13_tf / fp4_peak, 4), "traffic": None,
+                     "peak_note": "4 x measured sustained bf16 cuBLAS (nominal fp4/bf16 ratio), of " + peaks["src"]},
+        "stages_ms": {n: round(v, 4) for n, v in zip(["quantize", "route", "gather", "w13", "w2", "combine"], stage)},
+        "w2": {"achieved_tflops": round(w2_tf, 1), "frac": round(w2_tf / fp4_peak, 4)},
+        "quantize": {"achieved_gbs": round(q_gbs, 1), "peak_gbs": peaks["hbm"], "frac": round(q_gbs / peaks["hbm"], 4),
+                     "algorithmic_bytes": q_bytes, "note": "dynamic g: amax pass + quantize pass, 2.5625 B/elem counted"},
+        "weight_stream": {"touched_bytes": b.touched_weight_bytes(),
+                          "gbs_layer": round(b.touched_weight_bytes() / (ms * 1e-3) / 1e9, 1)},
+        "e2e": {"value": round(world * flops / (e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "ms_per_step": round(e_ms, 4),
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": MoeBench.LAUNCHES_PER_STEP * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_moe(b)
+    return line
+
+
+def cpu_baseline_moe(b, n_tokens=1):
+    """The oracle as it stands on a bounded sample: `n_tokens` tokens with all
+    of their top-k experts; the oracle quantizes and dequantizes each touched
+    expert's bf16 weights itself (MX then remap for the Flash workload).
+    Inputs are copied to the host before the clock starts."""
+    import numpy as np
+
+    import synth
+    from oracle import moe as MO
+    from oracle import quant as Q
+
+    sigma = WORKLOADS[b.name][6]
+    g = Q.nv_global_scale(b.x.float().abs().amax().reshape(1, 1).cpu().numpy())
+    xs = b.x[:n_tokens].float().cpu().numpy()
+    ids = b.ids[:n_tokens].cpu().numpy()
+    hg = b.h_g.cpu().numpy()
+    wts = b.w[:n_tokens].cpu().numpy().astype(np.float64)
+    experts = sorted(set(int(e) for e in ids.reshape(-1)))
+    wb = {}
+    for e in experts:
+        w13 = synth.weights_bf16((2 * b.I, b.H), sigma, 0.005, 30.0, seed=1000 * 2 + e, device="cuda")
+        w2 = synth.weights_bf16((b.H, b.I), sigma, 0.005, 30.0, seed=1000 * 3 + e, device="cuda")
+        wb[e] = (w13.float().cpu().numpy(), w2.float().cpu().numpy())
+
+    def deq(w):
+        if b.name == "flash":
+            c, sc = Q.mxfp4_quantize(w)
+            sf, gg = Q.mx_to_nv(c, sc, 1)
+            return Q.nvfp4_dequantize(c, sf, gg[0])
+        return Q.nvfp4_dequantize(*Q.nvfp4_quantize(w))
+
+    t0 = time.perf_counter()
+    x_dq = Q.nvfp4_dequantize(*Q.nvfp4_quantize(xs, g=g))
+    dq = {e: (MO.deinterleave_w13(deq(wb[e][0])), deq(wb[e][1])) for e in experts}
+    out = np.zeros((n_tokens, b.H))
+    for t in range(n_tokens):
+        for s in range(b.k):
+            e = int(ids[t, s])
+            (w1d, w3d), w2d = dq[e]
+            r = MO.expert_ffn_ref(x_dq[t:t + 1], w1d, w3d, w2d, hg[e])
+            out[t] += wts[t, s] * r["y"][0]
+    dt = time.perf_counter() - t0
+    flops = 2.0 * 3 * b.H * b.I * b.k * n_tokens
+    return {"value": round(flops / dt / 1e12, 9), "unit": "TFLOP/s", "cores": len(os.sched_getaffinity(0)),
+            "kind": "oracle",
+            "sample": f"{n_tokens} token(s) x top-{b.k} experts of the same layer, including the oracle's own"
+                      f" quantize/dequantize of the {len(experts)} touched experts' weights: {dt:.1f} s"}
+
+
+# ---------------------------------------------------------------------------
+def run_dense(args, world, rank, peaks):
+    import torch
+
+    import fp4_block_scaled_03_b200 as fp4
+    import synth
+
+    M = N = K = 4096
+    a_bf = synth.activations_bf16((M, K), seed=rank, device="cuda")
+    b_bf = synth.weights_bf16((N, K), 0.02, 0.005, 30.0, seed=rank + 1, device="cuda")
+    b_c, b_sf, b_g = fp4.quantize_nv(b_bf, tiled=True)
+    a_c = torch.empty((M, K // 2), dtype=torch.uint8, device="cuda")
+    a_sf = torch.empty(fp4.fp4_sf_tiled_bytes(M, K), dtype=torch.uint8, device="cuda")
+    a_g = torch.empty(1, dtype=torch.float32, device="cuda")
+    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    c = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+
+    def step(ev=None):
+        if ev:
+            ev[0].record()
+        fp4.fp4_quantize(fp4.FP4_NV, a_bf, M, K, K, a_c, a_sf, a_g, fp4.FP4_SCALE_LAYOUT_TILED, ws, 256)
+        if ev:
+            ev[1].record()
+        fp4.fp4_gemm(a_c, a_sf, a_g, b_c, b_sf, b_g, c, fp4.FP4_OUT_BF16, M, N, K)
+        if ev:
+            ev[2].record()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    barrier(world)
+    tot = 0.0
+    q = g = 0.0
+    for i in range(args.steps):
+        flush.zero_()  # L2 flush between timed iterations (256 MB > 126 MB L2)
+        torch.cuda.synchronize()
+        step(evs[i])
+        torch.cuda.synchronize()
+        q += evs[i][0].elapsed_time(evs[i][1])
+        g += evs[i][1].elapsed_time(evs[i][2])
+        tot += evs[i][0].elapsed_time(evs[i][2])
+    clocks = sampler.stop() if sampler else None
+    ms = max_over_ranks(tot / args.steps, world)
+    gms = g / args.steps
+    flops = 2.0 * M * N * K
+    fp4_peak = 4.0 * peaks["bf16"]
+    return {
+        "metric": METRIC, "value": round(world * flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e2m1, e4m3/16 scales, fp32 accumulate)",
+        "data": "synthetic (seeded)",
+        "config": {"workload": "Dense NVFP4 W4A4 GEMM 4096x4096x4096, activations quantized on device each call, bf16 out",
+                   "l2": "flushed (256 MB write) before each timed step"},
+        "roofline": {"bound": "tensor", "kernel": "fp4_gemm_kernel<256, bf16>", "achieved": round(flops / (gms * 1e-3) / 1e12, 1),
+                     "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(flops / (gms * 1e-3) / 1e12 / fp4_peak, 4),
+                     "traffic": None, "peak_note": "4 x measured burst bf16 cuBLAS, of " + peaks["src"]},
+        "stages_ms": {"quantize": round(q / args.steps, 4), "gemm": round(gms, 4)},
+        "gpu_launches": 3 * args.steps, "clocks": clocks,
+    }
+
+
+def run_quant(args, world, rank, peaks):
+    import torch
+
+    import fp4_block_scaled_03_b200 as fp4
+    import synth
+
+    H = 7168
+    res = []
+    for T in [1024 * 2**i for i in range(8)]:
+        x = synth.activations_bf16((T, H), seed=T, device="cuda")
+        c = torch.empty((T, H // 2), dtype=torch.uint8, device="cuda")
+        s = torch.empty((T, H // 16), dtype=torch.uint8, device="cuda")
+        g = torch.tensor([1.0 / 448], dtype=torch.float32, device="cuda")
+        gd = torch.empty(1, dtype=torch.float32, device="cuda")
+        ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+        out = {}
+        for mode, flags, gg in (("static", fp4.FP4_STATIC_GLOBAL_SCALE, g), ("dynamic", 0, gd)):
+            for _ in range(args.warmup):
+                fp4.fp4_quantize(fp4.FP4_NV, x, T, H, H, c, s, gg, flags, ws, 256)
+            times = []
+            for _ in range(args.steps):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                fp4.fp4_quantize(fp4.FP4_NV, x, T, H, H, c, s, gg, flags, ws, 256)
+                e1.record()
+                torch.cuda.synchronize()
+                times.append(e0.elapsed_time(e1))
+            ms = sorted(times)[len(times) // 2]
+            out[mode] = round(T * H * 2.5625 / (ms * 1e-3) / 1e9, 1)
+        res.append({"T": T, "static_gbs": out["static"], "dynamic_gbs": out["dynamic"]})
+        del x, c, s, flush
+    top = res[-1]
+    return {"metric": METRIC, "value": top["static_gbs"], "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16 -> nvfp4", "data": "synthetic N(0,1)",
+            "config": {"workload": "NVFP4 activation quantize bf16 [T,7168], T=1k..128k", "l2": "flushed"},
+            "roofline": {"bound": "hbm", "achieved": top["static_gbs"], "peak": peaks["hbm"], "unit": "GB/s",
+                         "frac": round(top["static_gbs"] / peaks["hbm"], 4), "traffic": None},
+            "sweep": res, "gpu_launches": None}
+
+
+# ---------------------------------------------------------------------------
+def run_reference(args, world, rank):
+    """The oracle on the host cores, same workload, bounded sample per step."""
+    if rank != 0:
+        return None
+    import torch
+
+    import synth  # noqa: F401
+
+    t_all = []
+    b = None
+    if args.workload in WORKLOADS and torch.cuda.is_available():
+        b = MoeBench(args.workload, seed=0)
+    res = None
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        if b is not None:
+            res = cpu_baseline_moe(b, n_tokens=1)
+        else:
+            res = cpu_dense_sample()
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            t_all.append(res["value"])
+    v = sum(t_all) / len(t_all)
+    return {"metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": None, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded)", "impl": "reference",
+            "config": {"workload": WORKLOADS[args.workload][-1] if args.workload in WORKLOADS else args.workload},
+            "cpu_baseline": dict(res, value=v),
+            "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def cpu_dense_sample(rows=64):
+    import numpy as np
+
+    import synth
+    from oracle import gemm as G
+    from oracle import quant as Q
+
+    t0 = time.perf_counter()
+    a = synth.activations_bf16((rows, 4096), seed=0).float().numpy()
+    b = synth.weights_bf16((4096, 4096), 0.02, 0.005, 30.0, seed=1).float().numpy()
+    G.nvfp4_gemm_ref(*Q.nvfp4_quantize(a), *Q.nvfp4_quantize(b))
+    dt = time.perf_counter() - t0
+    return {"value": 2.0 * rows * 4096 * 4096 / dt / 1e12, "unit": "TFLOP/s", "cores": len(os.sched_getaffinity(0)),
+            "kind": "oracle", "sample": f"{rows} rows of the 4096^3 GEMM, {dt:.1f} s"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="pro", choices=list(WORKLOADS) + ["dense4096", "quant"])
+    ap.add_argument("--impl", default="fp4", choices=["fp4", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = setup_dist(args)
+    peaks = load_peaks()
+    if args.impl == "reference":
+        line = run_reference(args, world, rank)
+    elif args.workload in WORKLOADS:
+        line = run_moe(args, world, rank, peaks)
+    elif args.workload == "dense4096":
+        line = run_dense(args, world, rank, peaks)
+    else:
+        line = run_quant(args, world, rank, peaks)
+    if rank == 0 and line is not None:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -227,12 +227,15 @@ def quantize_mx(x):
     return codes, scales
 
 
-def mx_to_nv(codes, mx_scales, num_tensors):
+def mx_to_nv(codes, mx_scales, num_tensors, tiled=False):
     total_rows, half = codes.shape
     rows, cols = total_rows // num_tensors, half * 2
-    nv = torch.empty((total_rows, cols // 16), dtype=torch.uint8, device=codes.device)
+    if tiled:
+        nv = _u8(num_tensors * fp4_sf_tiled_bytes(rows, cols), codes.device)
+    else:
+        nv = torch.empty((total_rows, cols // 16), dtype=torch.uint8, device=codes.device)
     g = torch.empty(num_tensors, dtype=torch.float32, device=codes.device)
-    fp4_mx_to_nv(codes, mx_scales, rows, cols, num_tensors, nv, g)
+    fp4_mx_to_nv(codes, mx_scales, rows, cols, num_tensors, nv, g, FP4_SCALE_LAYOUT_TILED if tiled else 0)
     return nv, g
 
 

@@ -150,15 +150,16 @@ __device__ __forceinline__ float pow2_f32(int e) {  // exact 2^e, e in [-149, 12
   return __uint_as_float(1u << (e + 149));
 }
 
+template <bool kTiled>
 __global__ void __launch_bounds__(kThreads) mx_to_nv_kernel(const uint8_t *__restrict__ codes,
                                                             const uint8_t *__restrict__ mx, int64_t rows,
                                                             int64_t cols, uint8_t *__restrict__ nv,
-                                                            float *__restrict__ nv_global) {
+                                                            float *__restrict__ nv_global, int64_t tiled_bytes) {
   const int64_t t = blockIdx.x;
   const int64_t nb = rows * (cols / 32);
   const uint8_t *cb = codes + t * rows * (cols / 2);
   const uint8_t *sb = mx + t * nb;
-  uint8_t *ob = nv + t * rows * (cols / 16);
+  uint8_t *ob = nv + (kTiled ? t * tiled_bytes : t * rows * (cols / 16));
   int emax = -1000, emin = 1000, bad = 0;
   for (int64_t i = threadIdx.x; i < nb; i += blockDim.x) {
     const uint4 c = *reinterpret_cast<const uint4 *>(cb + i * 16);
@@ -198,7 +199,12 @@ __global__ void __launch_bounds__(kThreads) mx_to_nv_kernel(const uint8_t *__res
       const int k = ((int)sb[i] - 127) - emax + 8;  // in [-9, 8]
       code = k >= -6 ? (uint32_t)((k + 7) << 3) : (1u << (k + 9));
     }
-    *reinterpret_cast<uint16_t *>(ob + 2 * i) = (uint16_t)(code | (code << 8));
+    if (kTiled) {  // block i = (row, 32-block j): 16-blocks 2j and 2j+1 are adjacent bytes
+      const int64_t r = i / (cols / 32), j = i - r * (cols / 32);
+      *reinterpret_cast<uint16_t *>(ob + sf_tiled_offset(r, 2 * j, cols / 64)) = (uint16_t)(code | (code << 8));
+    } else {
+      *reinterpret_cast<uint16_t *>(ob + 2 * i) = (uint16_t)(code | (code << 8));
+    }
   }
 }
 
@@ -253,14 +259,19 @@ fp4_status fp4_quantize(fp4_format fmt, const void *x_bf16, int64_t rows, int64_
 fp4_status fp4_mx_to_nv(const uint8_t *codes, const uint8_t *mx_scales, int64_t rows, int64_t cols,
                         int64_t num_tensors, uint8_t *nv_scales, float *nv_global, uint32_t flags,
                         fp4_stream_t stream) {
-  (void)flags;
   if (!codes || !mx_scales || !nv_scales || !nv_global || rows <= 0 || cols <= 0 || num_tensors <= 0)
     return FP4_ERR_INVALID_ARG;
-  if (cols % 32) return FP4_ERR_UNSUPPORTED_SHAPE;
+  const bool tiled = flags & FP4_SCALE_LAYOUT_TILED;
+  if (cols % 32 || (tiled && cols % 64)) return FP4_ERR_UNSUPPORTED_SHAPE;
   if (!aligned16(codes) || (reinterpret_cast<uintptr_t>(nv_scales) & 1u)) return FP4_ERR_ALIGNMENT;
   if (num_tensors > 2147483647) return FP4_ERR_UNSUPPORTED_SHAPE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  mx_to_nv_kernel<<<(unsigned)num_tensors, kThreads, 0, s>>>(codes, mx_scales, rows, cols, nv_scales, nv_global);
+  if (tiled)
+    mx_to_nv_kernel<true><<<(unsigned)num_tensors, kThreads, 0, s>>>(codes, mx_scales, rows, cols, nv_scales, nv_global,
+                                                                    (int64_t)fp4_sf_tiled_bytes(rows, cols));
+  else
+    mx_to_nv_kernel<false><<<(unsigned)num_tensors, kThreads, 0, s>>>(codes, mx_scales, rows, cols, nv_scales,
+                                                                     nv_global, 0);
   FP4_HOST_CHECK(cudaGetLastError());
   // offline step: report refused tensors (NaN globals) synchronously
   FP4_HOST_CHECK(cudaStreamSynchronize(s));

@@ -115,9 +115,11 @@ fp4_status fp4_quantize(fp4_format fmt, const void *x_bf16, int64_t rows, int64_
  * uint8 [num_tensors*rows][cols/2], mx_scales UE8M0 [..][cols/32]).  Per
  * tensor: e_max = the largest MX exponent among blocks holding a nonzero
  * magnitude code; nv_global[t] = 2^(e_max-8); each such block's E4M3 scale
- * is 2^(e - e_max + 8), written to both of its 16-element halves
- * (nv_scales canonical [..][cols/16]); blocks of zeros get scale 0.  Codes
- * are not touched (they are identical in both formats).
+ * is 2^(e - e_max + 8), written to both of its 16-element halves; blocks of
+ * zeros get scale 0.  nv_scales: canonical [num_tensors*rows][cols/16], or
+ * with FP4_SCALE_LAYOUT_TILED (cols % 64 == 0) one tiled buffer per tensor,
+ * tensor t at byte offset t * fp4_sf_tiled_bytes(rows, cols).  Codes are not
+ * touched (they are identical in both formats).
  * A tensor whose live exponents span more than 17 octaves (or holds a UE8M0
  * NaN byte) cannot be remapped exactly: its scales are left untouched and its
  * nv_global is set to NaN.  This call is an offline weight-preparation step

@@ -1,0 +1,78 @@
+"""Builds one seeded MoE test case on the GPU (through the library) and its
+oracle mirror on the host (through oracle/ only, from the same bf16 inputs).
+
+Weights: w13 [E, 2I, H] bf16 drawn directly in the fused order (rows 32j..32j+15
+are gate rows, 32j+16..32j+31 up rows), w2 [E, H, I]; each expert's matrix is
+NVFP4-quantized with its own dynamic tensor scale (NV) or MXFP4-quantized and
+remapped (MX)."""
+import numpy as np
+import torch
+
+import synth
+from oracle import moe as MO
+from oracle import quant as Q
+from tests._util import f32
+
+
+class Case:
+    pass
+
+
+def build(T, H, I, E, k, seed=0, zipf=0.0, h_g=1e-3, w_sigma=0.02, w_frac=0.005, w_factor=30.0, fmt="nv",
+          oracle_experts=None):
+    import fp4_block_scaled_03_b200 as fp4
+
+    c = Case()
+    c.T, c.H, c.I, c.E, c.k = T, H, I, E, k
+    dev = "cuda"
+    c.x = synth.activations_bf16((T, H), seed=seed, device=dev)
+    c.ids, c.w, c.counts = synth.router(T, E, k, seed=seed + 1, zipf_s=zipf, device=dev)
+    w13 = synth.weights_bf16((E * 2 * I, H), w_sigma, w_frac, w_factor, seed=seed + 2, device=dev)
+    w2 = synth.weights_bf16((E * H, I), w_sigma, w_frac, w_factor, seed=seed + 3, device=dev)
+    c.w13_codes = torch.empty((E * 2 * I, H // 2), dtype=torch.uint8, device=dev)
+    c.w2_codes = torch.empty((E * H, I // 2), dtype=torch.uint8, device=dev)
+    c.w13_sf = torch.empty(fp4.fp4_sf_tiled_bytes(E * 2 * I, H), dtype=torch.uint8, device=dev)
+    c.w2_sf = torch.empty(fp4.fp4_sf_tiled_bytes(E * H, I), dtype=torch.uint8, device=dev)
+    c.w13_g = torch.empty(E, dtype=torch.float32, device=dev)
+    c.w2_g = torch.empty(E, dtype=torch.float32, device=dev)
+    s13 = fp4.fp4_sf_tiled_bytes(2 * I, H)
+    s2 = fp4.fp4_sf_tiled_bytes(H, I)
+    for e in range(E):
+        for (wb, codes, sf, g, rows, cols, sfb) in ((w13, c.w13_codes, c.w13_sf, c.w13_g, 2 * I, H, s13),
+                                                     (w2, c.w2_codes, c.w2_sf, c.w2_g, H, I, s2)):
+            sl = slice(e * rows, (e + 1) * rows)
+            if fmt == "nv":
+                cc, ss, gg = fp4.quantize_nv(wb[sl], tiled=True)
+                codes[sl] = cc
+                sf[e * sfb:(e + 1) * sfb] = ss
+                g[e] = gg[0]
+            else:
+                raise ValueError(fmt)
+    c.h_g = torch.full((E,), h_g, dtype=torch.float32, device=dev)
+    c.weights = fp4.MoeWeightSet(c.w13_codes, c.w13_sf, c.w13_g, c.w2_codes, c.w2_sf, c.w2_g, c.h_g)
+    # host copies for the oracle
+    c.x_f32 = f32(c.x)
+    c.ids_np = c.ids.cpu().numpy()
+    c.w_np = c.w.cpu().numpy()
+    c.w13_bf = w13
+    c.w2_bf = w2
+    c.h_g_np = np.full(E, np.float32(h_g), dtype=np.float32)
+    return c
+
+
+def oracle_expert_weights(c, e):
+    """Dequantized fp64 (W1 [I,H], W3 [I,H], W2 [H,I]) of expert e, quantized
+    by the oracle from the same bf16 weights."""
+    I, H = c.I, c.H
+    w13 = f32(c.w13_bf[e * 2 * I:(e + 1) * 2 * I])
+    w2 = f32(c.w2_bf[e * H:(e + 1) * H])
+    q13 = Q.nvfp4_quantize(w13)
+    q2 = Q.nvfp4_quantize(w2)
+    d13 = Q.nvfp4_dequantize(*q13)
+    w1, w3 = MO.deinterleave_w13(d13)
+    return w1, w3, Q.nvfp4_dequantize(*q2), q13, q2
+
+
+def oracle_x(c):
+    xq = Q.nvfp4_quantize(c.x_f32)
+    return xq, Q.nvfp4_dequantize(*xq)

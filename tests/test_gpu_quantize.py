@@ -138,3 +138,17 @@ def test_remap_refuses_wide_span():
     assert gh[0] == np.float32(2.0**-8) and np.isnan(gh[1])
     assert torch.all(nv[rows:] == 0xAB)  # the refused tensor's scales are untouched
     assert fp4.fp4_get_device_status() == 0
+
+
+def test_remap_tiled_layout():
+    nt, rows, cols = 3, 64, 192  # rows not a multiple of 128: each tensor padded on its own
+    w = synth.weights_bf16((nt * rows, cols), 0.02, 0.005, 30.0, seed=12, device="cuda")
+    codes, sc = _lib().quantize_mx(w)
+    nv_t, g = _lib().mx_to_nv(codes, sc, nt, tiled=True)
+    rc, rs = Q.mxfp4_quantize(f32(w))
+    rnv, rg = Q.mx_to_nv(rc, rs, nt)
+    tb = _lib().fp4_sf_tiled_bytes(rows, cols)
+    for t in range(nt):
+        got = LY.sf_from_mma(np_u8(nv_t[t * tb:(t + 1) * tb]), rows, cols)
+        assert np.array_equal(got, rnv[t * rows:(t + 1) * rows])
+    assert f32_bits_equal(g.cpu().numpy(), rg)
