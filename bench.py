@@ -39,6 +39,8 @@ WORKLOADS = {
     "flash": (4096, 4096, 2048, 256, 6, 0.0, 0.02,
               "Flash-shaped MoE layer: hidden 4096, 256 experts, I 2048, top-6 uniform, 4096 tokens, MX weights remapped"),
     "decode": (64, 7168, 2048, 384, 6, 1.1, 0.01, "Pro-shaped MoE layer at 64 decode tokens (weight-read bound)"),
+    "pro64": (4096, 7168, 2048, 64, 6, 1.1, 0.01,
+              "Pro-shaped expert matrices, 64 experts, 4096 tokens, top-6, Zipf 1.1 (profiling size)"),
 }
 
 METRIC = "NVFP4 W4A4 grouped-MoE GEMM TFLOPS (% FP4 peak); quantize GB/s (% HBM)"
@@ -282,11 +284,13 @@ def run_moe(args, world, rank, peaks):
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.profiler.start()  # a profiler attached with capture off sees only the timed steps
     t0.record(stream)
     for i in range(args.steps):
         b.step(events=evs[i])
     t1.record(stream)
     torch.cuda.synchronize()
+    torch.cuda.profiler.stop()
     barrier(world)
     clocks = sampler.stop() if sampler else None
     assert fp4.fp4_get_device_status() == 0

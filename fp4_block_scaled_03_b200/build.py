@@ -1,6 +1,6 @@
 """Build libfp4.so in-tree for sm_100a with nvcc (no GPU needed to build).
 
-    python -m fp4_block_scaled_03_b200.build [-v]
+    python fp4_block_scaled_03_b200/build.py [-v] [--ptxas]
 
 Objects go to fp4_block_scaled_03_b200/_build/, the shared library to
 fp4_block_scaled_03_b200/libfp4.so.  A source is recompiled when it or any

@@ -111,7 +111,7 @@ def test_gather_bit_exact():
 
 def _band_quantize_check(h_ref, tol, g, codes_gpu, sf_gpu):
     """h_ref, tol: fp64 [n, 16*nb]; codes_gpu unpacked [n, 16*nb]; sf_gpu [n, nb].
-    Returns (n_exact_blocks, n_band_blocks, ok) where a block is 'stable' if
+    Returns (n_differing_blocks, n_band_blocks, ok) where a block is 'stable' if
     every value in [h-tol, h+tol] quantizes like h itself (checked at both
     band ends for the scale and for every element)."""
     n, cols = h_ref.shape
@@ -141,7 +141,7 @@ def _band_quantize_check(h_ref, tol, g, codes_gpu, sf_gpu):
     stable = (sf_lo == sf_hi) & (v_lo == v_hi).reshape(n, nb, 16).all(2)
     exact = (sf_gpu == s_mid) & (v_gpu == F.e2m1_decode(c_mid)).reshape(n, nb, 16).all(2)
     ok = np.where(stable, exact, sf_ok & el_ok.reshape(n, nb, 16).all(2))
-    return int(stable.sum()), int((~stable).sum()), ok
+    return int((~exact).sum()), int((~stable).sum()), ok
 
 
 def _run_stages(c, dump=True):
@@ -172,7 +172,7 @@ def test_w13_swiglu_requant(T, H, I, E, k, zipf):
     h_dump = out["h_d"].cpu().numpy()
     h_codes = F.unpack_nibbles(np_u8(out["h_c"]))
     h_sf = LY.sf_from_mma(np_u8(out["h_s"]), out["cap"], I)
-    total_band = 0
+    total_diff = 0
     for e in range(E):
         if counts[e] == 0:
             continue
@@ -185,10 +185,12 @@ def test_w13_swiglu_requant(T, H, I, E, k, zipf):
         prow = toff[e] * 128 + np.arange(counts[e])
         err = np.abs(h_dump[prow] - h)
         assert np.all(err <= tol), (e, float((err / tol).max()))
-        n_st, n_band, ok = _band_quantize_check(h, tol, c.h_g_np[e], h_codes[prow], h_sf[prow])
+        n_diff, n_band, ok = _band_quantize_check(h, tol, c.h_g_np[e], h_codes[prow], h_sf[prow])
         assert ok.all(), (e, int((~ok).sum()))
-        total_band += n_band
-    assert total_band <= 0.01 * (T * k * I // 16) + 8
+        total_diff += n_diff
+    # blocks whose codes differ from the oracle's own rounding of h (allowed
+    # only inside the band, checked above) stay rare
+    assert total_diff <= 0.01 * (T * k * I // 16) + 8, total_diff
 
 
 def test_w2_weighted_rows():
