@@ -81,6 +81,7 @@ _SIGS = {
     ),
     "fp4_moe_route_scratch_bytes": (_SZ, [_I64, _I32]),
     "fp4_moe_route": (ctypes.c_int, [_P, _I64, _I32, _I32, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "fp4_moe_route_noalloc": (ctypes.c_int, [_P, _I64, _I32, _I32, _P, _P, _P, _P, _P, _P]),
     "fp4_moe_gather": (ctypes.c_int, [_P, _P, _I64, _I32, _I64, _I32, _P, _P, _P, _P, _P, _I64, _P]),
     "fp4_moe_w13": (
         ctypes.c_int,
@@ -141,6 +142,13 @@ def fp4_moe_route(expert_ids, T, topk, E, counts, offsets, tile_offsets, perm, i
     _check(lib.fp4_moe_route(_ptr(expert_ids), T, topk, E, _ptr(counts), _ptr(offsets), _ptr(tile_offsets),
                              _ptr(perm), _ptr(inv), _ptr(scratch), scratch.numel() * scratch.element_size(),
                              _stream()), "fp4_moe_route")
+
+
+def fp4_moe_route_noalloc(expert_ids, T, topk, E, counts, offsets, tile_offsets, perm, inv):
+    """Routing for callers that cannot allocate device memory: the library's
+    own 1 MiB per-device scratch array replaces the scratch argument."""
+    _check(lib.fp4_moe_route_noalloc(_ptr(expert_ids), T, topk, E, _ptr(counts), _ptr(offsets), _ptr(tile_offsets),
+                                     _ptr(perm), _ptr(inv), _stream()), "fp4_moe_route_noalloc")
 
 
 def fp4_moe_gather(x_codes, x_sf, T, topk, H, E, offsets, tile_offsets, perm, a_codes, a_sf, rows_cap):

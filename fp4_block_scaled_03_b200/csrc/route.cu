@@ -6,6 +6,8 @@
 // token, slot) order -- a stable counting sort of the flattened expert ids --
 // so each expert's rows are contiguous; each expert's block of rows is padded
 // to a multiple of 128 (the GEMM's M tile).
+#include <mutex>
+
 #include "common.cuh"
 
 namespace fp4 {
@@ -193,6 +195,31 @@ int sm_count() {
 
 bool al16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Scratch of fp4_moe_route_noalloc: the per-chunk expert counts live in this
+// module array (1 MiB on every device that loads the library, kept until the
+// process exits) instead of a caller buffer.
+constexpr size_t kNoAllocRouteScratchBytes = size_t(1) << 20;
+static __device__ __align__(256) int32_t g_route_scratch[kNoAllocRouteScratchBytes / 4];
+
+// The array's name is a host-side stand-in in host code; the device address
+// comes from cudaGetSymbolAddress, taken once per device with that device
+// current and cached.
+std::mutex g_noalloc_mu;
+int32_t *g_noalloc_scratch[64];
+
+fp4_status noalloc_route_scratch(int32_t **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FP4_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_scratch[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || !p) return FP4_ERR_CUDA;
+    g_noalloc_scratch[dev] = static_cast<int32_t *>(p);
+  }
+  *out = g_noalloc_scratch[dev];
+  return FP4_OK;
+}
+
 }  // namespace
 }  // namespace fp4
 
@@ -269,6 +296,26 @@ fp4_status fp4_moe_combine(const float *y, const int32_t *inv, int64_t T, int32_
   combine_kernel<<<(unsigned)grid, 256, 0, s>>>(y, inv, T, topk, H, static_cast<__nv_bfloat16 *>(out_bf16));
   FP4_HOST_CHECK(cudaGetLastError());
   return FP4_OK;
+}
+
+// Routing with no scratch argument, for callers that cannot allocate device
+// memory.  The chunk-count scratch is the module array above: every call on a
+// device shares it, so calls whose kernels overlap on the GPU (different
+// streams without ordering) race and must not be issued.  Nothing in the
+// array has to start at zero: the counting pass writes every entry the later
+// passes read.  The first call on a device looks up the array's address
+// (cudaGetSymbolAddress); make that first call before any stream capture.
+fp4_status fp4_moe_route_noalloc(const int32_t *expert_ids, int64_t T, int32_t topk, int32_t E, int32_t *counts,
+                                 int32_t *offsets, int32_t *tile_offsets, int32_t *perm, int32_t *inv,
+                                 fp4_stream_t stream) {
+  if (!expert_ids || !counts || !offsets || !tile_offsets || !perm || !inv) return FP4_ERR_INVALID_ARG;
+  if (T < 0 || topk < 1 || topk > 16 || E < 1 || E > 4096) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (fp4_moe_route_scratch_bytes(T * topk, E) > kNoAllocRouteScratchBytes) return FP4_ERR_WORKSPACE;
+  int32_t *scratch = nullptr;
+  const fp4_status st = noalloc_route_scratch(&scratch);
+  if (st != FP4_OK) return st;
+  return fp4_moe_route(expert_ids, T, topk, E, counts, offsets, tile_offsets, perm, inv, scratch,
+                       kNoAllocRouteScratchBytes, stream);
 }
 
 }  // extern "C"

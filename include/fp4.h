@@ -212,6 +212,22 @@ fp4_status fp4_moe_route(const int32_t *expert_ids, int64_t T, int32_t topk, int
                          int32_t *counts, int32_t *offsets, int32_t *tile_offsets, int32_t *perm,
                          int32_t *inv, void *scratch, size_t scratch_bytes, fp4_stream_t stream);
 
+/* fp4_moe_route without a scratch argument.  The pages have no counterpart:
+ * this entry point exists for callers that cannot allocate device memory --
+ * e.g. a runtime that reserves all of HBM for weights and caches up front and
+ * hands a kernel library only its inputs and outputs, or plain-C code with no
+ * device allocator at hand.  The scratch is a 1 MiB array inside the library
+ * (one per device that loads it, held until the process exits), so it
+ * accepts sizes with fp4_moe_route_scratch_bytes(T*topk, E) <= 1 MiB, i.e.
+ * ceil(T*topk/1024)*E <= 262144, and returns FP4_ERR_WORKSPACE beyond that
+ * without launching.  All calls on a device share the array: calls that
+ * overlap on the GPU race.  Its first call on a device looks up the array's
+ * device address; make that first call before any stream capture.  Outputs
+ * and errors are those of fp4_moe_route. */
+fp4_status fp4_moe_route_noalloc(const int32_t *expert_ids, int64_t T, int32_t topk, int32_t E,
+                                 int32_t *counts, int32_t *offsets, int32_t *tile_offsets,
+                                 int32_t *perm, int32_t *inv, fp4_stream_t stream);
+
 /* Gather token rows into expert-contiguous, 128-padded rows: a_codes
  * [rows_cap][H/2], a_sf tiled for [rows_cap, H]; x_sf canonical [T][H/16].
  * rows_cap >= 128*tile_offsets[E] (T*topk + 127*E always suffices). */

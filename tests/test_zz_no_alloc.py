@@ -1,0 +1,77 @@
+"""The allocation-free routing entry point, fp4_moe_route_noalloc.
+
+Some callers cannot allocate device memory (a runtime that has reserved all
+of HBM for weights and caches and gives a kernel library only its inputs and
+outputs, or plain-C code with no device allocator).  For them the library
+keeps the routing scratch in its own 1 MiB per-device array.  This test calls
+that entry point through the C ABI and checks that it routes exactly like
+fp4_moe_route with a caller-provided scratch buffer, on two calls in a row
+(the second call reuses the array the first one left behind), and that a size
+beyond the array is refused on the host.  This file is collected last.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def _tables(T, k, E):
+    d = "cuda"
+    R = T * k
+    return dict(counts=torch.full((E,), -9, dtype=torch.int32, device=d),
+                offsets=torch.full((E + 1,), -9, dtype=torch.int32, device=d),
+                tile_offsets=torch.full((E + 1,), -9, dtype=torch.int32, device=d),
+                perm=torch.full((R,), -9, dtype=torch.int32, device=d),
+                inv=torch.full((R,), -9, dtype=torch.int32, device=d))
+
+
+def _route_with_scratch(fp4, ids, T, k, E):
+    t = _tables(T, k, E)
+    scratch = torch.empty(fp4.fp4_moe_route_scratch_bytes(T * k, E), dtype=torch.uint8, device="cuda")
+    fp4.fp4_moe_route(ids, T, k, E, t["counts"], t["offsets"], t["tile_offsets"], t["perm"], t["inv"], scratch)
+    return t
+
+
+def _route_noalloc_cabi(fp4, ids, T, k, E):
+    t = _tables(T, k, E)
+    fn = fp4.lib.fp4_moe_route_noalloc  # the C entry point itself
+    st = fn(ctypes.c_void_p(ids.data_ptr()), T, k, E, ctypes.c_void_p(t["counts"].data_ptr()),
+            ctypes.c_void_p(t["offsets"].data_ptr()), ctypes.c_void_p(t["tile_offsets"].data_ptr()),
+            ctypes.c_void_p(t["perm"].data_ptr()), ctypes.c_void_p(t["inv"].data_ptr()),
+            ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 0, fp4.STATUS.get(st, st)
+    return t
+
+
+def test_noalloc_route_matches_route_on_two_calls():
+    import fp4_block_scaled_03_b200 as fp4
+
+    for T, k, E, seed, zipf in [(16384, 6, 384, 1, 1.1), (777, 8, 64, 2, 0.0)]:
+        ids, _, _ = synth.router(T, E, k, seed=seed, zipf_s=zipf, device="cuda")
+        ref = _route_with_scratch(fp4, ids, T, k, E)
+        got = _route_noalloc_cabi(fp4, ids, T, k, E)
+        torch.cuda.synchronize()
+        for name in ref:
+            assert np.array_equal(got[name].cpu().numpy(), ref[name].cpu().numpy()), name
+    assert fp4.fp4_get_device_status() == 0
+
+
+def test_noalloc_route_refuses_sizes_beyond_its_array():
+    import fp4_block_scaled_03_b200 as fp4
+
+    # ceil(T*k/1024) * E = 1025 * 256 entries > 262144: refused before any launch
+    T, k, E = 1025 * 1024 // 8, 8, 256
+    ids = torch.zeros((1, 1), dtype=torch.int32, device="cuda")
+    t = _tables(1, 1, E)
+    st = fp4.lib.fp4_moe_route_noalloc(ctypes.c_void_p(ids.data_ptr()), T, k, E, ctypes.c_void_p(t["counts"].data_ptr()),
+                                       ctypes.c_void_p(t["offsets"].data_ptr()),
+                                       ctypes.c_void_p(t["tile_offsets"].data_ptr()),
+                                       ctypes.c_void_p(t["perm"].data_ptr()), ctypes.c_void_p(t["inv"].data_ptr()),
+                                       ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 6  # FP4_ERR_WORKSPACE
+    assert torch.all(t["counts"] == -9)  # nothing was launched
