@@ -10,18 +10,24 @@
 //               B tile (packed codes, 128-byte swizzle) plus their scale tiles
 //               (bulk copies of the tiled scale layout) into a ring of shared
 //               memory stages, completing on the stage's "full" mbarrier.
-//   warp 1      allocates tensor memory; one lane copies each stage's scale
-//               tiles shared -> TMEM (tcgen05.cp) and issues 4 MMAs of
-//               K = 64, then commits to the stage's "empty" barrier; after
-//               the last K stage it commits to "acc_full".
-//   warps 2-5   epilogue: tcgen05.ld of the 128 x BN fp32 accumulator (each
-//               thread one row), then the fused output step for the caller:
+//   warp 2      scale copier: copies each stage's scale tiles shared -> TMEM
+//               (tcgen05.cp, into a TMEM slot per stage) and commits to the
+//               stage's "sf_full" barrier.  Kept off the MMA thread: each
+//               copy costs tens of cycles of issue, which would otherwise
+//               stall the MMA stream.
+//   warp 1      allocates tensor memory; one lane issues the stage's 4 MMAs of
+//               K = 64 with precomputed descriptors once the stage's data and
+//               scales are in place, then commits to the stage's "empty"
+//               barrier; after the last K stage it commits to "acc_full".
+//   warps 3-10  epilogue, two warps per 32-lane TMEM quarter, one per half
+//               of the tile's columns: tcgen05.ld of 128 fp32 columns into
+//               registers, arrive on "acc_empty" at once (the next tile's
+//               MMAs start while the stores run), then the fused output step:
 //                 dense    alpha * acc -> fp32 or bf16
 //                 w13      SwiGLU over interleaved 16-column gate/up groups,
 //                          then NVFP4 re-quantization of h with a static
 //                          per-expert scale (codes + tiled scales)
 //                 w2       routing weight * alpha * acc -> fp32 rows
-//               and arrives on "acc_empty".
 //
 // The grid is persistent (at most one CTA per SM); every role walks the same
 // tile sequence.  Grouped (MoE) tiles are (128-row tile of one expert's
@@ -37,7 +43,9 @@ namespace {
 
 constexpr int BM = 128;        // rows per tile (MMA M)
 constexpr int BK_BYTES = 128;  // one 128-byte swizzle row = 256 FP4 elements per stage
-constexpr int kThreads = 192;
+constexpr int kFirstEpiWarp = 3;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 32 * (kFirstEpiWarp + kEpiWarps);
 
 enum Epi { EPI_F32 = 0, EPI_BF16 = 1, EPI_W13 = 2, EPI_W2 = 3 };
 
@@ -52,11 +60,12 @@ struct Cfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
   static constexpr int TMEM_COLS = 512;
   static constexpr int ACC_COL = 0;
-  static constexpr int SFA_COL = 256;                 // 4 K-words x 4 columns
-  static constexpr int SFB_COL = 256 + 16;            // 4 K-words x 4*HALVES columns
+  static constexpr int SF_SLOT_COLS = 16 + 16 * HALVES;  // SFA: 4 K-words x 4; SFB: 4 x 4*HALVES
+  static constexpr int SF_COL0 = 256;                     // slot s at SF_COL0 + s * SF_SLOT_COLS
   static constexpr int SMEM_BYTES = kStages * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
-  static_assert(BN % 32 == 0 && BN <= 256, "BN");
-  static_assert(SFB_COL + 16 * HALVES <= TMEM_COLS, "tmem");
+  static_assert(BN == 256, "the early-release epilogue splits 256 columns into two halves");
+  static_assert(SF_COL0 + kStages * SF_SLOT_COLS <= TMEM_COLS, "tmem");
+  static_assert((3 * kStages + 4) * 8 <= 256, "barriers");
 };
 
 struct Params {
@@ -150,11 +159,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *smSFA = smB + C::kStages * C::B_BYTES;
   uint8_t *smSFB = smSFA + C::kStages * C::SFA_BYTES;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smSFB + C::kStages * C::SFB_BYTES);
-  uint64_t *full = bars;
-  uint64_t *empty = bars + C::kStages;
-  uint64_t *acc_full = bars + 2 * C::kStages;
-  uint64_t *acc_empty = acc_full + 1;
-  uint64_t *drain = acc_full + 2;
+  uint64_t *full = bars;                       // TMA data landed        (count 1 + tx)
+  uint64_t *empty = bars + C::kStages;         // MMAs done with a stage (tcgen05.commit)
+  uint64_t *sf_full = bars + 2 * C::kStages;   // stage scales in TMEM   (tcgen05.commit)
+  uint64_t *acc_full = bars + 3 * C::kStages;  // tile accumulated       (tcgen05.commit)
+  uint64_t *acc_empty = acc_full + 1;          // accumulator read out   (one per epilogue warp)
+  uint64_t *drain_mma = acc_full + 2;          // unwinding after an abort
+  uint64_t *drain_sf = acc_full + 3;
   __shared__ uint32_t s_tmem_base;
   __shared__ volatile int s_abort;
   __shared__ int s_total;
@@ -165,10 +176,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&sf_full[s], 1);
     }
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 4);
-    mbar_init(drain, 1);
+    mbar_init(acc_empty, kEpiWarps);
+    mbar_init(drain_mma, 1);
+    mbar_init(drain_sf, 1);
     fence_barrier_init();
     s_abort = 0;
     prefetch_tmap(&tmA);
@@ -224,6 +237,41 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (issued[s]) mbar_drain(&full[s], issued_par[s], 1000000000ull);
       }
     }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ scale copier
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true, any = false;
+      for (int t = blockIdx.x; ok && t < total; t += gridDim.x) {
+        for (int kt = 0; kt < p.k_stages; ++kt) {
+          if (!mbar_wait(&full[stage], phase, &s_abort, p.status, lim)) { ok = false; break; }
+          tc_fence_after();
+          const int nk = min(4, p.kw - kt * 4);
+          const uint32_t ta = tmem + C::SF_COL0 + stage * C::SF_SLOT_COLS;
+          const uint32_t tb = ta + 16;
+          // descriptors of the first 512-byte scale tile; tile i is +i*512 bytes (+i*32 in 16-byte units)
+          const uint64_t da = smem_desc(smem_u32(smSFA + stage * C::SFA_BYTES), 0, 128, 0);
+          const uint64_t db = smem_desc(smem_u32(smSFB + stage * C::SFB_BYTES), 0, 128, 0);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            if (j < nk) {
+              tmem_cp_sf(ta + j * 4, da + (uint64_t)(j * 32));
+#pragma unroll
+              for (int h = 0; h < C::HALVES; ++h)
+                tmem_cp_sf(tb + j * 4 * C::HALVES + h * 4, db + (uint64_t)((h * 4 + j) * 32));
+            }
+          }
+          any = true;
+          tc_commit(&sf_full[stage]);
+          if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok && any) {
+        tc_commit(drain_sf);
+        mbar_drain(drain_sf, 0, 1000000000ull);
+      }
+    }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -232,30 +280,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true, any_mma = false;
       const uint32_t t_acc = tmem + C::ACC_COL;
-      const uint32_t t_sfa = tmem + C::SFA_COL;
-      const uint32_t t_sfb = tmem + C::SFB_COL;
       for (int t = blockIdx.x; ok && t < total; t += gridDim.x) {
         if (!mbar_wait(acc_empty, acc_phase ^ 1u, &s_abort, p.status, lim)) { ok = false; break; }
         tc_fence_after();
         for (int kt = 0; kt < p.k_stages; ++kt) {
           if (!mbar_wait(&full[stage], phase, &s_abort, p.status, lim)) { ok = false; break; }
+          if (!mbar_wait(&sf_full[stage], phase, &s_abort, p.status, lim)) { ok = false; break; }
           tc_fence_after();
           const int nk = min(4, p.kw - kt * 4);
-          const uint32_t a_base = smem_u32(smA + stage * C::A_BYTES);
-          const uint32_t b_base = smem_u32(smB + stage * C::B_BYTES);
-          const uint32_t sfa_base = smem_u32(smSFA + stage * C::SFA_BYTES);
-          const uint32_t sfb_base = smem_u32(smSFB + stage * C::SFB_BYTES);
-          for (int j = 0; j < nk; ++j) {
-            tmem_cp_sf(t_sfa + j * 4, smem_desc(sfa_base + j * 512, 0, 128, 0));
+          const uint32_t ta = tmem + C::SF_COL0 + stage * C::SF_SLOT_COLS;
+          const uint32_t tb = ta + 16;
+          // K step j: +32 bytes inside the 128-byte swizzled rows (+2 in 16-byte units)
+          const uint64_t ad = smem_desc(smem_u32(smA + stage * C::A_BYTES), 16, 1024, 2);
+          const uint64_t bd = smem_desc(smem_u32(smB + stage * C::B_BYTES), 16, 1024, 2);
 #pragma unroll
-            for (int h = 0; h < C::HALVES; ++h)
-              tmem_cp_sf(t_sfb + j * 4 * C::HALVES + h * 4, smem_desc(sfb_base + (h * 4 + j) * 512, 0, 128, 0));
-          }
-          for (int j = 0; j < nk; ++j) {
-            const uint64_t ad = smem_desc(a_base + j * 32, 16, 1024, 2);
-            const uint64_t bd = smem_desc(b_base + j * 32, 16, 1024, 2);
-            mma_nvf4(t_acc, ad, bd, idesc, t_sfa + j * 4, t_sfb + j * 4 * C::HALVES, (kt > 0 || j > 0) ? 1u : 0u);
-          }
+          for (int j = 0; j < 4; ++j)
+            if (j < nk)
+              mma_nvf4(t_acc, ad + (uint64_t)(j * 2), bd + (uint64_t)(j * 2), idesc, ta + j * 4,
+                       tb + j * 4 * C::HALVES, (kt > 0 || j > 0) ? 1u : 0u);
           any_mma = true;
           tc_commit(&empty[stage]);
           if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
@@ -264,47 +306,54 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_commit(acc_full);
         acc_phase ^= 1u;
       }
-      if (!ok && any_mma) {  // wait for issued MMAs / copies before freeing TMEM
-        tc_commit(drain);
-        mbar_drain(drain, 0, 1000000000ull);
+      if (!ok && any_mma) {  // wait for issued MMAs before freeing TMEM
+        tc_commit(drain_mma);
+        mbar_drain(drain_mma, 0, 1000000000ull);
       }
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int q = warp & 3;                       // TMEM lane quarter this warp may access
+    const int half = (warp - kFirstEpiWarp) >> 2;  // which 128 columns of the tile
     const int row = q * 32 + lane;
+    constexpr int HC = BN / 2;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
       const TileInfo ti = tile_info<BN, kGrouped>(p, t);
       if (!mbar_wait(acc_full, acc_phase, &s_abort, p.status, lim)) break;
       tc_fence_after();
+      float v[HC];
+#pragma unroll
+      for (int c = 0; c < HC / 32; ++c) {
+        __syncwarp();
+        tmem_ld32(tmem + C::ACC_COL + ((uint32_t)(q * 32) << 16) + half * HC + c * 32, v + 32 * c);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);  // the accumulator is in registers now
+      acc_phase ^= 1u;
+
       const bool row_ok = row < ti.rows_valid;
+      if (!row_ok) continue;
       float alpha;
       if (EPI == EPI_F32 || EPI == EPI_BF16) alpha = __fmul_rn(*p.a_g, *p.b_g);
       else if (EPI == EPI_W13) alpha = __fmul_rn(*p.a_g, p.w_g[ti.e]);
       else alpha = __fmul_rn(p.h_g[ti.e], p.w_g[ti.e]);
-      float wrow = 1.0f;
-      if (EPI == EPI_W2 && row_ok && p.topk_w) wrow = p.topk_w[p.perm[ti.out_row0 + row]];
-      const float scale = (EPI == EPI_W2) ? __fmul_rn(alpha, wrow) : alpha;
-      float hg = 0.f;
-      if (EPI == EPI_W13) hg = p.h_g[ti.e];
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        float v[32];
-        __syncwarp();
-        tmem_ld32(tmem + C::ACC_COL + ((uint32_t)(q * 32) << 16) + c * 32, v);
-        const int col0 = ti.n0 + c * 32;
-        if (!row_ok || col0 >= p.N) {
-          // nothing to store for this row / column block
-        } else if (EPI == EPI_F32) {
+      float scale = alpha;
+      if (EPI == EPI_W2 && p.topk_w) scale = __fmul_rn(alpha, p.topk_w[p.perm[ti.out_row0 + row]]);
+      const int colh = ti.n0 + half * HC;
+#pragma unroll
+      for (int c = 0; c < HC / 32; ++c) {
+        const float *w = v + 32 * c;
+        const int col0 = colh + c * 32;
+        if (col0 >= p.N) break;
+        if (EPI == EPI_F32) {
           float *dst = static_cast<float *>(p.c) + (int64_t)(ti.out_row0 + row) * p.N + col0;
 #pragma unroll
-          for (int i = 0; i < 32; i += 4) {
+          for (int i = 0; i < 32; i += 4)
             if (col0 + i < p.N)
-              *reinterpret_cast<float4 *>(dst + i) =
-                  make_float4(__fmul_rn(v[i], scale), __fmul_rn(v[i + 1], scale), __fmul_rn(v[i + 2], scale),
-                              __fmul_rn(v[i + 3], scale));
-          }
+              *reinterpret_cast<float4 *>(dst + i) = make_float4(__fmul_rn(w[i], scale), __fmul_rn(w[i + 1], scale),
+                                                                 __fmul_rn(w[i + 2], scale), __fmul_rn(w[i + 3], scale));
         } else if (EPI == EPI_BF16) {
           __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.c) + (int64_t)(ti.out_row0 + row) * p.N + col0;
 #pragma unroll
@@ -313,7 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               __nv_bfloat162 b[4];
 #pragma unroll
               for (int j = 0; j < 4; ++j)
-                b[j] = __floats2bfloat162_rn(__fmul_rn(v[i + 2 * j], scale), __fmul_rn(v[i + 2 * j + 1], scale));
+                b[j] = __floats2bfloat162_rn(__fmul_rn(w[i + 2 * j], scale), __fmul_rn(w[i + 2 * j + 1], scale));
               *reinterpret_cast<uint4 *>(dst + i) = *reinterpret_cast<uint4 *>(b);
             }
           }
@@ -323,14 +372,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           float h[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float gte = __fmul_rn(v[i], scale);
-            const float up = __fmul_rn(v[16 + i], scale);
+            const float gte = __fmul_rn(w[i], scale);
+            const float up = __fmul_rn(w[16 + i], scale);
             h[i] = __fmul_rn(silu_f32(gte), up);
           }
           const int hc = col0 / 2;
           const int64_t prow = (int64_t)ti.a_row0 + row;  // padded row
           uint32_t lo, hi;
-          const uint32_t sf = nvfp4_block16(h, hg, &lo, &hi);
+          const uint32_t sf = nvfp4_block16(h, p.h_g[ti.e], &lo, &hi);
           *reinterpret_cast<uint2 *>(p.h_codes + prow * (p.I / 2) + hc / 2) = make_uint2(lo, hi);
           p.h_sf[sf_tiled_offset(prow, hc / 16, p.I / 64)] = (uint8_t)sf;
           if (p.h_dump) {
@@ -342,15 +391,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           float *dst = p.y + (int64_t)(ti.out_row0 + row) * p.N + col0;
 #pragma unroll
           for (int i = 0; i < 32; i += 4)
-            *reinterpret_cast<float4 *>(dst + i) =
-                make_float4(__fmul_rn(v[i], scale), __fmul_rn(v[i + 1], scale), __fmul_rn(v[i + 2], scale),
-                            __fmul_rn(v[i + 3], scale));
+            *reinterpret_cast<float4 *>(dst + i) = make_float4(__fmul_rn(w[i], scale), __fmul_rn(w[i + 1], scale),
+                                                               __fmul_rn(w[i + 2], scale), __fmul_rn(w[i + 3], scale));
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty);
-      acc_phase ^= 1u;
     }
   }
 
