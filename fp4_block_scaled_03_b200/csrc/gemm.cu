@@ -49,23 +49,28 @@ constexpr int kThreads = 32 * (kFirstEpiWarp + kEpiWarps);
 
 enum Epi { EPI_F32 = 0, EPI_BF16 = 1, EPI_W13 = 2, EPI_W2 = 3 };
 
-template <int BN>
+template <int BN, int EPI>
 struct Cfg {
-  static constexpr int kStages = 4;
+  // w2 keeps one stage fewer to make room for its store staging buffers
+  static constexpr int kStages = (EPI == 3) ? 3 : 4;
   static constexpr int A_BYTES = BM * BK_BYTES;
   static constexpr int B_BYTES = BN * BK_BYTES;
   static constexpr int HALVES = (BN + 127) / 128;  // 128-row scale slabs of B per tile
   static constexpr int SFA_BYTES = 4 * 512;
   static constexpr int SFB_BYTES = HALVES * 4 * 512;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  // w2 epilogue: one 32-row x 32-column fp32 box (4 KB, 128-byte swizzle) per epilogue warp
+  static constexpr int STG_BYTES = (EPI == 3) ? kEpiWarps * 4096 : 0;
   static constexpr int TMEM_COLS = 512;
   static constexpr int ACC_COL = 0;
   static constexpr int SF_SLOT_COLS = 16 + 16 * HALVES;  // SFA: 4 K-words x 4; SFB: 4 x 4*HALVES
   static constexpr int SF_COL0 = 256;                     // slot s at SF_COL0 + s * SF_SLOT_COLS
-  static constexpr int SMEM_BYTES = kStages * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int SMEM_BYTES = kStages * STAGE_BYTES + STG_BYTES + 1024 /*align*/ + 256 /*barriers*/;
   static_assert(BN == 256, "the early-release epilogue splits 256 columns into two halves");
   static_assert(SF_COL0 + kStages * SF_SLOT_COLS <= TMEM_COLS, "tmem");
   static_assert((3 * kStages + 4) * 8 <= 256, "barriers");
+  static_assert(STAGE_BYTES % 1024 == 0, "stage buffers stay 1024-byte aligned");
+  static_assert(SMEM_BYTES + 1024 <= 232448, "shared memory");
 };
 
 struct Params {
@@ -149,8 +154,8 @@ __device__ __forceinline__ float silu_f32(float z) {
 template <int BN, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const Params p) {
-  using C = Cfg<BN>;
+                    const __grid_constant__ CUtensorMap tmY, const Params p) {
+  using C = Cfg<BN, EPI>;
   constexpr bool kGrouped = (EPI == EPI_W13 || EPI == EPI_W2);
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -158,7 +163,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *smB = smA + C::kStages * C::A_BYTES;
   uint8_t *smSFA = smB + C::kStages * C::B_BYTES;
   uint8_t *smSFB = smSFA + C::kStages * C::SFA_BYTES;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smSFB + C::kStages * C::SFB_BYTES);
+  uint8_t *smStg = smSFB + C::kStages * C::SFB_BYTES;  // 1024-aligned (stage sizes are)
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smStg + C::STG_BYTES);
   uint64_t *full = bars;                       // TMA data landed        (count 1 + tx)
   uint64_t *empty = bars + C::kStages;         // MMAs done with a stage (tcgen05.commit)
   uint64_t *sf_full = bars + 2 * C::kStages;   // stage scales in TMEM   (tcgen05.commit)
@@ -334,6 +340,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       acc_phase ^= 1u;
 
       const bool row_ok = row < ti.rows_valid;
+      // w2: a warp whose 32 rows are all valid writes through TMA (collective
+      // per warp); otherwise each valid row is stored by its own thread
+      const bool full_box = (EPI == EPI_W2) && (q * 32 + 32 <= ti.rows_valid);
       if (!row_ok) continue;
       float alpha;
       if (EPI == EPI_F32 || EPI == EPI_BF16) alpha = __fmul_rn(*p.a_g, *p.b_g);
@@ -387,15 +396,31 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 4; ++i) d[i] = make_float4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
           }
-        } else {  // EPI_W2
+        } else if (!full_box) {  // EPI_W2, a warp holding the expert's last rows
           float *dst = p.y + (int64_t)(ti.out_row0 + row) * p.N + col0;
 #pragma unroll
           for (int i = 0; i < 32; i += 4)
             *reinterpret_cast<float4 *>(dst + i) = make_float4(__fmul_rn(w[i], scale), __fmul_rn(w[i + 1], scale),
                                                                __fmul_rn(w[i + 2], scale), __fmul_rn(w[i + 3], scale));
+        } else {  // EPI_W2, all 32 rows valid: stage the box and store it with TMA
+          uint8_t *stg = smStg + (warp - kFirstEpiWarp) * 4096;
+          if (lane == 0) bulk_wait_read_all();  // previous box has left the buffer
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 8; ++j)  // 16-byte chunk j of row `lane`, 128-byte swizzle
+            *reinterpret_cast<float4 *>(stg + lane * 128 + ((j ^ (lane & 7)) * 16)) =
+                make_float4(__fmul_rn(w[4 * j], scale), __fmul_rn(w[4 * j + 1], scale),
+                            __fmul_rn(w[4 * j + 2], scale), __fmul_rn(w[4 * j + 3], scale));
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmY, stg, col0, ti.out_row0 + q * 32);
+            bulk_commit();
+          }
         }
       }
     }
+    if (EPI == EPI_W2 && lane == 0) bulk_wait_all();  // stores complete before the CTA exits
   }
 
   tc_fence_before();
@@ -440,6 +465,20 @@ bool make_code_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t row
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// fp32 matrix [rows][cols] as a 2-D tensor map with a 32 x 32 box and
+// 128-byte swizzle (the w2 epilogue's store staging layout).
+bool make_f32_store_map(CUtensorMap *m, void *base, uint64_t rows, uint64_t cols) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 4};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 int sm_count() {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
@@ -448,11 +487,12 @@ int sm_count() {
 }
 
 template <int BN, int EPI>
-fp4_status launch(const CUtensorMap &ta, const CUtensorMap &tb, const Params &p, int grid, cudaStream_t s) {
-  using C = Cfg<BN>;
+fp4_status launch(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &ty, const Params &p, int grid,
+                  cudaStream_t s) {
+  using C = Cfg<BN, EPI>;
   auto kern = fp4_gemm_kernel<BN, EPI>;
   FP4_HOST_CHECK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
-  kern<<<grid, kThreads, C::SMEM_BYTES, s>>>(ta, tb, p);
+  kern<<<grid, kThreads, C::SMEM_BYTES, s>>>(ta, tb, ty, p);
   FP4_HOST_CHECK(cudaGetLastError());
   return FP4_OK;
 }
@@ -497,8 +537,8 @@ fp4_status fp4_gemm(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_
   if (tiles > 2147483647LL) return FP4_ERR_UNSUPPORTED_SHAPE;
   const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (c_dtype == FP4_OUT_F32) return launch<kBN, EPI_F32>(ta, tb, p, grid, s);
-  return launch<kBN, EPI_BF16>(ta, tb, p, grid, s);
+  if (c_dtype == FP4_OUT_F32) return launch<kBN, EPI_F32>(ta, tb, tb, p, grid, s);
+  return launch<kBN, EPI_BF16>(ta, tb, tb, p, grid, s);
 }
 
 fp4_status fp4_moe_w13(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_g, const fp4_moe_weights *w,
@@ -533,7 +573,7 @@ fp4_status fp4_moe_w13(const uint8_t *a_codes, const uint8_t *a_sf, const float 
   p.h_dump = (flags & FP4_DEBUG_DUMP_H) ? h_dump : nullptr;
   p.status = ctx->status;
   p.wait_limit = ctx->wait_limit_ns;
-  return launch<kBN, EPI_W13>(ta, tb, p, sm_count(), reinterpret_cast<cudaStream_t>(stream));
+  return launch<kBN, EPI_W13>(ta, tb, tb, p, sm_count(), reinterpret_cast<cudaStream_t>(stream));
 }
 
 fp4_status fp4_moe_w2(const uint8_t *h_codes, const uint8_t *h_sf, const fp4_moe_weights *w, int64_t H, int64_t I,
@@ -563,7 +603,9 @@ fp4_status fp4_moe_w2(const uint8_t *h_codes, const uint8_t *h_sf, const fp4_moe
   p.perm = perm; p.topk_w = topk_weights; p.y = y;
   p.status = ctx->status;
   p.wait_limit = ctx->wait_limit_ns;
-  return launch<kBN, EPI_W2>(ta, tb, p, sm_count(), reinterpret_cast<cudaStream_t>(stream));
+  CUtensorMap ty;
+  if (!make_f32_store_map(&ty, y, (uint64_t)rows_cap, (uint64_t)H)) return FP4_ERR_CUDA;
+  return launch<kBN, EPI_W2>(ta, tb, ty, p, sm_count(), reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"
