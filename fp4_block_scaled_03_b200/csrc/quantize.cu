@@ -35,15 +35,28 @@ __global__ void __launch_bounds__(kThreads) amax_bf16_kernel(const uint16_t *__r
                                                              unsigned int *__restrict__ amax_bits) {
   const int64_t vec_per_row = cols / 8;
   const int64_t total = rows * vec_per_row;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   uint32_t m = 0;
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t r = i / vec_per_row, c = (i - r * vec_per_row) * 8;
-    const uint4 v = __ldcs(reinterpret_cast<const uint4 *>(x + r * ld + c));
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  // four independent 16-byte loads in flight per thread
+  for (int64_t i0 = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i0 < total; i0 += 4 * stride) {
+    uint4 v[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      m = max(m, w[j] & 0x7FFFu);
-      m = max(m, (w[j] >> 16) & 0x7FFFu);
+    for (int u = 0; u < 4; ++u) {
+      const int64_t i = i0 + u * stride;
+      v[u] = make_uint4(0, 0, 0, 0);
+      if (i < total) {
+        const int64_t r = i / vec_per_row, c = (i - r * vec_per_row) * 8;
+        v[u] = __ldcs(reinterpret_cast<const uint4 *>(x + r * ld + c));
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        m = max(m, w[j] & 0x7FFFu);
+        m = max(m, (w[j] >> 16) & 0x7FFFu);
+      }
     }
   }
 #pragma unroll
@@ -75,24 +88,41 @@ __global__ void __launch_bounds__(kThreads) nvfp4_quantize_kernel(
   const int64_t nb = cols / 16;
   const int64_t total = rows * nb;
   const int64_t n_ksteps = cols / 64;
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t r = i / nb, b = i - r * nb;
-    const uint4 *src = reinterpret_cast<const uint4 *>(x + r * ld + b * 16);
-    const uint4 v0 = __ldcs(src), v1 = __ldcs(src + 1);
-    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-    float f[16];
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  // two blocks (four independent 16-byte loads) in flight per thread
+  for (int64_t i0 = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i0 < total; i0 += 2 * stride) {
+    uint4 v[2][2];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      f[2 * j] = bf16_bits_to_f32(w[j] & 0xFFFFu);
-      f[2 * j + 1] = bf16_bits_to_f32(w[j] >> 16);
+    for (int u = 0; u < 2; ++u) {
+      const int64_t i = i0 + u * stride;
+      v[u][0] = v[u][1] = make_uint4(0, 0, 0, 0);
+      if (i < total) {
+        const int64_t r = i / nb, b = i - r * nb;
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + r * ld + b * 16);
+        v[u][0] = __ldcs(src);
+        v[u][1] = __ldcs(src + 1);
+      }
     }
-    uint32_t lo, hi;
-    const uint32_t sf = nvfp4_block16(f, g, &lo, &hi);
-    *reinterpret_cast<uint2 *>(codes + r * (cols / 2) + b * 8) = make_uint2(lo, hi);
-    if (kTiled)
-      scales[sf_tiled_offset(r, b, n_ksteps)] = (uint8_t)sf;
-    else
-      scales[i] = (uint8_t)sf;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int64_t i = i0 + u * stride;
+      if (i >= total) break;
+      const int64_t r = i / nb, b = i - r * nb;
+      const uint32_t w[8] = {v[u][0].x, v[u][0].y, v[u][0].z, v[u][0].w, v[u][1].x, v[u][1].y, v[u][1].z, v[u][1].w};
+      float f[16];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        f[2 * j] = bf16_bits_to_f32(w[j] & 0xFFFFu);
+        f[2 * j + 1] = bf16_bits_to_f32(w[j] >> 16);
+      }
+      uint32_t lo, hi;
+      const uint32_t sf = nvfp4_block16(f, g, &lo, &hi);
+      *reinterpret_cast<uint2 *>(codes + r * (cols / 2) + b * 8) = make_uint2(lo, hi);
+      if (kTiled)
+        scales[sf_tiled_offset(r, b, n_ksteps)] = (uint8_t)sf;
+      else
+        scales[i] = (uint8_t)sf;
+    }
   }
 }
 
