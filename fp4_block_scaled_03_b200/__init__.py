@@ -80,6 +80,7 @@ _SIGS = {
         [_P, _P, _P, _I64, _I32, ctypes.POINTER(MoeWeights), _I64, _I64, _I32, _P, _P, _SZ, _U32, _P, _P],
     ),
     "fp4_moe_route_scratch_bytes": (_SZ, [_I64, _I32]),
+    "fp4_moe_topk": (ctypes.c_int, [_P, _I64, _I32, _I32, _P, _P, _P]),
     "fp4_moe_route": (ctypes.c_int, [_P, _I64, _I32, _I32, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "fp4_moe_route_noalloc": (ctypes.c_int, [_P, _I64, _I32, _I32, _P, _P, _P, _P, _P, _P]),
     "fp4_moe_gather": (ctypes.c_int, [_P, _P, _I64, _I32, _I64, _I32, _P, _P, _P, _P, _P, _I64, _P]),
@@ -136,6 +137,11 @@ def fp4_mx_to_nv(codes, mx_scales, rows, cols, num_tensors, nv_scales, nv_global
 def fp4_gemm(a_codes, a_sf, a_g, b_codes, b_sf, b_g, c, c_dtype, M, N, K, flags=0):
     _check(lib.fp4_gemm(_ptr(a_codes), _ptr(a_sf), _ptr(a_g), _ptr(b_codes), _ptr(b_sf), _ptr(b_g), _ptr(c),
                         c_dtype, M, N, K, flags, _stream()), "fp4_gemm")
+
+
+def fp4_moe_topk(logits, T, E, topk, expert_ids, topk_weights):
+    _check(lib.fp4_moe_topk(_ptr(logits), T, E, topk, _ptr(expert_ids), _ptr(topk_weights), _stream()),
+           "fp4_moe_topk")
 
 
 def fp4_moe_route(expert_ids, T, topk, E, counts, offsets, tile_offsets, perm, inv, scratch):

@@ -186,6 +186,49 @@ __global__ void combine_kernel(const float *__restrict__ y, const int32_t *__res
   }
 }
 
+// Router top-k: one warp per token.  Each of k rounds takes the warp-wide
+// largest remaining logit (ties to the lower expert id); the weights are the
+// softmax of the k chosen logits, fp32, summed in slot order.
+__global__ void topk_softmax_kernel(const float *__restrict__ logits, int64_t T, int32_t E, int32_t k,
+                                    int32_t *__restrict__ ids, float *__restrict__ weights) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
+  for (int64_t t = blockIdx.x * (int64_t)(blockDim.x / 32) + (threadIdx.x >> 5); t < T; t += warps) {
+    const float *z = logits + t * E;
+    int chosen[16];
+    float val[16];
+    for (int s = 0; s < k; ++s) {
+      float best = -INFINITY;
+      int bi = 0x7fffffff;
+      for (int e = lane; e < E; e += 32) {
+        bool taken = false;
+        for (int u = 0; u < s; ++u) taken |= (chosen[u] == e);
+        const float v = z[e];
+        if (!taken && (v > best || (v == best && e < bi))) { best = v; bi = e; }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, best, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (ov > best || (ov == best && oi < bi)) { best = ov; bi = oi; }
+      }
+      chosen[s] = bi;
+      val[s] = best;
+    }
+    if (lane == 0) {
+      float e[16], sum = 0.0f;
+      for (int s = 0; s < k; ++s) {
+        e[s] = expf(__fsub_rn(val[s], val[0]));
+        sum = __fadd_rn(sum, e[s]);
+      }
+      for (int s = 0; s < k; ++s) {
+        ids[t * k + s] = chosen[s];
+        weights[t * k + s] = __fdiv_rn(e[s], sum);
+      }
+    }
+  }
+}
+
 int sm_count() {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
@@ -257,6 +300,20 @@ fp4_status fp4_moe_route(const int32_t *expert_ids, int64_t T, int32_t topk, int
     route_scatter_kernel<<<nchunks, 32, esm, s>>>(expert_ids, R, E, cc, perm, inv);
     FP4_HOST_CHECK(cudaGetLastError());
   }
+  return FP4_OK;
+}
+
+fp4_status fp4_moe_topk(const float *logits, int64_t T, int32_t E, int32_t topk, int32_t *expert_ids,
+                        float *topk_weights, fp4_stream_t stream) {
+  if (!logits || !expert_ids || !topk_weights) return FP4_ERR_INVALID_ARG;
+  if (T < 0 || E < 1 || E > 65536 || topk < 1 || topk > 16 || topk > E) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return FP4_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int64_t grid = (T + 7) / 8;
+  const int64_t cap = (int64_t)sm_count() * 16;
+  if (grid > cap) grid = cap;
+  topk_softmax_kernel<<<(unsigned)grid, 256, 0, s>>>(logits, T, E, topk, expert_ids, topk_weights);
+  FP4_HOST_CHECK(cudaGetLastError());
   return FP4_OK;
 }
 

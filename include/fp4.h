@@ -199,6 +199,14 @@ fp4_status fp4_moe_grouped_gemm(const void *tokens_bf16, const int32_t *expert_i
 
 /* ---- the layer's stages, each callable on its own ------------------------ */
 
+/* Router top-k [QAT §3.1: each token is sent to its top-k experts; ARCH §2.1:
+ * top-6 of 384]: logits fp32 [T][E] -> expert_ids int32 [T][topk] (the topk
+ * largest logits in descending order, ties to the lower expert id) and
+ * topk_weights fp32 [T][topk] = softmax over the chosen logits (fp32,
+ * exp(z - z_max), summed in slot order).  1 <= topk <= min(16, E). */
+fp4_status fp4_moe_topk(const float *logits, int64_t T, int32_t E, int32_t topk, int32_t *expert_ids,
+                        float *topk_weights, fp4_stream_t stream);
+
 /* Routing tables written by fp4_moe_route (all device int32):
  *   counts[E]          rows per expert
  *   offsets[E+1]       exclusive prefix of counts (row index in routed order)

@@ -43,6 +43,18 @@ def route(expert_ids, num_experts):
     return counts, offsets, perm, inv.reshape(T, k)
 
 
+def topk_softmax(logits, k):
+    """Router top-k ("DeepSeek-V4 FP4 QAT" §3.1: each token picks its top-k
+    experts): expert ids = the k largest logits, ties to the lower expert id
+    (a stable sort of -logits); weights = softmax over the k chosen logits,
+    in fp64.  logits fp32 [T, E] -> (ids int64 [T, k], weights fp64 [T, k])."""
+    z = np.asarray(logits, dtype=np.float32).astype(np.float64)
+    order = np.argsort(-z, axis=1, kind="stable")[:, :k]
+    sel = np.take_along_axis(z, order, axis=1)
+    e = np.exp(sel - sel[:, :1])
+    return order.astype(np.int64), e / e.sum(axis=1, keepdims=True)
+
+
 def silu(z):
     z = np.asarray(z, dtype=np.float64)
     return z / (1.0 + np.exp(-z))

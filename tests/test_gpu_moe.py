@@ -315,3 +315,22 @@ def _unstable_blocks(h, tol, g):
     m = F.unpack_nibbles(c_mid).reshape(n, -1, 16)
     same = (s_lo == s_mid) & (s_hi == s_mid) & ((a & 7) == (m & 7)).all(2) & ((b & 7) == (m & 7)).all(2)
     return ~same
+
+
+@pytest.mark.parametrize("T,E,k,grid", [(4096, 384, 6, None), (777, 256, 8, None), (300, 64, 6, 0.25), (5, 16, 16, None)])
+def test_topk_softmax(T, E, k, grid):
+    """Router top-k: ids bit-exact against the oracle's stable sort (ties to
+    the lower id, forced by rounding logits to a coarse grid); weights within
+    2e-6 relative (fp32 exp, sum and divide against fp64)."""
+    fp4 = _lib()
+    g = torch.Generator(device="cuda")
+    g.manual_seed(T + E)
+    z = torch.randn((T, E), generator=g, device="cuda", dtype=torch.float32)
+    if grid:
+        z = torch.round(z / grid) * grid
+    ids = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    fp4.fp4_moe_topk(z, T, E, k, ids, w)
+    rid, rw = MO.topk_softmax(z.cpu().numpy(), k)
+    assert np.array_equal(ids.cpu().numpy(), rid)
+    np.testing.assert_allclose(w.cpu().numpy(), rw, rtol=2e-6, atol=0)

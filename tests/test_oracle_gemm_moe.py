@@ -116,3 +116,18 @@ def test_expert_ffn_requantizes_h_with_static_scale():
     c2, s2, _ = Q.nvfp4_quantize(r["h"].astype(np.float32), g=np.float32(0.01))
     assert np.array_equal(c2, r["h_codes"]) and np.array_equal(s2, r["h_sf"])
     np.testing.assert_allclose(r["y"], r["h_dq"] @ w2.T, rtol=1e-15)
+
+
+def test_topk_softmax_brute_force_and_ties():
+    rng = np.random.default_rng(3)
+    z = rng.standard_normal((50, 20)).astype(np.float32)
+    z[0, 3] = z[0, 7] = z[0, 11] = 9.0  # a three-way tie at the top: lower ids first
+    ids, w = M.topk_softmax(z, 4)
+    for t in range(50):
+        brute = sorted(range(20), key=lambda e: (-float(z[t, e]), e))[:4]
+        assert ids[t].tolist() == brute
+    assert ids[0, :3].tolist() == [3, 7, 11]
+    np.testing.assert_allclose(w.sum(axis=1), 1.0, rtol=1e-15)
+    # softmax of the chosen logits, closed form for one row
+    sel = z[5, ids[5]].astype(np.float64)
+    np.testing.assert_allclose(w[5], np.exp(sel) / np.exp(sel).sum(), rtol=1e-14)
