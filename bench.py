@@ -255,26 +255,27 @@ class MoeBench:
         assert fp4.fp4_get_device_status() == 0
 
     def step(self, events=None, dump=None):
+        """One pass of the hot path, stage by stage (the same kernels, in the same
+        order, as fp4_moe_grouped_gemm), with CUDA events between stages."""
         fp4 = self.fp4
         T, H, I, E, k, cap = self.T, self.H, self.I, self.E, self.k, self.cap
         ev = (lambda i: events[i].record()) if events else (lambda i: None)
         ev(0)
-        fp4.fp4_quantize(fp4.FP4_NV, self.x, T, H, H, self.xc, self.xs, self.xg, 0, self.qws, 256)
-        ev(1)
         fp4.fp4_moe_route(self.ids, T, k, E, self.counts_d, self.offs, self.toffs, self.perm, self.inv, self.scratch)
+        ev(1)
+        fp4.fp4_moe_quantize_gather(self.x, T, k, H, E, self.offs, self.toffs, self.inv, self.a_c, self.a_s, cap,
+                                    self.xg, self.qws)
         ev(2)
-        fp4.fp4_moe_gather(self.xc, self.xs, T, k, H, E, self.offs, self.toffs, self.perm, self.a_c, self.a_s, cap)
-        ev(3)
         fp4.fp4_moe_w13(self.a_c, self.a_s, self.xg, self.wset, H, I, E, self.counts_d, self.toffs, cap, self.h_c,
                         self.h_s, fp4.FP4_DEBUG_DUMP_H if dump is not None else 0, dump)
-        ev(4)
+        ev(3)
         fp4.fp4_moe_w2(self.h_c, self.h_s, self.wset, H, I, E, self.counts_d, self.offs, self.toffs, self.perm, self.w,
                        cap, self.y)
-        ev(5)
+        ev(4)
         fp4.fp4_moe_combine(self.y, self.inv, T, k, H, self.out)
-        ev(6)
+        ev(5)
 
-    LAUNCHES_PER_STEP = 9  # amax, quantize, 3 routing, gather, w13, w2, combine
+    LAUNCHES_PER_STEP = 8  # 3 routing, amax, quantize+gather, w13, w2, combine
 
     def flops(self):
         return 2.0 * 3.0 * self.H * self.I * self.R
@@ -295,7 +296,7 @@ def run_moe(args, world, rank, peaks):
     for _ in range(args.warmup):
         b.step()
     torch.cuda.synchronize()
-    nst = 7
+    nst = 6
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nst)] for _ in range(args.steps)]
     sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
     if sampler:
@@ -326,13 +327,13 @@ def run_moe(args, world, rank, peaks):
     fp4_peak = 4.0 * peaks["bf16_sus"]
     # dominant kernel: the grouped w13 GEMM (2/3 of the layer's FLOPs)
     w13_flops = 2.0 * 2 * b.I * b.H * b.R
-    w13_tf = w13_flops / (stage[3] * 1e-3) / 1e12
+    w13_tf = w13_flops / (stage[2] * 1e-3) / 1e12
     # algorithmic bytes of the w13 launch: touched experts' w13 weights, the gathered rows, h out
     n_touched = int((b.counts > 0).sum().item())
     w13_bytes = n_touched * 2 * b.I * b.H * 0.5625 + b.R * b.H * 0.5625 + b.R * b.I * 0.5625
-    w2_tf = (2.0 * b.I * b.H * b.R) / (stage[4] * 1e-3) / 1e12
-    q_bytes = b.T * b.H * 2.5625
-    q_gbs = q_bytes / (stage[0] * 1e-3) / 1e9
+    w2_tf = (2.0 * b.I * b.H * b.R) / (stage[3] * 1e-3) / 1e12
+    q_bytes = b.T * b.H * 2.0 + b.R * b.H * 0.5625  # read x once, write every routed row
+    q_gbs = q_bytes / (stage[1] * 1e-3) / 1e9
 
     # e2e through the public call: every step copies its inputs (x, expert ids, top-k
     # weights) from pinned host memory and its bf16 output back, inside the timed
@@ -414,13 +415,15 @@ def run_moe(args, world, rank, peaks):
                      "frac": round(w13_tf / fp4_peak, 4), "traffic": measured_traffic(args.workload, "w13"),
                      "algorithmic_bytes": w13_bytes,
                      "frac_of_max_flops_bytes": round(max(w13_flops / (fp4_peak * 1e12), w13_bytes / (peaks["hbm"] * 1e9))
-                                                      / (stage[3] * 1e-3), 4),
+                                                      / (stage[2] * 1e-3), 4),
                      "peak_note": "4 x measured sustained bf16 cuBLAS (nominal fp4/bf16 ratio), of " + peaks["src"]},
-        "stages_ms": {n: round(v, 4) for n, v in zip(["quantize", "route", "gather", "w13", "w2", "combine"], stage)},
+        "stages_ms": {n: round(v, 4) for n, v in zip(["route", "quantize_gather", "w13", "w2", "combine"], stage)},
         "w2": {"achieved_tflops": round(w2_tf, 1), "frac": round(w2_tf / fp4_peak, 4),
                "traffic": measured_traffic(args.workload, "w2")},
         "quantize": {"achieved_gbs": round(q_gbs, 1), "peak_gbs": peaks["hbm"], "frac": round(q_gbs / peaks["hbm"], 4),
-                     "algorithmic_bytes": q_bytes, "note": "dynamic g: amax pass + quantize pass, 2.5625 B/elem counted"},
+                     "algorithmic_bytes": q_bytes,
+                     "note": "dynamic g, fused with the gather: x read once (2 B/elem) + every routed row written"
+                             " (0.5625 B/elem); the amax pass's second read of x is not counted"},
         "weight_stream": {"touched_bytes": b.touched_weight_bytes(),
                           "gbs_layer": round(b.touched_weight_bytes() / (ms * 1e-3) / 1e9, 1)},
         "e2e": {"value": round(world * flops / (e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "ms_per_step": round(e_ms, 4),

@@ -84,6 +84,7 @@ _SIGS = {
     "fp4_moe_route": (ctypes.c_int, [_P, _I64, _I32, _I32, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "fp4_moe_route_noalloc": (ctypes.c_int, [_P, _I64, _I32, _I32, _P, _P, _P, _P, _P, _P]),
     "fp4_moe_gather": (ctypes.c_int, [_P, _P, _I64, _I32, _I64, _I32, _P, _P, _P, _P, _P, _I64, _P]),
+    "fp4_moe_quantize_gather": (ctypes.c_int, [_P, _I64, _I32, _I64, _I32, _P, _P, _P, _P, _P, _I64, _P, _P, _SZ, _P]),
     "fp4_moe_w13": (
         ctypes.c_int,
         [_P, _P, _P, ctypes.POINTER(MoeWeights), _I64, _I64, _I32, _P, _P, _I64, _P, _P, _U32, _P, _P],
@@ -160,6 +161,14 @@ def fp4_moe_route_noalloc(expert_ids, T, topk, E, counts, offsets, tile_offsets,
 def fp4_moe_gather(x_codes, x_sf, T, topk, H, E, offsets, tile_offsets, perm, a_codes, a_sf, rows_cap):
     _check(lib.fp4_moe_gather(_ptr(x_codes), _ptr(x_sf), T, topk, H, E, _ptr(offsets), _ptr(tile_offsets),
                               _ptr(perm), _ptr(a_codes), _ptr(a_sf), rows_cap, _stream()), "fp4_moe_gather")
+
+
+def fp4_moe_quantize_gather(x, T, topk, H, E, offsets, tile_offsets, inv, a_codes, a_sf, rows_cap, global_scale,
+                            workspace):
+    _check(lib.fp4_moe_quantize_gather(_ptr(x), T, topk, H, E, _ptr(offsets), _ptr(tile_offsets), _ptr(inv),
+                                       _ptr(a_codes), _ptr(a_sf), rows_cap, _ptr(global_scale), _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(), _stream()),
+           "fp4_moe_quantize_gather")
 
 
 def fp4_moe_w13(a_codes, a_sf, a_g, w, H, I, E, counts, tile_offsets, rows_cap, h_codes, h_sf, flags=0, h_dump=None):

@@ -1,5 +1,6 @@
-// The routed-expert MoE layer as one call: quantize x -> route -> gather ->
-// grouped w13 (+SwiGLU +NVFP4 re-quantize) -> grouped w2 -> combine.
+// The routed-expert MoE layer as one call: route -> quantize x straight into
+// the expert rows -> grouped w13 (+SwiGLU +NVFP4 re-quantize) -> grouped w2 ->
+// combine.
 //
 // "DeepSeek-V4 FP4 QAT", §3.1 (tokens go to their top-k experts; outputs are
 // summed), "DeepSeek-V4 architecture", §5.1 (SwiGLU feed-forward experts),
@@ -12,7 +13,7 @@
 namespace {
 
 struct MoeLayout {
-  size_t header, x_codes, x_sf, counts, offsets, tile_offsets, perm, inv, scratch, a_codes, a_sf, h_codes, h_sf, y;
+  size_t header, counts, offsets, tile_offsets, perm, inv, scratch, a_codes, a_sf, h_codes, h_sf, y;
   size_t total;
   int64_t rows_cap;
 };
@@ -30,8 +31,6 @@ MoeLayout moe_layout(int64_t T, int32_t topk, int64_t H, int64_t I, int32_t E) {
     return at;
   };
   L.header = take(512);  // [0,256) quantize workspace, [256,260) g_x
-  L.x_codes = take((size_t)(T * H / 2));
-  L.x_sf = take((size_t)(T * H / 16));
   L.counts = take((size_t)E * 4);
   L.offsets = take((size_t)(E + 1) * 4);
   L.tile_offsets = take((size_t)(E + 1) * 4);
@@ -72,13 +71,11 @@ fp4_status fp4_moe_grouped_gemm(const void *tokens_bf16, const int32_t *expert_i
   float *g_x = reinterpret_cast<float *>(ws + L.header + 256);
   auto I32 = [&](size_t off) { return reinterpret_cast<int32_t *>(ws + off); };
   fp4_status st;
-  st = fp4_quantize(FP4_NV, tokens_bf16, T, H, H, ws + L.x_codes, ws + L.x_sf, g_x, 0, ws + L.header, 256, stream);
-  if (st != FP4_OK) return st;
   st = fp4_moe_route(expert_ids, T, topk, E, I32(L.counts), I32(L.offsets), I32(L.tile_offsets), I32(L.perm),
                      I32(L.inv), ws + L.scratch, fp4_moe_route_scratch_bytes(T * topk, E), stream);
   if (st != FP4_OK) return st;
-  st = fp4_moe_gather(ws + L.x_codes, ws + L.x_sf, T, topk, H, E, I32(L.offsets), I32(L.tile_offsets), I32(L.perm),
-                      ws + L.a_codes, ws + L.a_sf, L.rows_cap, stream);
+  st = fp4_moe_quantize_gather(tokens_bf16, T, topk, H, E, I32(L.offsets), I32(L.tile_offsets), I32(L.inv),
+                               ws + L.a_codes, ws + L.a_sf, L.rows_cap, g_x, ws + L.header, 256, stream);
   if (st != FP4_OK) return st;
   st = fp4_moe_w13(ws + L.a_codes, ws + L.a_sf, g_x, w, H, I, E, I32(L.counts), I32(L.tile_offsets), L.rows_cap,
                    ws + L.h_codes, ws + L.h_sf, flags & FP4_DEBUG_DUMP_H, h_dump, stream);

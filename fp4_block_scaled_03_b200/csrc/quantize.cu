@@ -126,6 +126,74 @@ __global__ void __launch_bounds__(kThreads) nvfp4_quantize_kernel(
   }
 }
 
+// ---- NVFP4 quantize fused with the routing gather ---------------------------
+// One CTA per token row at a time: the row's k destination rows (its routed
+// rows, padded per expert to 128) are looked up once into shared memory, then
+// each thread quantizes 16-element blocks and writes codes and the tiled scale
+// to every destination row.  Same arithmetic as nvfp4_quantize_kernel.
+__device__ __forceinline__ int expert_of_row(const int32_t *__restrict__ offsets, int E, int32_t r) {
+  int lo = 0, hi = E;  // offsets[lo] <= r < offsets[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (offsets[mid] <= r) lo = mid; else hi = mid;
+  }
+  return lo;
+}
+
+__global__ void __launch_bounds__(128) nvfp4_quantize_gather_kernel(
+    const uint16_t *__restrict__ x, int64_t T, int64_t H, int32_t topk, int32_t E,
+    const int32_t *__restrict__ offsets, const int32_t *__restrict__ tile_offsets, const int32_t *__restrict__ inv,
+    uint8_t *__restrict__ a_codes, uint8_t *__restrict__ a_sf, const unsigned int *__restrict__ amax_bits,
+    float *__restrict__ g_out) {
+  // each thread quantizes one 64-element K step (four 16-element blocks), so it
+  // writes 32 contiguous code bytes and one 4-byte scale word per destination
+  __shared__ int64_t dst[16];
+  const float g = __fdiv_rn(__uint_as_float(*amax_bits), 2688.0f);
+  if (blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
+  const int64_t n_ksteps = H / 64;
+  for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+    __syncthreads();  // previous row's destinations no longer in use
+    if (threadIdx.x < topk) {
+      const int32_t r = inv[t * topk + threadIdx.x];
+      int64_t d = -1;
+      if (r >= 0) {
+        const int e = expert_of_row(offsets, E, r);
+        d = (int64_t)tile_offsets[e] * 128 + (r - offsets[e]);
+      }
+      dst[threadIdx.x] = d;
+    }
+    __syncthreads();
+    for (int64_t kw = threadIdx.x; kw < n_ksteps; kw += blockDim.x) {
+      const uint4 *src = reinterpret_cast<const uint4 *>(x + t * H + kw * 64);
+      uint4 v[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v[q] = __ldcs(src + q);
+      uint32_t code[8], sfw = 0;
+#pragma unroll
+      for (int blk = 0; blk < 4; ++blk) {
+        const uint32_t w[8] = {v[2 * blk].x, v[2 * blk].y, v[2 * blk].z, v[2 * blk].w,
+                               v[2 * blk + 1].x, v[2 * blk + 1].y, v[2 * blk + 1].z, v[2 * blk + 1].w};
+        float f[16];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          f[2 * j] = bf16_bits_to_f32(w[j] & 0xFFFFu);
+          f[2 * j + 1] = bf16_bits_to_f32(w[j] >> 16);
+        }
+        const uint32_t sf = nvfp4_block16(f, g, &code[2 * blk], &code[2 * blk + 1]);
+        sfw |= sf << (8 * blk);
+      }
+      for (int s = 0; s < topk; ++s) {
+        const int64_t d = dst[s];
+        if (d < 0) continue;
+        uint4 *out = reinterpret_cast<uint4 *>(a_codes + d * (H / 2) + kw * 32);
+        out[0] = make_uint4(code[0], code[1], code[2], code[3]);
+        out[1] = make_uint4(code[4], code[5], code[6], code[7]);
+        *reinterpret_cast<uint32_t *>(a_sf + sf_tiled_offset(d, kw * 4, n_ksteps)) = sfw;
+      }
+    }
+  }
+}
+
 // ---- MXFP4 quantize: one thread per 32-element block -----------------------
 __global__ void __launch_bounds__(kThreads) mxfp4_quantize_kernel(const uint16_t *__restrict__ x, int64_t rows,
                                                                   int64_t cols, int64_t ld,
@@ -314,6 +382,33 @@ fp4_status fp4_mx_to_nv(const uint8_t *codes, const uint8_t *mx_scales, int64_t 
       if (host[i] != host[i]) st = FP4_ERR_RANGE;
   }
   return st;
+}
+
+fp4_status fp4_moe_quantize_gather(const void *x_bf16, int64_t T, int32_t topk, int64_t H, int32_t E,
+                                   const int32_t *offsets, const int32_t *tile_offsets, const int32_t *inv,
+                                   uint8_t *a_codes, uint8_t *a_sf, int64_t rows_cap, float *global_scale,
+                                   void *workspace, size_t ws_bytes, fp4_stream_t stream) {
+  if (!x_bf16 || !offsets || !tile_offsets || !inv || !a_codes || !a_sf || !global_scale || !workspace)
+    return FP4_ERR_INVALID_ARG;
+  if (T < 0 || topk < 1 || topk > 16 || E < 1 || E > 4096 || H <= 0 || H % 64) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (rows_cap < T * topk + 127LL * E) return FP4_ERR_WORKSPACE;
+  if (ws_bytes < fp4_quantize_workspace_size()) return FP4_ERR_WORKSPACE;
+  if (!aligned16(x_bf16) || !aligned16(a_codes) || !aligned16(workspace)) return FP4_ERR_ALIGNMENT;
+  if (T == 0) return FP4_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const uint16_t *x = static_cast<const uint16_t *>(x_bf16);
+  unsigned int *amax = static_cast<unsigned int *>(workspace);
+  FP4_HOST_CHECK(cudaMemsetAsync(amax, 0, sizeof(unsigned int), s));
+  amax_bf16_kernel<<<grid_for(T * (H / 8)), kThreads, 0, s>>>(x, T, H, H, amax);
+  FP4_HOST_CHECK(cudaGetLastError());
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t grid = T < (int64_t)sms * 16 ? T : (int64_t)sms * 16;
+  nvfp4_quantize_gather_kernel<<<(unsigned)grid, 128, 0, s>>>(x, T, H, topk, E, offsets, tile_offsets, inv, a_codes,
+                                                               a_sf, amax, global_scale);
+  FP4_HOST_CHECK(cudaGetLastError());
+  return FP4_OK;
 }
 
 }  // extern "C"

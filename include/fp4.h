@@ -244,6 +244,16 @@ fp4_status fp4_moe_gather(const uint8_t *x_codes, const uint8_t *x_sf, int64_t T
                           const int32_t *perm, uint8_t *a_codes, uint8_t *a_sf, int64_t rows_cap,
                           fp4_stream_t stream);
 
+/* Dynamic NVFP4 quantize of x fused with the gather: the same codes, scales and
+ * global scale as fp4_quantize(FP4_NV, dynamic) followed by fp4_moe_gather,
+ * written straight into the expert rows (a_codes [rows_cap][H/2], tiled a_sf)
+ * from the routing tables of fp4_moe_route.  global_scale: device fp32[1],
+ * output.  workspace >= fp4_quantize_workspace_size() bytes. */
+fp4_status fp4_moe_quantize_gather(const void *x_bf16, int64_t T, int32_t topk, int64_t H, int32_t E,
+                                   const int32_t *offsets, const int32_t *tile_offsets, const int32_t *inv,
+                                   uint8_t *a_codes, uint8_t *a_sf, int64_t rows_cap, float *global_scale,
+                                   void *workspace, size_t ws_bytes, fp4_stream_t stream);
+
 /* Grouped w13 GEMM + SwiGLU + NVFP4 re-quantize of h with h_g[e]:
  * a = gathered rows (codes [rows_cap][H/2], tiled sf), a_g = fp32[1] tensor
  * scale of x; writes h_codes [rows_cap][I/2] and tiled h_sf for [rows_cap, I]

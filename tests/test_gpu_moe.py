@@ -334,3 +334,28 @@ def test_topk_softmax(T, E, k, grid):
     rid, rw = MO.topk_softmax(z.cpu().numpy(), k)
     assert np.array_equal(ids.cpu().numpy(), rid)
     np.testing.assert_allclose(w.cpu().numpy(), rw, rtol=2e-6, atol=0)
+
+
+@pytest.mark.parametrize("T,H,k,E,zipf", [(300, 1024, 4, 9, 1.1), (1000, 7168, 6, 64, 1.1), (5, 256, 6, 8, 0.0)])
+def test_quantize_gather_fused_bit_exact(T, H, k, E, zipf):
+    """Dynamic NVFP4 quantize written straight into the expert rows: every
+    routed row holds the oracle's codes and scales of its token, and the
+    global scale is the oracle's."""
+    fp4 = _lib()
+    x = synth.activations_bf16((T, H), seed=T + 1, device="cuda")
+    ids, _, _ = synth.router(T, E, k, seed=T + 2, zipf_s=zipf, device="cuda")
+    r = _route_gpu(ids, T, k, E)
+    cap = fp4.moe_rows_cap(T, k, E)
+    a_c = torch.zeros((cap, H // 2), dtype=torch.uint8, device="cuda")
+    a_s = torch.zeros(fp4.fp4_sf_tiled_bytes(cap, H), dtype=torch.uint8, device="cuda")
+    g = torch.empty(1, dtype=torch.float32, device="cuda")
+    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    fp4.fp4_moe_quantize_gather(x, T, k, H, E, r["offsets"], r["tile_offsets"], r["inv"], a_c, a_s, cap, g, ws)
+    counts, offsets, perm, inv = MO.route(ids.cpu().numpy(), E)
+    toff = _tile_offsets_ref(counts)
+    rc, rs, rg = Q.nvfp4_quantize(x.float().cpu().numpy())
+    assert g.cpu().numpy().view(np.uint32)[0] == np.float32(rg).view(np.uint32)
+    pad_rows = np.concatenate([toff[e] * 128 + np.arange(counts[e]) for e in range(E)]).astype(np.int64)
+    tokens = perm // k
+    assert np.array_equal(np_u8(a_c)[pad_rows], rc[tokens])
+    assert np.array_equal(LY.sf_from_mma(np_u8(a_s), cap, H)[pad_rows], rs[tokens])
