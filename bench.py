@@ -409,7 +409,9 @@ def run_moe(args, world, rank, peaks):
         "config": {"workload": b.desc, "tokens": b.T, "hidden": b.H, "intermediate": b.I, "experts": b.E,
                    "topk": b.k, "routed_rows": b.R, "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (weights %.2f GB)" % (b.E * 3 * b.H * b.I * 0.5625 / 1e9),
-                   "experts_touched": int((b.counts > 0).sum().item())},
+                   "experts_touched": int((b.counts > 0).sum().item()),
+                   "tile_rows": int(b.toffs[b.E].item()) * 128,
+                   "padding_frac": round(1.0 - b.R / max(1, int(b.toffs[b.E].item()) * 128), 4)},
         "roofline": {"bound": "tensor", "kernel": "fp4_gemm_kernel<256, w13> (grouped w13 + SwiGLU + requant)",
                      "achieved": round(w13_tf, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
                      "frac": round(w13_tf / fp4_peak, 4), "traffic": measured_traffic(args.workload, "w13"),

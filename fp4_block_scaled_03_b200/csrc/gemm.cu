@@ -29,6 +29,9 @@
 //                          per-expert scale (codes + tiled scales)
 //                 w2       routing weight * alpha * acc -> fp32 rows
 //
+// (w2 stages its stores 32 rows x 8 columns at a time through a 1 KB buffer per
+// warp, so every epilogue keeps the 4-stage pipeline.)
+//
 // The grid is persistent (at most one CTA per SM); every role walks the same
 // tile sequence.  Grouped (MoE) tiles are (128-row tile of one expert's
 // padded rows) x (BN columns of that expert's weights).  Every mbarrier wait
@@ -51,16 +54,15 @@ enum Epi { EPI_F32 = 0, EPI_BF16 = 1, EPI_W13 = 2, EPI_W2 = 3 };
 
 template <int BN, int EPI>
 struct Cfg {
-  // w2 keeps one stage fewer to make room for its store staging buffers
-  static constexpr int kStages = (EPI == 3) ? 3 : 4;
+  static constexpr int kStages = 4;
   static constexpr int A_BYTES = BM * BK_BYTES;
   static constexpr int B_BYTES = BN * BK_BYTES;
   static constexpr int HALVES = (BN + 127) / 128;  // 128-row scale slabs of B per tile
   static constexpr int SFA_BYTES = 4 * 512;
   static constexpr int SFB_BYTES = HALVES * 4 * 512;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-  // w2 epilogue: one 32-row x 32-column fp32 box (4 KB, 128-byte swizzle) per epilogue warp
-  static constexpr int STG_BYTES = (EPI == 3) ? kEpiWarps * 4096 : 0;
+  // w2 epilogue: one 32-row x 8-column fp32 box (1 KB, 32-byte swizzle) per epilogue warp
+  static constexpr int STG_BYTES = (EPI == 3) ? kEpiWarps * 1024 : 0;
   static constexpr int TMEM_COLS = 512;
   static constexpr int ACC_COL = 0;
   static constexpr int SF_SLOT_COLS = 16 + 16 * HALVES;  // SFA: 4 K-words x 4; SFB: 4 x 4*HALVES
@@ -402,20 +404,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 32; i += 4)
             *reinterpret_cast<float4 *>(dst + i) = make_float4(__fmul_rn(w[i], scale), __fmul_rn(w[i + 1], scale),
                                                                __fmul_rn(w[i + 2], scale), __fmul_rn(w[i + 3], scale));
-        } else {  // EPI_W2, all 32 rows valid: stage the box and store it with TMA
-          uint8_t *stg = smStg + (warp - kFirstEpiWarp) * 4096;
-          if (lane == 0) bulk_wait_read_all();  // previous box has left the buffer
-          __syncwarp();
+        } else {  // EPI_W2, all 32 rows valid: stage 32 x 8 boxes and store them with TMA
+          uint8_t *stg = smStg + (warp - kFirstEpiWarp) * 1024;
 #pragma unroll
-          for (int j = 0; j < 8; ++j)  // 16-byte chunk j of row `lane`, 128-byte swizzle
-            *reinterpret_cast<float4 *>(stg + lane * 128 + ((j ^ (lane & 7)) * 16)) =
-                make_float4(__fmul_rn(w[4 * j], scale), __fmul_rn(w[4 * j + 1], scale),
-                            __fmul_rn(w[4 * j + 2], scale), __fmul_rn(w[4 * j + 3], scale));
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(&tmY, stg, col0, ti.out_row0 + q * 32);
-            bulk_commit();
+          for (int bx = 0; bx < 4; ++bx) {
+            if (lane == 0) bulk_wait_read_all();  // previous box has left the buffer
+            __syncwarp();
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {  // 16-byte chunk j of row `lane`, 32-byte swizzle (chunk ^= row bit 2)
+              const int c = 8 * bx + 4 * j;
+              *reinterpret_cast<float4 *>(stg + lane * 32 + ((j ^ ((lane >> 2) & 1)) * 16)) =
+                  make_float4(__fmul_rn(w[c], scale), __fmul_rn(w[c + 1], scale), __fmul_rn(w[c + 2], scale),
+                              __fmul_rn(w[c + 3], scale));
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmY, stg, col0 + 8 * bx, ti.out_row0 + q * 32);
+              bulk_commit();
+            }
           }
         }
       }
@@ -465,17 +472,17 @@ bool make_code_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t row
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// fp32 matrix [rows][cols] as a 2-D tensor map with a 32 x 32 box and
-// 128-byte swizzle (the w2 epilogue's store staging layout).
+// fp32 matrix [rows][cols] as a 2-D tensor map with an 8-column x 32-row box
+// and 32-byte swizzle (the w2 epilogue's store staging layout).
 bool make_f32_store_map(CUtensorMap *m, void *base, uint64_t rows, uint64_t cols) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols * 4};
-  cuuint32_t box[2] = {32, 32};
+  cuuint32_t box[2] = {8, 32};
   cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+            CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
          CUDA_SUCCESS;
 }
 
