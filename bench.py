@@ -490,7 +490,7 @@ def cpu_baseline_moe(b, n_tokens=1):
 
 
 # ---------------------------------------------------------------------------
-def run_dense(args, world, rank, peaks):
+def run_dense(args, world, rank, peaks, mx=False):
     import torch
 
     import fp4_block_scaled_03_b200 as fp4
@@ -499,9 +499,13 @@ def run_dense(args, world, rank, peaks):
     M = N = K = 4096
     a_bf = synth.activations_bf16((M, K), seed=rank, device="cuda")
     b_bf = synth.weights_bf16((N, K), 0.02, 0.005, 30.0, seed=rank + 1, device="cuda")
-    b_c, b_sf, b_g = fp4.quantize_nv(b_bf, tiled=True)
+    if mx:
+        b_c, b_sf = fp4.quantize_mx(b_bf, tiled=True)
+        b_g = None
+    else:
+        b_c, b_sf, b_g = fp4.quantize_nv(b_bf, tiled=True)
     a_c = torch.empty((M, K // 2), dtype=torch.uint8, device="cuda")
-    a_sf = torch.empty(fp4.fp4_sf_tiled_bytes(M, K), dtype=torch.uint8, device="cuda")
+    a_sf = torch.empty(fp4.fp4_sf_tiled_bytes(M, K) // (2 if mx else 1), dtype=torch.uint8, device="cuda")
     a_g = torch.empty(1, dtype=torch.float32, device="cuda")
     ws = torch.empty(256, dtype=torch.uint8, device="cuda")
     c = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
@@ -510,10 +514,12 @@ def run_dense(args, world, rank, peaks):
     def step(ev=None):
         if ev:
             ev[0].record()
-        fp4.fp4_quantize(fp4.FP4_NV, a_bf, M, K, K, a_c, a_sf, a_g, fp4.FP4_SCALE_LAYOUT_TILED, ws, 256)
+        fp4.fp4_quantize(fp4.FP4_MX if mx else fp4.FP4_NV, a_bf, M, K, K, a_c, a_sf, a_g, fp4.FP4_SCALE_LAYOUT_TILED,
+                         ws, 256)
         if ev:
             ev[1].record()
-        fp4.fp4_gemm(a_c, a_sf, a_g, b_c, b_sf, b_g, c, fp4.FP4_OUT_BF16, M, N, K)
+        fp4.fp4_gemm(a_c, a_sf, None if mx else a_g, b_c, b_sf, b_g, c, fp4.FP4_OUT_BF16, M, N, K,
+                     fp4.FP4_GEMM_MX if mx else 0)
         if ev:
             ev[2].record()
 
@@ -546,9 +552,10 @@ def run_dense(args, world, rank, peaks):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e2m1, e4m3/16 scales, fp32 accumulate)",
         "data": "synthetic (seeded)",
-        "config": {"workload": "Dense NVFP4 W4A4 GEMM 4096x4096x4096, activations quantized on device each call, bf16 out",
+        "config": {"workload": ("Dense MXFP4 (UE8M0/32)" if mx else "Dense NVFP4") +
+                   " W4A4 GEMM 4096x4096x4096, activations quantized on device each call, bf16 out",
                    "l2": "flushed (256 MB write) before each timed step"},
-        "roofline": {"bound": "tensor", "kernel": "fp4_gemm_kernel<256, bf16>", "achieved": round(flops / (gms * 1e-3) / 1e12, 1),
+        "roofline": {"bound": "tensor", "kernel": "fp4_gemm_kernel<256, bf16, " + ("mxf4" if mx else "nvf4") + ">", "achieved": round(flops / (gms * 1e-3) / 1e12, 1),
                      "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(flops / (gms * 1e-3) / 1e12 / fp4_peak, 4),
                      "traffic": None, "peak_note": "4 x measured burst bf16 cuBLAS, of " + peaks["src"]},
         "stages_ms": {"quantize": round(q / args.steps, 4), "gemm": round(gms, 4)},
@@ -652,7 +659,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="pro", choices=list(WORKLOADS) + ["dense4096", "quant"])
+    ap.add_argument("--workload", default="pro", choices=list(WORKLOADS) + ["dense4096", "dense4096mx", "quant"])
     ap.add_argument("--impl", default="fp4", choices=["fp4", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -664,8 +671,8 @@ def main():
         line = run_reference(args, world, rank)
     elif args.workload in WORKLOADS:
         line = run_moe(args, world, rank, peaks)
-    elif args.workload == "dense4096":
-        line = run_dense(args, world, rank, peaks)
+    elif args.workload in ("dense4096", "dense4096mx"):
+        line = run_dense(args, world, rank, peaks, mx=args.workload.endswith("mx"))
     else:
         line = run_quant(args, world, rank, peaks)
     if rank == 0 and line is not None:

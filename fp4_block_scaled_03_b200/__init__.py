@@ -23,6 +23,7 @@ FP4_OUT_F32, FP4_OUT_BF16 = 0, 1
 FP4_STATIC_GLOBAL_SCALE = 0x1
 FP4_SCALE_LAYOUT_TILED = 0x2
 FP4_DEBUG_DUMP_H = 0x4
+FP4_GEMM_MX = 0x8
 
 STATUS = {
     0: "FP4_OK",
@@ -241,12 +242,16 @@ def quantize_nv(x, g=None, tiled=False):
     return codes, scales, gs
 
 
-def quantize_mx(x):
+def quantize_mx(x, tiled=False):
     rows, cols = x.shape
     dev = x.device
     codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
-    scales = torch.empty((rows, cols // 32), dtype=torch.uint8, device=dev)
-    fp4_quantize(FP4_MX, x, rows, cols, x.stride(0), codes, scales, None, 0, None, 0)
+    if tiled:
+        scales = _u8(fp4_sf_tiled_bytes(rows, cols) // 2, dev)
+    else:
+        scales = torch.empty((rows, cols // 32), dtype=torch.uint8, device=dev)
+    fp4_quantize(FP4_MX, x, rows, cols, x.stride(0), codes, scales, None, FP4_SCALE_LAYOUT_TILED if tiled else 0,
+                 None, 0)
     return codes, scales
 
 
@@ -262,10 +267,10 @@ def mx_to_nv(codes, mx_scales, num_tensors, tiled=False):
     return nv, g
 
 
-def gemm(a_codes, a_sf, a_g, b_codes, b_sf, b_g, M, N, K, out_dtype=torch.float32):
+def gemm(a_codes, a_sf, a_g, b_codes, b_sf, b_g, M, N, K, out_dtype=torch.float32, mx=False):
     c = torch.empty((M, N), dtype=out_dtype, device=a_codes.device)
     fp4_gemm(a_codes, a_sf, a_g, b_codes, b_sf, b_g, c, FP4_OUT_F32 if out_dtype == torch.float32 else FP4_OUT_BF16,
-             M, N, K)
+             M, N, K, FP4_GEMM_MX if mx else 0)
     return c
 
 

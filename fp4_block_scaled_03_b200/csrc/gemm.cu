@@ -80,7 +80,8 @@ struct Params {
   int n_tiles;       // ceil(N / BN)
   int m_tiles;       // dense only
   int k_stages;      // ceil(K / 256)
-  int kw;            // K / 64 (scale words per row)
+  int kw;            // K / 64 (MMA K steps per row)
+  int kw_sf;         // scale words (4 scales) per row: K / 64 (NVFP4) or K / 128 (MXFP4)
   const uint8_t *a_sf;
   const uint8_t *b_sf;
   int64_t b_sf_rows;  // rows covered by b's tiled scale buffer (padded to 128)
@@ -153,12 +154,14 @@ __device__ __forceinline__ float silu_f32(float z) {
   return __fdiv_rn(z, __fadd_rn(1.0f, expf(-z)));
 }
 
-template <int BN, int EPI>
+template <int BN, int EPI, bool MX>
 __global__ void __launch_bounds__(kThreads, 1)
     fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmY, const Params p) {
   using C = Cfg<BN, EPI>;
   constexpr bool kGrouped = (EPI == EPI_W13 || EPI == EPI_W2);
+  constexpr int WPS = MX ? 2 : 4;   // scale words per row per 256-element stage
+  static_assert(!MX || !kGrouped, "MXFP4 operands are wired for the dense GEMM");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *smA = smem;
@@ -222,7 +225,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kt = 0; kt < p.k_stages; ++kt) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, &s_abort, p.status, lim)) { ok = false; break; }
           const int nk = min(4, p.kw - kt * 4);
-          const uint32_t sf_bytes = (uint32_t)nk * 512u;
+          const int nw = MX ? (nk + 1) / 2 : nk;  // scale words this stage
+          const uint32_t sf_bytes = (uint32_t)nw * 512u;
           int halves = 0;
           for (int h = 0; h < C::HALVES; ++h)
             if ((int64_t)(b_slab0 + h) * 128 < p.b_sf_rows) ++halves;
@@ -230,11 +234,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(&full[stage], bytes);
           tma_load_2d(smA + stage * C::A_BYTES, &tmA, &full[stage], kt * BK_BYTES, ti.a_row0);
           tma_load_2d(smB + stage * C::B_BYTES, &tmB, &full[stage], kt * BK_BYTES, ti.b_row0);
-          bulk_load(smSFA + stage * C::SFA_BYTES, p.a_sf + ((int64_t)ti.a_slab * p.kw + kt * 4) * 512, sf_bytes,
+          bulk_load(smSFA + stage * C::SFA_BYTES, p.a_sf + ((int64_t)ti.a_slab * p.kw_sf + kt * WPS) * 512, sf_bytes,
                     &full[stage]);
           for (int h = 0; h < halves; ++h)
-            bulk_load(smSFB + stage * C::SFB_BYTES + h * 4 * 512,
-                      p.b_sf + ((int64_t)(b_slab0 + h) * p.kw + kt * 4) * 512, sf_bytes, &full[stage]);
+            bulk_load(smSFB + stage * C::SFB_BYTES + h * WPS * 512,
+                      p.b_sf + ((int64_t)(b_slab0 + h) * p.kw_sf + kt * WPS) * 512, sf_bytes, &full[stage]);
           issued[stage] = 1;
           issued_par[stage] = phase;
           if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
@@ -256,18 +260,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait(&full[stage], phase, &s_abort, p.status, lim)) { ok = false; break; }
           tc_fence_after();
           const int nk = min(4, p.kw - kt * 4);
+          const int nw = MX ? (nk + 1) / 2 : nk;
           const uint32_t ta = tmem + C::SF_COL0 + stage * C::SF_SLOT_COLS;
           const uint32_t tb = ta + 16;
           // descriptors of the first 512-byte scale tile; tile i is +i*512 bytes (+i*32 in 16-byte units)
           const uint64_t da = smem_desc(smem_u32(smSFA + stage * C::SFA_BYTES), 0, 128, 0);
           const uint64_t db = smem_desc(smem_u32(smSFB + stage * C::SFB_BYTES), 0, 128, 0);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            if (j < nk) {
-              tmem_cp_sf(ta + j * 4, da + (uint64_t)(j * 32));
+          for (int w = 0; w < WPS; ++w) {
+            if (w < nw) {
+              tmem_cp_sf(ta + w * 4, da + (uint64_t)(w * 32));
 #pragma unroll
               for (int h = 0; h < C::HALVES; ++h)
-                tmem_cp_sf(tb + j * 4 * C::HALVES + h * 4, db + (uint64_t)((h * 4 + j) * 32));
+                tmem_cp_sf(tb + w * 4 * C::HALVES + h * 4, db + (uint64_t)((h * WPS + w) * 32));
             }
           }
           any = true;
@@ -283,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_mxf4nvf4(BM, BN);
+      constexpr uint32_t idesc = MX ? idesc_mxf4(BM, BN) : idesc_mxf4nvf4(BM, BN);
       int stage = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true, any_mma = false;
@@ -302,10 +307,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t ad = smem_desc(smem_u32(smA + stage * C::A_BYTES), 16, 1024, 2);
           const uint64_t bd = smem_desc(smem_u32(smB + stage * C::B_BYTES), 16, 1024, 2);
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            if (j < nk)
-              mma_nvf4(t_acc, ad + (uint64_t)(j * 2), bd + (uint64_t)(j * 2), idesc, ta + j * 4,
-                       tb + j * 4 * C::HALVES, (kt > 0 || j > 0) ? 1u : 0u);
+          for (int j = 0; j < 4; ++j) {
+            if (j < nk) {
+              if (MX) {  // K step j: scale word j/2, bytes 2*(j%2) and 2*(j%2)+1
+                const uint32_t byte = 2u * (uint32_t)(j & 1);
+                const uint32_t w = (uint32_t)(j >> 1);
+                mma_mxf4(t_acc, ad + (uint64_t)(j * 2), bd + (uint64_t)(j * 2), idesc | (byte << 29) | (byte << 4),
+                         (ta + w * 4) | (byte << 30), (tb + w * 4 * C::HALVES) | (byte << 30),
+                         (kt > 0 || j > 0) ? 1u : 0u);
+              } else {
+                mma_nvf4(t_acc, ad + (uint64_t)(j * 2), bd + (uint64_t)(j * 2), idesc, ta + j * 4,
+                         tb + j * 4 * C::HALVES, (kt > 0 || j > 0) ? 1u : 0u);
+              }
+            }
+          }
           any_mma = true;
           tc_commit(&empty[stage]);
           if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
@@ -347,7 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool full_box = (EPI == EPI_W2) && (q * 32 + 32 <= ti.rows_valid);
       if (!row_ok) continue;
       float alpha;
-      if (EPI == EPI_F32 || EPI == EPI_BF16) alpha = __fmul_rn(*p.a_g, *p.b_g);
+      if (EPI == EPI_F32 || EPI == EPI_BF16) alpha = MX ? 1.0f : __fmul_rn(*p.a_g, *p.b_g);
       else if (EPI == EPI_W13) alpha = __fmul_rn(*p.a_g, p.w_g[ti.e]);
       else alpha = __fmul_rn(p.h_g[ti.e], p.w_g[ti.e]);
       float scale = alpha;
@@ -493,11 +508,11 @@ int sm_count() {
   return sms;
 }
 
-template <int BN, int EPI>
+template <int BN, int EPI, bool MX = false>
 fp4_status launch(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &ty, const Params &p, int grid,
                   cudaStream_t s) {
   using C = Cfg<BN, EPI>;
-  auto kern = fp4_gemm_kernel<BN, EPI>;
+  auto kern = fp4_gemm_kernel<BN, EPI, MX>;
   FP4_HOST_CHECK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
   kern<<<grid, kThreads, C::SMEM_BYTES, s>>>(ta, tb, ty, p);
   FP4_HOST_CHECK(cudaGetLastError());
@@ -518,10 +533,10 @@ extern "C" {
 fp4_status fp4_gemm(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_g, const uint8_t *b_codes,
                     const uint8_t *b_sf, const float *b_g, void *c, fp4_out_dtype c_dtype, int64_t M, int64_t N,
                     int64_t K, uint32_t flags, fp4_stream_t stream) {
-  (void)flags;
-  if (!a_codes || !a_sf || !a_g || !b_codes || !b_sf || !b_g || !c) return FP4_ERR_INVALID_ARG;
+  const bool mx = flags & FP4_GEMM_MX;
+  if (!a_codes || !a_sf || !b_codes || !b_sf || !c || (!mx && (!a_g || !b_g))) return FP4_ERR_INVALID_ARG;
   if (c_dtype != FP4_OUT_F32 && c_dtype != FP4_OUT_BF16) return FP4_ERR_INVALID_ARG;
-  if (M < 1 || N < 1 || K < 64 || K % 64 || N % 8) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (M < 1 || N < 1 || K < 64 || K % 64 || N % 8 || (mx && K % 128)) return FP4_ERR_UNSUPPORTED_SHAPE;
   if (M > (1LL << 30) || N > (1LL << 30) || K > (1LL << 30)) return FP4_ERR_UNSUPPORTED_SHAPE;
   if (!al16(a_codes) || !al16(b_codes) || !al16(a_sf) || !al16(b_sf) || !al16(c)) return FP4_ERR_ALIGNMENT;
   const DeviceCtx *ctx = device_ctx();
@@ -535,6 +550,7 @@ fp4_status fp4_gemm(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_
   p.m_tiles = (int)((M + BM - 1) / BM);
   p.k_stages = (int)((K + 255) / 256);
   p.kw = (int)(K / 64);
+  p.kw_sf = mx ? (int)(K / 128) : (int)(K / 64);
   p.a_sf = a_sf; p.b_sf = b_sf;
   p.b_sf_rows = ((N + 127) / 128) * 128;
   p.a_g = a_g; p.b_g = b_g; p.c = c;
@@ -544,6 +560,10 @@ fp4_status fp4_gemm(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_
   if (tiles > 2147483647LL) return FP4_ERR_UNSUPPORTED_SHAPE;
   const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (mx) {
+    if (c_dtype == FP4_OUT_F32) return launch<kBN, EPI_F32, true>(ta, tb, tb, p, grid, s);
+    return launch<kBN, EPI_BF16, true>(ta, tb, tb, p, grid, s);
+  }
   if (c_dtype == FP4_OUT_F32) return launch<kBN, EPI_F32>(ta, tb, tb, p, grid, s);
   return launch<kBN, EPI_BF16>(ta, tb, tb, p, grid, s);
 }
@@ -571,6 +591,7 @@ fp4_status fp4_moe_w13(const uint8_t *a_codes, const uint8_t *a_sf, const float 
   p.n_tiles = (int)(2 * I / kBN);
   p.k_stages = (int)(H / 256);
   p.kw = (int)(H / 64);
+  p.kw_sf = p.kw;
   p.a_sf = a_sf; p.b_sf = w->w13_sf;
   p.b_sf_rows = (int64_t)E * 2 * I;
   p.a_g = a_g;
@@ -603,6 +624,7 @@ fp4_status fp4_moe_w2(const uint8_t *h_codes, const uint8_t *h_sf, const fp4_moe
   p.n_tiles = (int)(H / kBN);
   p.k_stages = (int)(I / 256);
   p.kw = (int)(I / 64);
+  p.kw_sf = p.kw;
   p.a_sf = h_sf; p.b_sf = w->w2_sf;
   p.b_sf_rows = (int64_t)E * H;
   p.E = E; p.counts = counts; p.offsets = offsets; p.tile_offsets = tile_offsets;

@@ -195,6 +195,7 @@ __global__ void __launch_bounds__(128) nvfp4_quantize_gather_kernel(
 }
 
 // ---- MXFP4 quantize: one thread per 32-element block -----------------------
+template <bool kTiled>
 __global__ void __launch_bounds__(kThreads) mxfp4_quantize_kernel(const uint16_t *__restrict__ x, int64_t rows,
                                                                   int64_t cols, int64_t ld,
                                                                   uint8_t *__restrict__ codes,
@@ -232,7 +233,10 @@ __global__ void __launch_bounds__(kThreads) mxfp4_quantize_kernel(const uint16_t
     }
     const uint4 out = make_uint4(pack8_e2m1(f), pack8_e2m1(f + 8), pack8_e2m1(f + 16), pack8_e2m1(f + 24));
     *reinterpret_cast<uint4 *>(codes + r * (cols / 2) + b * 16) = out;
-    scales[i] = (uint8_t)scale;
+    if (kTiled)  // same tile as NVFP4 with 32-element blocks: 4 scales per row per 128 columns
+      scales[sf_tiled_offset(r, b, cols / 128)] = (uint8_t)scale;
+    else
+      scales[i] = (uint8_t)scale;
   }
 }
 
@@ -324,13 +328,16 @@ fp4_status fp4_quantize(fp4_format fmt, const void *x_bf16, int64_t rows, int64_
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (rows == 0) return FP4_OK;
   const uint16_t *x = static_cast<const uint16_t *>(x_bf16);
+  const bool tiled = flags & FP4_SCALE_LAYOUT_TILED;
   if (fmt == FP4_MX) {
-    if (cols % 32) return FP4_ERR_UNSUPPORTED_SHAPE;
-    mxfp4_quantize_kernel<<<grid_for(rows * (cols / 32)), kThreads, 0, s>>>(x, rows, cols, ld, codes, scales);
+    if (cols % 32 || (tiled && cols % 128)) return FP4_ERR_UNSUPPORTED_SHAPE;
+    if (tiled)
+      mxfp4_quantize_kernel<true><<<grid_for(rows * (cols / 32)), kThreads, 0, s>>>(x, rows, cols, ld, codes, scales);
+    else
+      mxfp4_quantize_kernel<false><<<grid_for(rows * (cols / 32)), kThreads, 0, s>>>(x, rows, cols, ld, codes, scales);
     FP4_HOST_CHECK(cudaGetLastError());
     return FP4_OK;
   }
-  const bool tiled = flags & FP4_SCALE_LAYOUT_TILED;
   if (cols % 16 || (tiled && cols % 64)) return FP4_ERR_UNSUPPORTED_SHAPE;
   if (!global_scale) return FP4_ERR_INVALID_ARG;
   const bool stat = flags & FP4_STATIC_GLOBAL_SCALE;

@@ -75,6 +75,7 @@ typedef enum { FP4_OUT_F32 = 0, FP4_OUT_BF16 = 1 } fp4_out_dtype;
 #define FP4_STATIC_GLOBAL_SCALE 0x1u /* fp4_quantize(NV): *global_scale is an input */
 #define FP4_SCALE_LAYOUT_TILED 0x2u  /* fp4_quantize(NV): write scales in the tiled layout */
 #define FP4_DEBUG_DUMP_H 0x4u        /* MoE w13 stage: also write fp32 h */
+#define FP4_GEMM_MX 0x8u             /* fp4_gemm: MXFP4 operands (UE8M0 per 32) */
 
 /* Human-readable name of a status code (static string). */
 const char *fp4_status_string(fp4_status s);
@@ -101,8 +102,10 @@ size_t fp4_quantize_workspace_size(void);
  *   (dynamic mode only; may be NULL with FP4_STATIC_GLOBAL_SCALE).
  * FP4_MX (cols % 32 == 0): per 32-element block X = clamp(floor(log2 amax)-2,
  *   -127, 127), scale byte X+127 (0 for an all-zero block), code =
- *   E2M1_RNE(x * 2^-X).  scales: UE8M0 [rows][cols/32].  global_scale,
- *   workspace and flags are ignored.
+ *   E2M1_RNE(x * 2^-X).  scales: UE8M0 [rows][cols/32], or with
+ *   FP4_SCALE_LAYOUT_TILED (cols % 128 == 0) the tiled layout with 32-element
+ *   blocks (n_ksteps = cols/128; size fp4_sf_tiled_bytes(rows, cols) / 2).
+ *   global_scale and workspace are ignored.
  * Alignment: x, codes, workspace 16-byte aligned; ld*2 % 16 == 0.
  */
 fp4_status fp4_quantize(fp4_format fmt, const void *x_bf16, int64_t rows, int64_t cols, int64_t ld,
@@ -136,6 +139,10 @@ fp4_status fp4_mx_to_nv(const uint8_t *codes, const uint8_t *mx_scales, int64_t 
  * TILED scale buffers (fp4_sf_tiled_bytes(M,K) / (N,K)); a_g/b_g device fp32[1].
  * c: row-major [M,N], fp32 or bf16 (RNE).  fp32 accumulation in tensor memory.
  * Shapes: M,N >= 1; K % 64 == 0; N % 8 == 0.  Codes 16-byte aligned.
+ * With flags & FP4_GEMM_MX: MXFP4 operands [NVFP4 §三] -- a_sf/b_sf are UE8M0
+ * scales per 32 elements in the tiled layout with 32-element blocks (from
+ * fp4_quantize(FP4_MX, FP4_SCALE_LAYOUT_TILED)); a_g/b_g are ignored (may be
+ * NULL); C = A_dq . B_dq^T; K % 128 == 0.
  */
 fp4_status fp4_gemm(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_g,
                     const uint8_t *b_codes, const uint8_t *b_sf, const float *b_g, void *c,

@@ -15,7 +15,7 @@ one bf16 ulp of RNE_bf16(C_ref).
 """
 import numpy as np
 
-from .quant import nvfp4_dequantize
+from .quant import mxfp4_dequantize, nvfp4_dequantize
 
 FP32_REL_TOL = 1e-4
 
@@ -24,6 +24,14 @@ def nvfp4_gemm_ref(a_packed, a_sf, a_g, b_packed, b_sf, b_g):
     """fp64 C [M, N] and the error-bound matrix |A_dq| @ |B_dq|^T."""
     a = nvfp4_dequantize(a_packed, a_sf, a_g)
     b = nvfp4_dequantize(b_packed, b_sf, b_g)
+    return a @ b.T, np.abs(a) @ np.abs(b).T
+
+
+def mxfp4_gemm_ref(a_packed, a_scales, b_packed, b_scales):
+    """MXFP4 x MXFP4 ("DeepSeek-V4.1-Flash-NVFP4" §三: one UE8M0 scale per 32
+    elements): fp64 C = A_dq @ B_dq^T and the bound matrix |A_dq| @ |B_dq|^T."""
+    a = mxfp4_dequantize(a_packed, a_scales)
+    b = mxfp4_dequantize(b_packed, b_scales)
     return a @ b.T, np.abs(a) @ np.abs(b).T
 
 

@@ -101,3 +101,47 @@ def test_gemm_4096_cubed_bf16_sampled():
     cb = bf16_bits(c)[np.ix_(rows, cols)]
     ok = _check_bf16(cb, C, bound)
     assert ok.all(), int((~ok).sum())
+
+
+# ---- MXFP4 x MXFP4 (UE8M0 scale per 32 elements) -----------------------------
+
+@pytest.mark.parametrize("rows,cols", [(5, 128), (130, 384), (257, 4096)])
+def test_mx_quantize_tiled_layout(rows, cols):
+    from oracle import layouts as LY
+
+    x = synth.weights_bf16((rows, cols), 0.02, 0.005, 30.0, seed=rows, device="cuda")
+    codes, sc_t = _lib().quantize_mx(x, tiled=True)
+    rc, rs = Q.mxfp4_quantize(f32(x))
+    assert np.array_equal(codes.cpu().numpy(), rc)
+    assert np.array_equal(LY.sf_from_mma(sc_t.cpu().numpy(), rows, cols, block=32), rs)
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 256, 256), (200, 264, 384), (300, 520, 1152)])
+def test_mx_integer_gemm_bit_exact(M, N, K):
+    fp4 = _lib()
+    a = synth.random_codes((M, K // 2), seed=M + 3, device="cuda")
+    b = synth.random_codes((N, K // 2), seed=N + 4, device="cuda")
+    a_sc = tiled_const(fp4.fp4_sf_tiled_bytes(M, K) // 2, 127)  # UE8M0 2^0
+    b_sc = tiled_const(fp4.fp4_sf_tiled_bytes(N, K) // 2, 127)
+    c = fp4.gemm(a, a_sc, None, b, b_sc, None, M, N, K, mx=True).cpu().numpy()
+    ref = (_int_val(a.cpu().numpy()) @ _int_val(b.cpu().numpy()).T).astype(np.float64) / 4.0
+    assert np.array_equal(c.astype(np.float64), ref)
+
+
+@pytest.mark.parametrize("M,N,K,out", [(128, 256, 512, "f32"), (333, 136, 1152, "f32"), (64, 520, 384, "bf16"),
+                                       (512, 512, 4096, "bf16")])
+def test_mx_gemm_within_bound(M, N, K, out):
+    fp4 = _lib()
+    a_bf = synth.activations_bf16((M, K), seed=M + K, device="cuda")
+    b_bf = synth.weights_bf16((N, K), 0.02, 0.005, 30.0, seed=N + K, device="cuda")
+    a_c, a_sc = fp4.quantize_mx(a_bf, tiled=True)
+    b_c, b_sc = fp4.quantize_mx(b_bf, tiled=True)
+    dt = torch.float32 if out == "f32" else torch.bfloat16
+    c = fp4.gemm(a_c, a_sc, None, b_c, b_sc, None, M, N, K, out_dtype=dt, mx=True)
+    C, bound = G.mxfp4_gemm_ref(*Q.mxfp4_quantize(f32(a_bf)), *Q.mxfp4_quantize(f32(b_bf)))
+    if out == "f32":
+        err = np.abs(c.cpu().numpy().astype(np.float64) - C)
+        assert np.all(err <= G.FP32_REL_TOL * bound), float((err / np.maximum(bound, 1e-300)).max())
+    else:
+        ok = _check_bf16(bf16_bits(c), C, bound)
+        assert ok.all(), int((~ok).sum())

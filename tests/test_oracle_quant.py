@@ -220,3 +220,30 @@ def test_mma_layout_permutation():
     assert idx[130, 11] == 5 * 512 + 32 + 3
     sf = np.random.default_rng(6).integers(0, 256, (rows, cols // 16)).astype(np.uint8)
     assert np.array_equal(sf_from_mma(sf_to_mma(sf), rows, cols), sf)
+
+
+def test_mma_layout_permutation_mx_blocks():
+    rows, cols = 130, 384  # block 32: 3 K steps of 128 columns
+    idx = mma_sf_index(rows, cols, block=32)
+    assert idx.shape == (130, 12)
+    assert len(np.unique(idx)) == idx.size
+    # hand-worked: row 97 (slab 0, line 1, column group 3), block 6 (K step 1, byte 2)
+    assert idx[97, 6] == 1 * 512 + 1 * 16 + 3 * 4 + 2
+    # row 129 (slab 1), block 11 (K step 2, byte 3): (1*3 + 2)*512 + 1*16 + 0 + 3
+    assert idx[129, 11] == 5 * 512 + 16 + 3
+    sc = np.random.default_rng(7).integers(0, 255, (rows, cols // 32)).astype(np.uint8)
+    assert np.array_equal(sf_from_mma(sf_to_mma(sc, block=32), rows, cols, block=32), sc)
+
+
+def test_mx_gemm_oracle_integer_case():
+    """All UE8M0 scales 127 (= 1.0): the MX GEMM reduces to the integer matmul."""
+    from oracle import gemm as G
+
+    rng = np.random.default_rng(8)
+    a = rng.integers(0, 16, (20, 256)).astype(np.uint8)
+    b = rng.integers(0, 16, (24, 256)).astype(np.uint8)
+    two = np.array([0, 1, 2, 3, 4, 6, 8, 12])
+    iv = lambda c: np.where(c & 8, -two[c & 7], two[c & 7])  # noqa: E731
+    C, _ = G.mxfp4_gemm_ref(F.pack_nibbles(a), np.full((20, 8), 127, np.uint8), F.pack_nibbles(b),
+                            np.full((24, 8), 127, np.uint8))
+    assert np.array_equal(C * 4, (iv(a) @ iv(b).T).astype(np.float64))
