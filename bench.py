@@ -39,6 +39,8 @@ WORKLOADS = {
     "flash": (4096, 4096, 2048, 256, 6, 0.0, 0.02,
               "Flash-shaped MoE layer: hidden 4096, 256 experts, I 2048, top-6 uniform, 4096 tokens, MX weights remapped"),
     "decode": (64, 7168, 2048, 384, 6, 1.1, 0.01, "Pro-shaped MoE layer at 64 decode tokens (weight-read bound)"),
+    "flashmx": (4096, 4096, 2048, 256, 6, 0.0, 0.02,
+                "Flash-shaped MoE layer run natively in MXFP4 (UE8M0/32 weights, activations and h; no remap)"),
     "pro64": (4096, 7168, 2048, 64, 6, 1.1, 0.01,
               "Pro-shaped expert matrices, 64 experts, 4096 tokens, top-6, Zipf 1.1 (profiling size)"),
 }
@@ -176,6 +178,8 @@ class MoeBench:
         import synth
 
         self.fp4 = fp4
+        self.mx = name.endswith("mx")
+        self.flags = fp4.FP4_MOE_MX if self.mx else 0
         T, H, I, E, k, zipf, sigma, desc = WORKLOADS[name]
         self.T, self.H, self.I, self.E, self.k, self.desc, self.name = T, H, I, E, k, desc, name
         dev = "cuda"
@@ -183,17 +187,23 @@ class MoeBench:
         self.ids, self.w, self.counts = synth.router(T, E, k, seed=seed + 1, zipf_s=zipf, device=dev)
         self.w13_codes = torch.empty((E * 2 * I, H // 2), dtype=torch.uint8, device=dev)
         self.w2_codes = torch.empty((E * H, I // 2), dtype=torch.uint8, device=dev)
-        self.w13_sf = torch.empty(fp4.fp4_sf_tiled_bytes(E * 2 * I, H), dtype=torch.uint8, device=dev)
-        self.w2_sf = torch.empty(fp4.fp4_sf_tiled_bytes(E * H, I), dtype=torch.uint8, device=dev)
+        div = 2 if self.mx else 1
+        self.w13_sf = torch.empty(fp4.fp4_sf_tiled_bytes(E * 2 * I, H) // div, dtype=torch.uint8, device=dev)
+        self.w2_sf = torch.empty(fp4.fp4_sf_tiled_bytes(E * H, I) // div, dtype=torch.uint8, device=dev)
         self.w13_g = torch.empty(E, dtype=torch.float32, device=dev)
         self.w2_g = torch.empty(E, dtype=torch.float32, device=dev)
-        s13, s2 = fp4.fp4_sf_tiled_bytes(2 * I, H), fp4.fp4_sf_tiled_bytes(H, I)
+        s13, s2 = fp4.fp4_sf_tiled_bytes(2 * I, H) // div, fp4.fp4_sf_tiled_bytes(H, I) // div
         for e in range(E):
             for (rows, cols, codes, sf, g, sfb, off) in ((2 * I, H, self.w13_codes, self.w13_sf, self.w13_g, s13, 2),
                                                           (H, I, self.w2_codes, self.w2_sf, self.w2_g, s2, 3)):
                 wb = synth.weights_bf16((rows, cols), sigma, 0.005, 30.0, seed=seed + 1000 * off + e, device=dev)
                 sl = slice(e * rows, (e + 1) * rows)
-                if name == "flash":  # MXFP4 weights remapped losslessly to NVFP4
+                if self.mx:  # MXFP4 weights used as they are
+                    cc, ss = fp4.quantize_mx(wb, tiled=True)
+                    codes[sl] = cc
+                    sf[e * sfb:(e + 1) * sfb] = ss
+                    g[e] = 1.0
+                elif name == "flash":  # MXFP4 weights remapped losslessly to NVFP4
                     mc, ms = fp4.quantize_mx(wb)
                     nv, gg = fp4.mx_to_nv(mc, ms, 1, tiled=True)
                     codes[sl] = mc
@@ -226,7 +236,7 @@ class MoeBench:
         self.perm, self.inv = i32(R), i32(R)
         self.scratch = u8(fp4.fp4_moe_route_scratch_bytes(R, E))
         self.a_c = torch.empty((cap, H // 2), dtype=torch.uint8, device=d)
-        self.a_s = u8(fp4.fp4_sf_tiled_bytes(cap, H))
+        self.a_s = u8(fp4.fp4_sf_tiled_bytes(cap, H))  # (an MX run uses the first half)
         self.h_c = torch.empty((cap, I // 2), dtype=torch.uint8, device=d)
         self.h_s = u8(fp4.fp4_sf_tiled_bytes(cap, I))
         self.y = torch.empty((R, H), dtype=torch.float32, device=d)
@@ -235,10 +245,13 @@ class MoeBench:
                                      self.h_g)
 
     def calibrate(self):
-        """h_g[e] = max|h| over expert e's rows of this batch / 2688 (once)."""
+        """h_g[e] = max|h| over expert e's rows of this batch / 2688 (once;
+        an MXFP4 run needs no tensor scale)."""
         import torch
 
         fp4 = self.fp4
+        if self.mx:
+            return
         dump = torch.zeros((self.cap, self.I), dtype=torch.float32, device="cuda")
         self.step(events=None, dump=dump)
         torch.cuda.synchronize()
@@ -264,13 +277,13 @@ class MoeBench:
         fp4.fp4_moe_route(self.ids, T, k, E, self.counts_d, self.offs, self.toffs, self.perm, self.inv, self.scratch)
         ev(1)
         fp4.fp4_moe_quantize_gather(self.x, T, k, H, E, self.offs, self.toffs, self.inv, self.a_c, self.a_s, cap,
-                                    self.xg, self.qws)
+                                    self.xg, self.qws, self.flags)
         ev(2)
         fp4.fp4_moe_w13(self.a_c, self.a_s, self.xg, self.wset, H, I, E, self.counts_d, self.toffs, cap, self.h_c,
-                        self.h_s, fp4.FP4_DEBUG_DUMP_H if dump is not None else 0, dump)
+                        self.h_s, (fp4.FP4_DEBUG_DUMP_H if dump is not None else 0) | self.flags, dump)
         ev(3)
         fp4.fp4_moe_w2(self.h_c, self.h_s, self.wset, H, I, E, self.counts_d, self.offs, self.toffs, self.perm, self.w,
-                       cap, self.y)
+                       cap, self.y, self.flags)
         ev(4)
         fp4.fp4_moe_combine(self.y, self.inv, T, k, H, self.out)
         ev(5)
@@ -368,7 +381,8 @@ def run_moe(args, world, rank, peaks):
                 s_cmp.wait_event(ev_in[j])
                 if i >= nb:
                     s_cmp.wait_event(ev_out[j])  # step i-2's output has left buffer j
-                fp4.fp4_moe_grouped_gemm(x_d[j], ids_d[j], w_d[j], b.T, b.k, b.wset, b.H, b.I, b.E, out_d[j], ws)
+                fp4.fp4_moe_grouped_gemm(x_d[j], ids_d[j], w_d[j], b.T, b.k, b.wset, b.H, b.I, b.E, out_d[j], ws,
+                                         b.flags)
                 ev_cmp[j].record(s_cmp)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev_cmp[j])
@@ -465,6 +479,8 @@ def cpu_baseline_moe(b, n_tokens=1):
         wb[e] = (w13.float().cpu().numpy(), w2.float().cpu().numpy())
 
     def deq(w):
+        if b.mx:
+            return Q.mxfp4_dequantize(*Q.mxfp4_quantize(w))
         if b.name == "flash":
             c, sc = Q.mxfp4_quantize(w)
             sf, gg = Q.mx_to_nv(c, sc, 1)
@@ -472,14 +488,15 @@ def cpu_baseline_moe(b, n_tokens=1):
         return Q.nvfp4_dequantize(*Q.nvfp4_quantize(w))
 
     t0 = time.perf_counter()
-    x_dq = Q.nvfp4_dequantize(*Q.nvfp4_quantize(xs, g=g))
+    x_dq = Q.mxfp4_dequantize(*Q.mxfp4_quantize(xs)) if b.mx else Q.nvfp4_dequantize(*Q.nvfp4_quantize(xs, g=g))
     dq = {e: (MO.deinterleave_w13(deq(wb[e][0])), deq(wb[e][1])) for e in experts}
     out = np.zeros((n_tokens, b.H))
     for t in range(n_tokens):
         for s in range(b.k):
             e = int(ids[t, s])
             (w1d, w3d), w2d = dq[e]
-            r = MO.expert_ffn_ref(x_dq[t:t + 1], w1d, w3d, w2d, hg[e])
+            r = (MO.expert_ffn_ref_mx(x_dq[t:t + 1], w1d, w3d, w2d) if b.mx
+                 else MO.expert_ffn_ref(x_dq[t:t + 1], w1d, w3d, w2d, hg[e]))
             out[t] += wts[t, s] * r["y"][0]
     dt = time.perf_counter() - t0
     flops = 2.0 * 3 * b.H * b.I * b.k * n_tokens

@@ -24,6 +24,7 @@ FP4_STATIC_GLOBAL_SCALE = 0x1
 FP4_SCALE_LAYOUT_TILED = 0x2
 FP4_DEBUG_DUMP_H = 0x4
 FP4_GEMM_MX = 0x8
+FP4_MOE_MX = 0x10
 
 STATUS = {
     0: "FP4_OK",
@@ -85,14 +86,15 @@ _SIGS = {
     "fp4_moe_route": (ctypes.c_int, [_P, _I64, _I32, _I32, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "fp4_moe_route_noalloc": (ctypes.c_int, [_P, _I64, _I32, _I32, _P, _P, _P, _P, _P, _P]),
     "fp4_moe_gather": (ctypes.c_int, [_P, _P, _I64, _I32, _I64, _I32, _P, _P, _P, _P, _P, _I64, _P]),
-    "fp4_moe_quantize_gather": (ctypes.c_int, [_P, _I64, _I32, _I64, _I32, _P, _P, _P, _P, _P, _I64, _P, _P, _SZ, _P]),
+    "fp4_moe_quantize_gather": (ctypes.c_int,
+                                [_P, _I64, _I32, _I64, _I32, _P, _P, _P, _P, _P, _I64, _P, _P, _SZ, _U32, _P]),
     "fp4_moe_w13": (
         ctypes.c_int,
         [_P, _P, _P, ctypes.POINTER(MoeWeights), _I64, _I64, _I32, _P, _P, _I64, _P, _P, _U32, _P, _P],
     ),
     "fp4_moe_w2": (
         ctypes.c_int,
-        [_P, _P, ctypes.POINTER(MoeWeights), _I64, _I64, _I32, _P, _P, _P, _P, _P, _I64, _P, _P],
+        [_P, _P, ctypes.POINTER(MoeWeights), _I64, _I64, _I32, _P, _P, _P, _P, _P, _I64, _P, _U32, _P],
     ),
     "fp4_moe_combine": (ctypes.c_int, [_P, _P, _I64, _I32, _I64, _P, _P]),
     "fp4_get_device_status": (ctypes.c_int, [_P]),
@@ -165,11 +167,11 @@ def fp4_moe_gather(x_codes, x_sf, T, topk, H, E, offsets, tile_offsets, perm, a_
 
 
 def fp4_moe_quantize_gather(x, T, topk, H, E, offsets, tile_offsets, inv, a_codes, a_sf, rows_cap, global_scale,
-                            workspace):
+                            workspace, flags=0):
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib.fp4_moe_quantize_gather(_ptr(x), T, topk, H, E, _ptr(offsets), _ptr(tile_offsets), _ptr(inv),
                                        _ptr(a_codes), _ptr(a_sf), rows_cap, _ptr(global_scale), _ptr(workspace),
-                                       workspace.numel() * workspace.element_size(), _stream()),
-           "fp4_moe_quantize_gather")
+                                       ws_bytes, flags, _stream()), "fp4_moe_quantize_gather")
 
 
 def fp4_moe_w13(a_codes, a_sf, a_g, w, H, I, E, counts, tile_offsets, rows_cap, h_codes, h_sf, flags=0, h_dump=None):
@@ -178,10 +180,10 @@ def fp4_moe_w13(a_codes, a_sf, a_g, w, H, I, E, counts, tile_offsets, rows_cap, 
            "fp4_moe_w13")
 
 
-def fp4_moe_w2(h_codes, h_sf, w, H, I, E, counts, offsets, tile_offsets, perm, topk_weights, rows_cap, y):
+def fp4_moe_w2(h_codes, h_sf, w, H, I, E, counts, offsets, tile_offsets, perm, topk_weights, rows_cap, y, flags=0):
     _check(lib.fp4_moe_w2(_ptr(h_codes), _ptr(h_sf), ctypes.byref(w.c_struct()), H, I, E, _ptr(counts),
                           _ptr(offsets), _ptr(tile_offsets), _ptr(perm), _ptr(topk_weights), rows_cap, _ptr(y),
-                          _stream()), "fp4_moe_w2")
+                          flags, _stream()), "fp4_moe_w2")
 
 
 def fp4_moe_combine(y, inv, T, topk, H, out):
@@ -291,13 +293,13 @@ def moe_rows_cap(T, topk, E):
     return ((T * topk + 127 * E + 127) // 128) * 128
 
 
-def moe_layer(x, expert_ids, topk_weights, w, H, I, E, workspace=None, out=None, h_dump=None):
+def moe_layer(x, expert_ids, topk_weights, w, H, I, E, workspace=None, out=None, h_dump=None, mx=False):
     T, topk = expert_ids.shape
     dev = x.device
     if workspace is None:
         workspace = _u8(fp4_moe_workspace_size(T, topk, H, I, E), dev)
     if out is None:
         out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
-    flags = FP4_DEBUG_DUMP_H if h_dump is not None else 0
+    flags = (FP4_DEBUG_DUMP_H if h_dump is not None else 0) | (FP4_MOE_MX if mx else 0)
     fp4_moe_grouped_gemm(x, expert_ids, topk_weights, T, topk, w, H, I, E, out, workspace, flags, h_dump)
     return out

@@ -105,6 +105,32 @@ __device__ __forceinline__ uint32_t nvfp4_block16(const float *x, float g, uint3
   return sf;
 }
 
+// MXFP4 quantization of one 32-element block held in fp32 registers: scale
+// exponent X = clamp(floor(log2 amax) - 2, -127, 127), byte X + 127 (0 for an
+// all-zero block), code = E2M1_RNE(x * 2^-X).  Returns the scale byte and
+// writes 16 code bytes.
+__device__ __forceinline__ uint32_t mxfp4_block32(const float *x, uint32_t *codes4) {
+  float a = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) a = fmaxf(a, fabsf(x[i]));
+  int X = 0;
+  uint32_t scale = 0;
+  if (a > 0.0f) {
+    const uint32_t bits = __float_as_uint(a);
+    const int e = (int)(bits >> 23);
+    const int fl = e ? e - 127 : (31 - __clz((int)(bits & 0x7FFFFFu))) - 149;  // exact floor(log2 a)
+    X = min(max(fl - 2, -127), 127);
+    scale = (uint32_t)(X + 127);
+  }
+  const float p = __uint_as_float((uint32_t)(127 - X) << 23);  // 2^-X (X <= 125 for finite fp32)
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(x[i], p);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) codes4[q] = pack8_e2m1(v + 8 * q);
+  return scale;
+}
+
 // ---------------------------------------------------------------------------
 // shared memory, mbarriers, TMA
 // ---------------------------------------------------------------------------

@@ -161,7 +161,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   using C = Cfg<BN, EPI>;
   constexpr bool kGrouped = (EPI == EPI_W13 || EPI == EPI_W2);
   constexpr int WPS = MX ? 2 : 4;   // scale words per row per 256-element stage
-  static_assert(!MX || !kGrouped, "MXFP4 operands are wired for the dense GEMM");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *smA = smem;
@@ -361,13 +360,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       // per warp); otherwise each valid row is stored by its own thread
       const bool full_box = (EPI == EPI_W2) && (q * 32 + 32 <= ti.rows_valid);
       if (!row_ok) continue;
-      float alpha;
-      if (EPI == EPI_F32 || EPI == EPI_BF16) alpha = MX ? 1.0f : __fmul_rn(*p.a_g, *p.b_g);
+      float alpha;  // MXFP4 operands carry no tensor-level scale
+      if (MX) alpha = 1.0f;
+      else if (EPI == EPI_F32 || EPI == EPI_BF16) alpha = __fmul_rn(*p.a_g, *p.b_g);
       else if (EPI == EPI_W13) alpha = __fmul_rn(*p.a_g, p.w_g[ti.e]);
       else alpha = __fmul_rn(p.h_g[ti.e], p.w_g[ti.e]);
       float scale = alpha;
-      if (EPI == EPI_W2 && p.topk_w) scale = __fmul_rn(alpha, p.topk_w[p.perm[ti.out_row0 + row]]);
+      if (EPI == EPI_W2 && p.topk_w) scale = MX ? p.topk_w[p.perm[ti.out_row0 + row]]
+                                                : __fmul_rn(alpha, p.topk_w[p.perm[ti.out_row0 + row]]);
       const int colh = ti.n0 + half * HC;
+      if constexpr (EPI == EPI_W13 && MX) {
+        // MXFP4 h: one 32-element block per pair of 32-column chunks (16 gate +
+        // 16 up columns each), quantized with its own power-of-two scale
+#pragma unroll
+        for (int cp = 0; cp < HC / 64; ++cp) {
+          const int col0 = colh + cp * 64;
+          if (col0 >= p.N) break;
+          float h[32];
+#pragma unroll
+          for (int half2 = 0; half2 < 2; ++half2) {
+            const float *w = v + 64 * cp + 32 * half2;
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              h[16 * half2 + i] = __fmul_rn(silu_f32(__fmul_rn(w[i], scale)), __fmul_rn(w[16 + i], scale));
+          }
+          const int hc = col0 / 2;  // a multiple of 32
+          const int64_t prow = (int64_t)ti.a_row0 + row;
+          uint32_t cq[4];
+          const uint32_t sc = mxfp4_block32(h, cq);
+          *reinterpret_cast<uint4 *>(p.h_codes + prow * (p.I / 2) + hc / 2) = make_uint4(cq[0], cq[1], cq[2], cq[3]);
+          p.h_sf[sf_tiled_offset(prow, hc / 32, p.I / 128)] = (uint8_t)sc;
+          if (p.h_dump) {
+            float4 *d = reinterpret_cast<float4 *>(p.h_dump + prow * p.I + hc);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) d[i] = make_float4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
+          }
+        }
+      } else {
 #pragma unroll
       for (int c = 0; c < HC / 32; ++c) {
         const float *w = v + 32 * c;
@@ -441,6 +470,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      }  // generic epilogue
     }
     if (EPI == EPI_W2 && lane == 0) bulk_wait_all();  // stores complete before the CTA exits
   }
@@ -572,10 +602,11 @@ fp4_status fp4_moe_w13(const uint8_t *a_codes, const uint8_t *a_sf, const float 
                        int64_t H, int64_t I, int32_t E, const int32_t *counts, const int32_t *tile_offsets,
                        int64_t rows_cap, uint8_t *h_codes, uint8_t *h_sf, uint32_t flags, float *h_dump,
                        fp4_stream_t stream) {
-  if (!a_codes || !a_sf || !a_g || !w || !w->w13_codes || !w->w13_sf || !w->w13_g || !w->h_g || !counts ||
-      !tile_offsets || !h_codes || !h_sf)
+  if (!a_codes || !a_sf || !w || !w->w13_codes || !w->w13_sf || !counts || !tile_offsets || !h_codes || !h_sf)
     return FP4_ERR_INVALID_ARG;
+  if (!(flags & FP4_MOE_MX) && (!a_g || !w->w13_g || !w->h_g)) return FP4_ERR_INVALID_ARG;
   if ((flags & FP4_DEBUG_DUMP_H) && !h_dump) return FP4_ERR_INVALID_ARG;
+  const bool mx = flags & FP4_MOE_MX;
   if (H < 256 || H % 256 || I < 256 || I % 256 || E < 1 || E > 4096 || rows_cap < 1) return FP4_ERR_UNSUPPORTED_SHAPE;
   if ((int64_t)E * 2 * I > (1LL << 31) - 1 || rows_cap > (1LL << 31) - 1) return FP4_ERR_UNSUPPORTED_SHAPE;
   if (!al16(a_codes) || !al16(a_sf) || !al16(w->w13_codes) || !al16(w->w13_sf) || !al16(h_codes) || !al16(h_sf) ||
@@ -591,7 +622,7 @@ fp4_status fp4_moe_w13(const uint8_t *a_codes, const uint8_t *a_sf, const float 
   p.n_tiles = (int)(2 * I / kBN);
   p.k_stages = (int)(H / 256);
   p.kw = (int)(H / 64);
-  p.kw_sf = p.kw;
+  p.kw_sf = mx ? (int)(H / 128) : p.kw;
   p.a_sf = a_sf; p.b_sf = w->w13_sf;
   p.b_sf_rows = (int64_t)E * 2 * I;
   p.a_g = a_g;
@@ -601,16 +632,18 @@ fp4_status fp4_moe_w13(const uint8_t *a_codes, const uint8_t *a_sf, const float 
   p.h_dump = (flags & FP4_DEBUG_DUMP_H) ? h_dump : nullptr;
   p.status = ctx->status;
   p.wait_limit = ctx->wait_limit_ns;
+  if (mx) return launch<kBN, EPI_W13, true>(ta, tb, tb, p, sm_count(), reinterpret_cast<cudaStream_t>(stream));
   return launch<kBN, EPI_W13>(ta, tb, tb, p, sm_count(), reinterpret_cast<cudaStream_t>(stream));
 }
 
 fp4_status fp4_moe_w2(const uint8_t *h_codes, const uint8_t *h_sf, const fp4_moe_weights *w, int64_t H, int64_t I,
                       int32_t E, const int32_t *counts, const int32_t *offsets, const int32_t *tile_offsets,
-                      const int32_t *perm, const float *topk_weights, int64_t rows_cap, float *y,
+                      const int32_t *perm, const float *topk_weights, int64_t rows_cap, float *y, uint32_t flags,
                       fp4_stream_t stream) {
-  if (!h_codes || !h_sf || !w || !w->w2_codes || !w->w2_sf || !w->w2_g || !w->h_g || !counts || !offsets ||
-      !tile_offsets || !perm || !y)
+  const bool mx = flags & FP4_MOE_MX;
+  if (!h_codes || !h_sf || !w || !w->w2_codes || !w->w2_sf || !counts || !offsets || !tile_offsets || !perm || !y)
     return FP4_ERR_INVALID_ARG;
+  if (!mx && (!w->w2_g || !w->h_g)) return FP4_ERR_INVALID_ARG;
   if (H < 256 || H % 256 || I < 256 || I % 256 || E < 1 || E > 4096 || rows_cap < 1) return FP4_ERR_UNSUPPORTED_SHAPE;
   if ((int64_t)E * H > (1LL << 31) - 1 || rows_cap > (1LL << 31) - 1) return FP4_ERR_UNSUPPORTED_SHAPE;
   if (!al16(h_codes) || !al16(h_sf) || !al16(w->w2_codes) || !al16(w->w2_sf) || !al16(y)) return FP4_ERR_ALIGNMENT;
@@ -624,7 +657,7 @@ fp4_status fp4_moe_w2(const uint8_t *h_codes, const uint8_t *h_sf, const fp4_moe
   p.n_tiles = (int)(H / kBN);
   p.k_stages = (int)(I / 256);
   p.kw = (int)(I / 64);
-  p.kw_sf = p.kw;
+  p.kw_sf = mx ? (int)(I / 128) : p.kw;
   p.a_sf = h_sf; p.b_sf = w->w2_sf;
   p.b_sf_rows = (int64_t)E * H;
   p.E = E; p.counts = counts; p.offsets = offsets; p.tile_offsets = tile_offsets;
@@ -634,6 +667,7 @@ fp4_status fp4_moe_w2(const uint8_t *h_codes, const uint8_t *h_sf, const fp4_moe
   p.wait_limit = ctx->wait_limit_ns;
   CUtensorMap ty;
   if (!make_f32_store_map(&ty, y, (uint64_t)rows_cap, (uint64_t)H)) return FP4_ERR_CUDA;
+  if (mx) return launch<kBN, EPI_W2, true>(ta, tb, ty, p, sm_count(), reinterpret_cast<cudaStream_t>(stream));
   return launch<kBN, EPI_W2>(ta, tb, ty, p, sm_count(), reinterpret_cast<cudaStream_t>(stream));
 }
 

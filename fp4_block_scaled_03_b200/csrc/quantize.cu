@@ -194,6 +194,57 @@ __global__ void __launch_bounds__(128) nvfp4_quantize_gather_kernel(
   }
 }
 
+// MXFP4 variant: each thread quantizes one 128-element K step (four 32-element
+// blocks) and writes 64 code bytes and one 4-byte UE8M0 scale word per
+// destination row (tiled layout with 32-element blocks).
+__global__ void __launch_bounds__(128) mxfp4_quantize_gather_kernel(
+    const uint16_t *__restrict__ x, int64_t T, int64_t H, int32_t topk, int32_t E,
+    const int32_t *__restrict__ offsets, const int32_t *__restrict__ tile_offsets, const int32_t *__restrict__ inv,
+    uint8_t *__restrict__ a_codes, uint8_t *__restrict__ a_sf) {
+  __shared__ int64_t dst[16];
+  const int64_t n_ksteps = H / 128;
+  for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+    __syncthreads();
+    if (threadIdx.x < topk) {
+      const int32_t r = inv[t * topk + threadIdx.x];
+      int64_t d = -1;
+      if (r >= 0) {
+        const int e = expert_of_row(offsets, E, r);
+        d = (int64_t)tile_offsets[e] * 128 + (r - offsets[e]);
+      }
+      dst[threadIdx.x] = d;
+    }
+    __syncthreads();
+    for (int64_t kw = threadIdx.x; kw < n_ksteps; kw += blockDim.x) {
+      const uint4 *src = reinterpret_cast<const uint4 *>(x + t * H + kw * 128);
+      uint32_t code[16], sfw = 0;
+#pragma unroll
+      for (int blk = 0; blk < 4; ++blk) {
+        float f[32];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint4 v = __ldcs(src + 4 * blk + q);
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            f[8 * q + 2 * j] = bf16_bits_to_f32(w[j] & 0xFFFFu);
+            f[8 * q + 2 * j + 1] = bf16_bits_to_f32(w[j] >> 16);
+          }
+        }
+        sfw |= mxfp4_block32(f, code + 4 * blk) << (8 * blk);
+      }
+      for (int s = 0; s < topk; ++s) {
+        const int64_t d = dst[s];
+        if (d < 0) continue;
+        uint4 *out = reinterpret_cast<uint4 *>(a_codes + d * (H / 2) + kw * 64);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) out[q] = make_uint4(code[4 * q], code[4 * q + 1], code[4 * q + 2], code[4 * q + 3]);
+        *reinterpret_cast<uint32_t *>(a_sf + sf_tiled_offset(d, kw * 4, n_ksteps)) = sfw;
+      }
+    }
+  }
+}
+
 // ---- MXFP4 quantize: one thread per 32-element block -----------------------
 template <bool kTiled>
 __global__ void __launch_bounds__(kThreads) mxfp4_quantize_kernel(const uint16_t *__restrict__ x, int64_t rows,
@@ -394,16 +445,28 @@ fp4_status fp4_mx_to_nv(const uint8_t *codes, const uint8_t *mx_scales, int64_t 
 fp4_status fp4_moe_quantize_gather(const void *x_bf16, int64_t T, int32_t topk, int64_t H, int32_t E,
                                    const int32_t *offsets, const int32_t *tile_offsets, const int32_t *inv,
                                    uint8_t *a_codes, uint8_t *a_sf, int64_t rows_cap, float *global_scale,
-                                   void *workspace, size_t ws_bytes, fp4_stream_t stream) {
-  if (!x_bf16 || !offsets || !tile_offsets || !inv || !a_codes || !a_sf || !global_scale || !workspace)
-    return FP4_ERR_INVALID_ARG;
-  if (T < 0 || topk < 1 || topk > 16 || E < 1 || E > 4096 || H <= 0 || H % 64) return FP4_ERR_UNSUPPORTED_SHAPE;
+                                   void *workspace, size_t ws_bytes, uint32_t flags, fp4_stream_t stream) {
+  const bool mx = flags & FP4_MOE_MX;
+  if (!x_bf16 || !offsets || !tile_offsets || !inv || !a_codes || !a_sf) return FP4_ERR_INVALID_ARG;
+  if (!mx && (!global_scale || !workspace)) return FP4_ERR_INVALID_ARG;
+  if (T < 0 || topk < 1 || topk > 16 || E < 1 || E > 4096 || H <= 0 || H % 64 || (mx && H % 128))
+    return FP4_ERR_UNSUPPORTED_SHAPE;
   if (rows_cap < T * topk + 127LL * E) return FP4_ERR_WORKSPACE;
-  if (ws_bytes < fp4_quantize_workspace_size()) return FP4_ERR_WORKSPACE;
-  if (!aligned16(x_bf16) || !aligned16(a_codes) || !aligned16(workspace)) return FP4_ERR_ALIGNMENT;
+  if (!mx && ws_bytes < fp4_quantize_workspace_size()) return FP4_ERR_WORKSPACE;
+  if (!aligned16(x_bf16) || !aligned16(a_codes) || (!mx && !aligned16(workspace))) return FP4_ERR_ALIGNMENT;
   if (T == 0) return FP4_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const uint16_t *x = static_cast<const uint16_t *>(x_bf16);
+  if (mx) {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t grid = T < (int64_t)sms * 16 ? T : (int64_t)sms * 16;
+    mxfp4_quantize_gather_kernel<<<(unsigned)grid, 128, 0, s>>>(x, T, H, topk, E, offsets, tile_offsets, inv,
+                                                                 a_codes, a_sf);
+    FP4_HOST_CHECK(cudaGetLastError());
+    return FP4_OK;
+  }
   unsigned int *amax = static_cast<unsigned int *>(workspace);
   FP4_HOST_CHECK(cudaMemsetAsync(amax, 0, sizeof(unsigned int), s));
   amax_bf16_kernel<<<grid_for(T * (H / 8)), kThreads, 0, s>>>(x, T, H, H, amax);

@@ -76,6 +76,7 @@ typedef enum { FP4_OUT_F32 = 0, FP4_OUT_BF16 = 1 } fp4_out_dtype;
 #define FP4_SCALE_LAYOUT_TILED 0x2u  /* fp4_quantize(NV): write scales in the tiled layout */
 #define FP4_DEBUG_DUMP_H 0x4u        /* MoE w13 stage: also write fp32 h */
 #define FP4_GEMM_MX 0x8u             /* fp4_gemm: MXFP4 operands (UE8M0 per 32) */
+#define FP4_MOE_MX 0x10u             /* MoE layer / stages: MXFP4 weights, activations and h */
 
 /* Human-readable name of a status code (static string). */
 const char *fp4_status_string(fp4_status s);
@@ -170,6 +171,13 @@ fp4_status fp4_gemm(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_
  * Routed rows are ordered by (expert, token, slot) and padded per expert to
  * a multiple of 128 rows.
  * Shapes: H % 256 == 0, I % 256 == 0, 1 <= topk <= 16, 1 <= E <= 4096.
+ *
+ * MXFP4 variant (flags FP4_MOE_MX) [NVFP4 §三; ARCH §6.3]: the experts stay in
+ * their MXFP4 form (no remap): w13_sf / w2_sf hold UE8M0 scales per 32
+ * elements in the tiled layout with 32-element blocks; w13_g, w2_g and h_g
+ * are unused (may be NULL).  x is MXFP4-quantized (per 32-block power-of-two
+ * scale, no tensor scale), h is re-quantized to MXFP4 per 32-element block in
+ * the w13 epilogue, and y = w[t,s] * h_q.W2_e^T.
  * ------------------------------------------------------------------------- */
 typedef struct {
   const uint8_t *w13_codes;
@@ -255,17 +263,19 @@ fp4_status fp4_moe_gather(const uint8_t *x_codes, const uint8_t *x_sf, int64_t T
  * global scale as fp4_quantize(FP4_NV, dynamic) followed by fp4_moe_gather,
  * written straight into the expert rows (a_codes [rows_cap][H/2], tiled a_sf)
  * from the routing tables of fp4_moe_route.  global_scale: device fp32[1],
- * output.  workspace >= fp4_quantize_workspace_size() bytes. */
+ * output.  workspace >= fp4_quantize_workspace_size() bytes.
+ * With FP4_MOE_MX: MXFP4 instead (UE8M0 per 32, tiled with 32-element blocks,
+ * H % 128 == 0); global_scale and workspace are unused (may be NULL). */
 fp4_status fp4_moe_quantize_gather(const void *x_bf16, int64_t T, int32_t topk, int64_t H, int32_t E,
                                    const int32_t *offsets, const int32_t *tile_offsets, const int32_t *inv,
                                    uint8_t *a_codes, uint8_t *a_sf, int64_t rows_cap, float *global_scale,
-                                   void *workspace, size_t ws_bytes, fp4_stream_t stream);
+                                   void *workspace, size_t ws_bytes, uint32_t flags, fp4_stream_t stream);
 
 /* Grouped w13 GEMM + SwiGLU + NVFP4 re-quantize of h with h_g[e]:
  * a = gathered rows (codes [rows_cap][H/2], tiled sf), a_g = fp32[1] tensor
  * scale of x; writes h_codes [rows_cap][I/2] and tiled h_sf for [rows_cap, I]
  * (only rows that hold a routed row are written). h_dump (FP4_DEBUG_DUMP_H):
- * fp32 [rows_cap][I]. */
+ * fp32 [rows_cap][I].  FP4_MOE_MX: MXFP4 operands and h (a_g unused). */
 fp4_status fp4_moe_w13(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_g,
                        const fp4_moe_weights *w, int64_t H, int64_t I, int32_t E,
                        const int32_t *counts, const int32_t *tile_offsets, int64_t rows_cap,
@@ -273,11 +283,13 @@ fp4_status fp4_moe_w13(const uint8_t *a_codes, const uint8_t *a_sf, const float 
                        fp4_stream_t stream);
 
 /* Grouped w2 GEMM: y[offsets[e]+i] = w[perm[row]] * h_g[e]*w2_g[e] * (h . W2_e^T)
- * y: fp32 [T*topk][H] in routed order; topk_weights may be NULL. */
+ * y: fp32 [T*topk][H] in routed order; topk_weights may be NULL.
+ * FP4_MOE_MX: MXFP4 operands, y = w * (h . W2_e^T). */
 fp4_status fp4_moe_w2(const uint8_t *h_codes, const uint8_t *h_sf, const fp4_moe_weights *w,
                       int64_t H, int64_t I, int32_t E, const int32_t *counts,
                       const int32_t *offsets, const int32_t *tile_offsets, const int32_t *perm,
-                      const float *topk_weights, int64_t rows_cap, float *y, fp4_stream_t stream);
+                      const float *topk_weights, int64_t rows_cap, float *y, uint32_t flags,
+                      fp4_stream_t stream);
 
 /* out[t] = bf16_RNE(sum_{s=0..k-1} y[inv[t*k+s]]) (fp32 adds in slot order;
  * inv < 0 contributes nothing). */

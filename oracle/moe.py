@@ -21,7 +21,7 @@ caller's top-k weight (1.0 when none is given) and sums slots in order 0..k-1.
 import numpy as np
 
 from .formats import f64_to_bf16_rne
-from .quant import nvfp4_dequantize, nvfp4_quantize
+from .quant import mxfp4_dequantize, mxfp4_quantize, nvfp4_dequantize, nvfp4_quantize
 
 
 def route(expert_ids, num_experts):
@@ -77,6 +77,19 @@ def expert_ffn_ref(x_dq_rows, w1_dq, w3_dq, w2_dq, g_h):
     h_dq = nvfp4_dequantize(h_codes, h_sf, g_h)
     y = h_dq @ w2_dq.T
     return dict(gate=gate, up=up, h=h, h_codes=h_codes, h_sf=h_sf, h_dq=h_dq, y=y)
+
+
+def expert_ffn_ref_mx(x_dq_rows, w1_dq, w3_dq, w2_dq):
+    """MXFP4 variant of expert_ffn_ref: h is re-quantized to MXFP4 (one
+    power-of-two scale per 32 elements, no tensor scale) from h rounded once
+    to fp32."""
+    gate = x_dq_rows @ w1_dq.T
+    up = x_dq_rows @ w3_dq.T
+    h = swiglu(gate, up)
+    h_codes, h_sc = mxfp4_quantize(h.astype(np.float32))
+    h_dq = mxfp4_dequantize(h_codes, h_sc)
+    y = h_dq @ w2_dq.T
+    return dict(gate=gate, up=up, h=h, h_codes=h_codes, h_sc=h_sc, h_dq=h_dq, y=y)
 
 
 def combine_ref(y_rows, inv, topk_weights=None):
