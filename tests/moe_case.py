@@ -90,3 +90,51 @@ def oracle_x(c):
         return xq, Q.mxfp4_dequantize(*xq)
     xq = Q.nvfp4_quantize(c.x_f32)
     return xq, Q.nvfp4_dequantize(*xq)
+
+
+def oracle_token_rows(x_dq_rows, experts_w, slot_weights, g_h, fmt, h_tol_fn):
+    """Oracle output rows of a few tokens and the per-element slack the
+    layer bar allows (see test_gpu_moe.test_layer_end_to_end).
+
+    x_dq_rows: fp64 [n, H]; experts_w: per token, a list of k (w1, w3, w2)
+    dequantized fp64 matrices; slot_weights: fp64 [n, k]; g_h: per token, a
+    list of k h tensor scales (NV) or None (MX)."""
+    from oracle import formats as F
+    from oracle import gemm as G
+
+    n, H = x_dq_rows.shape
+    ref = np.zeros((n, H))
+    slack = np.zeros((n, H))
+    sum_abs = np.zeros((n, H))
+    for t in range(n):
+        for s, (w1, w3, w2) in enumerate(experts_w[t]):
+            xr = x_dq_rows[t:t + 1]
+            gate, up = xr @ w1.T, xr @ w3.T
+            h = MO.swiglu(gate, up)
+            tol = h_tol_fn(xr, w1, w3, gate, up, h)
+            blk = 32 if fmt == "mx" else 16
+            if fmt == "mx":
+                hc, hs = Q.mxfp4_quantize(h.astype(np.float32))
+                h_dq = Q.mxfp4_dequantize(hc, hs)
+                q = lambda v: Q.mxfp4_quantize(v)  # noqa: E731
+            else:
+                g = np.float32(g_h[t][s])
+                hc, hs, _ = Q.nvfp4_quantize(h.astype(np.float32), g=g)
+                h_dq = Q.nvfp4_dequantize(hc, hs, g)
+                q = lambda v: Q.nvfp4_quantize(v, g=g)[:2]  # noqa: E731
+            lo_c, lo_s = q((h - tol).astype(np.float32))
+            hi_c, hi_s = q((h + tol).astype(np.float32))
+            mid = F.unpack_nibbles(hc) & 7
+            unstable = ~((lo_s == hs) & (hi_s == hs) &
+                         ((F.unpack_nibbles(lo_c) & 7) == mid).reshape(1, -1, blk).all(2) &
+                         ((F.unpack_nibbles(hi_c) & 7) == mid).reshape(1, -1, blk).all(2))
+            # largest magnitude a band value can be coded with: 6 x the next scale up
+            amax_hi = (np.abs(h) + tol).reshape(1, -1, blk).max(2)
+            step = np.where(unstable, 12.0 * 2.0 * amax_hi, 0.0)
+            dh = np.repeat(step, blk, axis=1)
+            wt = float(slot_weights[t, s])
+            y = wt * (h_dq @ w2.T)
+            ref[t] += y[0]
+            sum_abs[t] += np.abs(y[0])
+            slack[t] += (abs(wt) * (dh @ np.abs(w2).T) + G.FP32_REL_TOL * abs(wt) * (np.abs(h_dq) @ np.abs(w2).T))[0]
+    return ref, slack, sum_abs
