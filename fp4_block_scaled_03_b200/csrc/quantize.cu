@@ -126,11 +126,12 @@ __global__ void __launch_bounds__(kThreads) nvfp4_quantize_kernel(
   }
 }
 
-// ---- NVFP4 quantize fused with the routing gather ---------------------------
-// One CTA per token row at a time: the row's k destination rows (its routed
-// rows, padded per expert to 128) are looked up once into shared memory, then
-// each thread quantizes 16-element blocks and writes codes and the tiled scale
-// to every destination row.  Same arithmetic as nvfp4_quantize_kernel.
+// ---- NVFP4 / MXFP4 quantize fused with the routing gather --------------------
+// One warp per token row, no block barriers: lanes 0..k-1 look up the row's
+// destination rows (its routed rows, padded per expert to 128) and every lane
+// gets them by shuffle; then each lane quantizes whole K steps and writes the
+// codes and one 4-byte scale word to every destination.  Same arithmetic as
+// nvfp4_quantize_kernel / mxfp4_quantize_kernel.
 __device__ __forceinline__ int expert_of_row(const int32_t *__restrict__ offsets, int E, int32_t r) {
   int lo = 0, hi = E;  // offsets[lo] <= r < offsets[hi]
   while (hi - lo > 1) {
@@ -140,30 +141,37 @@ __device__ __forceinline__ int expert_of_row(const int32_t *__restrict__ offsets
   return lo;
 }
 
+__device__ __forceinline__ void gather_destinations(const int32_t *__restrict__ offsets,
+                                                    const int32_t *__restrict__ tile_offsets,
+                                                    const int32_t *__restrict__ inv, int E, int topk, int64_t t,
+                                                    int lane, int64_t *dd) {
+  int64_t d = -1;
+  if (lane < topk) {
+    const int32_t r = inv[t * topk + lane];
+    if (r >= 0) {
+      const int e = expert_of_row(offsets, E, r);
+      d = (int64_t)tile_offsets[e] * 128 + (r - offsets[e]);
+    }
+  }
+#pragma unroll
+  for (int s = 0; s < 16; ++s) dd[s] = __shfl_sync(0xffffffffu, d, s);
+}
+
+// NVFP4: a lane's K step is 64 elements (four 16-element blocks).
 __global__ void __launch_bounds__(128) nvfp4_quantize_gather_kernel(
     const uint16_t *__restrict__ x, int64_t T, int64_t H, int32_t topk, int32_t E,
     const int32_t *__restrict__ offsets, const int32_t *__restrict__ tile_offsets, const int32_t *__restrict__ inv,
     uint8_t *__restrict__ a_codes, uint8_t *__restrict__ a_sf, const unsigned int *__restrict__ amax_bits,
     float *__restrict__ g_out) {
-  // each thread quantizes one 64-element K step (four 16-element blocks), so it
-  // writes 32 contiguous code bytes and one 4-byte scale word per destination
-  __shared__ int64_t dst[16];
   const float g = __fdiv_rn(__uint_as_float(*amax_bits), 2688.0f);
   if (blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
+  const int lane = threadIdx.x & 31;
   const int64_t n_ksteps = H / 64;
-  for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
-    __syncthreads();  // previous row's destinations no longer in use
-    if (threadIdx.x < topk) {
-      const int32_t r = inv[t * topk + threadIdx.x];
-      int64_t d = -1;
-      if (r >= 0) {
-        const int e = expert_of_row(offsets, E, r);
-        d = (int64_t)tile_offsets[e] * 128 + (r - offsets[e]);
-      }
-      dst[threadIdx.x] = d;
-    }
-    __syncthreads();
-    for (int64_t kw = threadIdx.x; kw < n_ksteps; kw += blockDim.x) {
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
+  for (int64_t t = blockIdx.x * (int64_t)(blockDim.x / 32) + (threadIdx.x >> 5); t < T; t += warps) {
+    int64_t dd[16];
+    gather_destinations(offsets, tile_offsets, inv, E, topk, t, lane, dd);
+    for (int64_t kw = lane; kw < n_ksteps; kw += 32) {
       const uint4 *src = reinterpret_cast<const uint4 *>(x + t * H + kw * 64);
       uint4 v[8];
 #pragma unroll
@@ -183,7 +191,7 @@ __global__ void __launch_bounds__(128) nvfp4_quantize_gather_kernel(
         sfw |= sf << (8 * blk);
       }
       for (int s = 0; s < topk; ++s) {
-        const int64_t d = dst[s];
+        const int64_t d = dd[s];
         if (d < 0) continue;
         uint4 *out = reinterpret_cast<uint4 *>(a_codes + d * (H / 2) + kw * 32);
         out[0] = make_uint4(code[0], code[1], code[2], code[3]);
@@ -194,28 +202,19 @@ __global__ void __launch_bounds__(128) nvfp4_quantize_gather_kernel(
   }
 }
 
-// MXFP4 variant: each thread quantizes one 128-element K step (four 32-element
-// blocks) and writes 64 code bytes and one 4-byte UE8M0 scale word per
-// destination row (tiled layout with 32-element blocks).
+// MXFP4: a lane's K step is 128 elements (four 32-element blocks, one UE8M0
+// scale word, 64 code bytes; tiled layout with 32-element blocks).
 __global__ void __launch_bounds__(128) mxfp4_quantize_gather_kernel(
     const uint16_t *__restrict__ x, int64_t T, int64_t H, int32_t topk, int32_t E,
     const int32_t *__restrict__ offsets, const int32_t *__restrict__ tile_offsets, const int32_t *__restrict__ inv,
     uint8_t *__restrict__ a_codes, uint8_t *__restrict__ a_sf) {
-  __shared__ int64_t dst[16];
+  const int lane = threadIdx.x & 31;
   const int64_t n_ksteps = H / 128;
-  for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
-    __syncthreads();
-    if (threadIdx.x < topk) {
-      const int32_t r = inv[t * topk + threadIdx.x];
-      int64_t d = -1;
-      if (r >= 0) {
-        const int e = expert_of_row(offsets, E, r);
-        d = (int64_t)tile_offsets[e] * 128 + (r - offsets[e]);
-      }
-      dst[threadIdx.x] = d;
-    }
-    __syncthreads();
-    for (int64_t kw = threadIdx.x; kw < n_ksteps; kw += blockDim.x) {
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
+  for (int64_t t = blockIdx.x * (int64_t)(blockDim.x / 32) + (threadIdx.x >> 5); t < T; t += warps) {
+    int64_t dd[16];
+    gather_destinations(offsets, tile_offsets, inv, E, topk, t, lane, dd);
+    for (int64_t kw = lane; kw < n_ksteps; kw += 32) {
       const uint4 *src = reinterpret_cast<const uint4 *>(x + t * H + kw * 128);
       uint32_t code[16], sfw = 0;
 #pragma unroll
@@ -234,7 +233,7 @@ __global__ void __launch_bounds__(128) mxfp4_quantize_gather_kernel(
         sfw |= mxfp4_block32(f, code + 4 * blk) << (8 * blk);
       }
       for (int s = 0; s < topk; ++s) {
-        const int64_t d = dst[s];
+        const int64_t d = dd[s];
         if (d < 0) continue;
         uint4 *out = reinterpret_cast<uint4 *>(a_codes + d * (H / 2) + kw * 64);
 #pragma unroll
@@ -461,7 +460,8 @@ fp4_status fp4_moe_quantize_gather(const void *x_bf16, int64_t T, int32_t topk, 
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int64_t grid = T < (int64_t)sms * 16 ? T : (int64_t)sms * 16;
+    const int64_t need = (T + 3) / 4;  // four rows (warps) per CTA
+    const int64_t grid = need < (int64_t)sms * 16 ? need : (int64_t)sms * 16;
     mxfp4_quantize_gather_kernel<<<(unsigned)grid, 128, 0, s>>>(x, T, H, topk, E, offsets, tile_offsets, inv,
                                                                  a_codes, a_sf);
     FP4_HOST_CHECK(cudaGetLastError());
@@ -474,7 +474,8 @@ fp4_status fp4_moe_quantize_gather(const void *x_bf16, int64_t T, int32_t topk, 
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t grid = T < (int64_t)sms * 16 ? T : (int64_t)sms * 16;
+  const int64_t need = (T + 3) / 4;  // four rows (warps) per CTA
+  const int64_t grid = need < (int64_t)sms * 16 ? need : (int64_t)sms * 16;
   nvfp4_quantize_gather_kernel<<<(unsigned)grid, 128, 0, s>>>(x, T, H, topk, E, offsets, tile_offsets, inv, a_codes,
                                                                a_sf, amax, global_scale);
   FP4_HOST_CHECK(cudaGetLastError());

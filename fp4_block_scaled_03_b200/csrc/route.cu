@@ -159,30 +159,41 @@ __global__ void gather_kernel(const uint8_t *__restrict__ x_codes, const uint8_t
   }
 }
 
-// out[t, c..c+7] = bf16(sum_s y[inv[t,s], c..c+7]), fp32 adds in slot order.
+// out[t, c..c+15] = bf16(sum_s y[inv[t,s], c..c+15]), fp32 adds in slot order.
+// Sixteen columns per thread: four independent 16-byte loads per slot.
 __global__ void combine_kernel(const float *__restrict__ y, const int32_t *__restrict__ inv, int64_t T,
                                int32_t topk, int64_t H, __nv_bfloat16 *__restrict__ out) {
-  const int64_t per_row = H / 8;
+  const int64_t per_row = H / 16;
   const int64_t total = T * per_row;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t t = i / per_row, c = (i - t * per_row) * 8;
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    const int64_t t = i / per_row, c = (i - t * per_row) * 16;
+    float acc[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) acc[j] = 0.0f;
     for (int s = 0; s < topk; ++s) {
       const int32_t r = inv[t * topk + s];
       if (r < 0) continue;
       const float4 *p = reinterpret_cast<const float4 *>(y + (int64_t)r * H + c);
-      const float4 a = __ldcs(p), b = __ldcs(p + 1);
-      acc[0] = __fadd_rn(acc[0], a.x); acc[1] = __fadd_rn(acc[1], a.y);
-      acc[2] = __fadd_rn(acc[2], a.z); acc[3] = __fadd_rn(acc[3], a.w);
-      acc[4] = __fadd_rn(acc[4], b.x); acc[5] = __fadd_rn(acc[5], b.y);
-      acc[6] = __fadd_rn(acc[6], b.z); acc[7] = __fadd_rn(acc[7], b.w);
+      float4 q[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) q[j] = __ldcs(p + j);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        acc[4 * j] = __fadd_rn(acc[4 * j], q[j].x);
+        acc[4 * j + 1] = __fadd_rn(acc[4 * j + 1], q[j].y);
+        acc[4 * j + 2] = __fadd_rn(acc[4 * j + 2], q[j].z);
+        acc[4 * j + 3] = __fadd_rn(acc[4 * j + 3], q[j].w);
+      }
     }
-    uint4 o;
-    __nv_bfloat162 h0 = __floats2bfloat162_rn(acc[0], acc[1]), h1 = __floats2bfloat162_rn(acc[2], acc[3]);
-    __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[4], acc[5]), h3 = __floats2bfloat162_rn(acc[6], acc[7]);
-    o.x = *reinterpret_cast<uint32_t *>(&h0); o.y = *reinterpret_cast<uint32_t *>(&h1);
-    o.z = *reinterpret_cast<uint32_t *>(&h2); o.w = *reinterpret_cast<uint32_t *>(&h3);
-    *reinterpret_cast<uint4 *>(out + t * H + c) = o;
+    uint32_t o[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[2 * j], acc[2 * j + 1]);
+      o[j] = *reinterpret_cast<uint32_t *>(&h2);
+    }
+    uint4 *dst = reinterpret_cast<uint4 *>(out + t * H + c);
+    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
   }
 }
 
@@ -342,11 +353,11 @@ fp4_status fp4_moe_gather(const uint8_t *x_codes, const uint8_t *x_sf, int64_t T
 fp4_status fp4_moe_combine(const float *y, const int32_t *inv, int64_t T, int32_t topk, int64_t H, void *out_bf16,
                            fp4_stream_t stream) {
   if (!y || !inv || !out_bf16) return FP4_ERR_INVALID_ARG;
-  if (T < 0 || topk < 1 || topk > 16 || H <= 0 || H % 8) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (T < 0 || topk < 1 || topk > 16 || H <= 0 || H % 16) return FP4_ERR_UNSUPPORTED_SHAPE;
   if (!al16(y) || !al16(out_bf16)) return FP4_ERR_ALIGNMENT;
   if (T == 0) return FP4_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const int64_t total = T * (H / 8);
+  const int64_t total = T * (H / 16);
   int64_t grid = (total + 255) / 256;
   const int64_t cap = (int64_t)sm_count() * 8;
   if (grid > cap) grid = cap;

@@ -292,7 +292,7 @@ fp4_status fp4_moe_w2(const uint8_t *h_codes, const uint8_t *h_sf, const fp4_moe
                       fp4_stream_t stream);
 
 /* out[t] = bf16_RNE(sum_{s=0..k-1} y[inv[t*k+s]]) (fp32 adds in slot order;
- * inv < 0 contributes nothing). */
+ * inv < 0 contributes nothing).  H % 16 == 0. */
 fp4_status fp4_moe_combine(const float *y, const int32_t *inv, int64_t T, int32_t topk, int64_t H,
                            void *out_bf16, fp4_stream_t stream);
 
