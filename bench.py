@@ -133,7 +133,9 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
-def setup_dist(args):
+def setup_dist(args, backend=None):
+    """One process per GPU (torchrun sets RANK / WORLD_SIZE / LOCAL_RANK).
+    NCCL on GPUs; gloo when there is no GPU (host-side tests)."""
     import torch
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -144,20 +146,25 @@ def setup_dist(args):
 
         import torch.distributed as dist
 
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        if backend is None:
+            backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return world, rank, local
 
 
 def max_over_ranks(x, world):
+    """The largest of every rank's x (the job's time is its slowest rank's)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -685,7 +692,16 @@ def main():
     world, rank, local = setup_dist(args)
     peaks = load_peaks()
     if args.impl == "reference":
+        # the CPU oracle runs on rank 0 alone; the other ranks leave at once
+        # (no collective follows, so nobody waits on the oracle's minutes)
         line = run_reference(args, world, rank)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+        return
     elif args.workload in WORKLOADS:
         line = run_moe(args, world, rank, peaks)
     elif args.workload in ("dense4096", "dense4096mx"):
