@@ -52,7 +52,7 @@ def gemm_source_hash():
     import hashlib
 
     h = hashlib.sha256()
-    for f in ("gemm.cu", "common.cuh"):
+    for f in ("gemm.cu", "moe_pair.cu", "common.cuh", "host.cuh"):
         h.update(open(os.path.join(ROOT, "fp4_block_scaled_03_b200", "csrc", f), "rb").read())
     return h.hexdigest()
 
@@ -178,7 +178,7 @@ def barrier(world):
 
 # ---------------------------------------------------------------------------
 class MoeBench:
-    def __init__(self, name, seed):
+    def __init__(self, name, seed, pair_tiles=False):
         import torch
 
         import fp4_block_scaled_03_b200 as fp4
@@ -187,6 +187,10 @@ class MoeBench:
         self.fp4 = fp4
         self.mx = name.endswith("mx")
         self.flags = fp4.FP4_MOE_MX if self.mx else 0
+        # NVFP4 grouped GEMMs on 1-CTA row tiles unless CTA pairs are asked for (MXFP4 always row tiles)
+        self.pair = pair_tiles and not self.mx
+        if self.pair:
+            self.flags |= fp4.FP4_MOE_PAIR_TILES
         T, H, I, E, k, zipf, sigma, desc = WORKLOADS[name]
         self.T, self.H, self.I, self.E, self.k, self.desc, self.name = T, H, I, E, k, desc, name
         dev = "cuda"
@@ -297,6 +301,23 @@ class MoeBench:
 
     LAUNCHES_PER_STEP = 8  # 3 routing, amax, quantize+gather, w13, w2, combine
 
+    def mma_rows(self):
+        """Routed rows the grouped GEMMs run through the tensor cores: each
+        expert's rows rounded up to 16 per 256-row chunk (CTA pairs) or to
+        128 (row tiles)."""
+        c = self.counts.cpu().tolist()
+        if self.pair:
+            return int(sum(256 * (n // 256) + ((n % 256 + 15) // 16) * 16 for n in c))
+        return int(sum((n + 127) // 128 * 128 for n in c))
+
+    def tiling_desc(self):
+        if self.pair:
+            return "CTA pairs (tcgen05 cta_group::2): 256 weight rows x up to 256 routed rows (rounded to 16)"
+        return "1-CTA tiles: 128 routed rows (padded per expert to 128) x 256 weight rows"
+
+    def kernel_name(self, stage):
+        return ("moe_pair_kernel<%s>" if self.pair else "fp4_gemm_kernel<256, %s>") % stage
+
     def flops(self):
         return 2.0 * 3.0 * self.H * self.I * self.R
 
@@ -310,7 +331,7 @@ def run_moe(args, world, rank, peaks):
     import torch
 
     fp4 = __import__("fp4_block_scaled_03_b200")
-    b = MoeBench(args.workload, seed=rank * 7919)
+    b = MoeBench(args.workload, seed=rank * 7919, pair_tiles=args.pair_tiles)
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
     for _ in range(args.warmup):
@@ -431,18 +452,18 @@ def run_moe(args, world, rank, peaks):
                    "topk": b.k, "routed_rows": b.R, "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (weights %.2f GB)" % (b.E * 3 * b.H * b.I * 0.5625 / 1e9),
                    "experts_touched": int((b.counts > 0).sum().item()),
-                   "tile_rows": int(b.toffs[b.E].item()) * 128,
-                   "padding_frac": round(1.0 - b.R / max(1, int(b.toffs[b.E].item()) * 128), 4)},
-        "roofline": {"bound": "tensor", "kernel": "fp4_gemm_kernel<256, w13> (grouped w13 + SwiGLU + requant)",
+                   "tiling": b.tiling_desc(), "mma_rows": b.mma_rows(),
+                   "padding_frac": round(1.0 - b.R / max(1, b.mma_rows()), 4)},
+        "roofline": {"bound": "tensor", "kernel": b.kernel_name("w13") + " (grouped w13 + SwiGLU + requant)",
                      "achieved": round(w13_tf, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
-                     "frac": round(w13_tf / fp4_peak, 4), "traffic": measured_traffic(args.workload, "w13"),
+                     "frac": round(w13_tf / fp4_peak, 4), "traffic": measured_traffic(args.workload, b.kernel_name("w13")),
                      "algorithmic_bytes": w13_bytes,
                      "frac_of_max_flops_bytes": round(max(w13_flops / (fp4_peak * 1e12), w13_bytes / (peaks["hbm"] * 1e9))
                                                       / (stage[2] * 1e-3), 4),
                      "peak_note": "4 x measured sustained bf16 cuBLAS (nominal fp4/bf16 ratio), of " + peaks["src"]},
         "stages_ms": {n: round(v, 4) for n, v in zip(["route", "quantize_gather", "w13", "w2", "combine"], stage)},
         "w2": {"achieved_tflops": round(w2_tf, 1), "frac": round(w2_tf / fp4_peak, 4),
-               "traffic": measured_traffic(args.workload, "w2")},
+               "traffic": measured_traffic(args.workload, b.kernel_name("w2"))},
         "quantize": {"achieved_gbs": round(q_gbs, 1), "peak_gbs": peaks["hbm"], "frac": round(q_gbs / peaks["hbm"], 4),
                      "algorithmic_bytes": q_bytes,
                      "note": "dynamic g, fused with the gather: x read once (2 B/elem) + every routed row written"
@@ -686,6 +707,8 @@ def main():
     ap.add_argument("--workload", default="pro", choices=list(WORKLOADS) + ["dense4096", "dense4096mx", "quant"])
     ap.add_argument("--impl", default="fp4", choices=["fp4", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--pair-tiles", action="store_true",
+                    help="MoE workloads: CTA-pair tiles (cta_group::2, tokens on N) for the NVFP4 grouped GEMMs")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

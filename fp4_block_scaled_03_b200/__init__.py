@@ -25,6 +25,7 @@ FP4_SCALE_LAYOUT_TILED = 0x2
 FP4_DEBUG_DUMP_H = 0x4
 FP4_GEMM_MX = 0x8
 FP4_MOE_MX = 0x10
+FP4_MOE_PAIR_TILES = 0x20
 
 STATUS = {
     0: "FP4_OK",
@@ -293,7 +294,8 @@ def moe_rows_cap(T, topk, E):
     return ((T * topk + 127 * E + 127) // 128) * 128
 
 
-def moe_layer(x, expert_ids, topk_weights, w, H, I, E, workspace=None, out=None, h_dump=None, mx=False):
+def moe_layer(x, expert_ids, topk_weights, w, H, I, E, workspace=None, out=None, h_dump=None, mx=False,
+              pair_tiles=False):
     T, topk = expert_ids.shape
     dev = x.device
     if workspace is None:
@@ -301,5 +303,6 @@ def moe_layer(x, expert_ids, topk_weights, w, H, I, E, workspace=None, out=None,
     if out is None:
         out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
     flags = (FP4_DEBUG_DUMP_H if h_dump is not None else 0) | (FP4_MOE_MX if mx else 0)
+    flags |= FP4_MOE_PAIR_TILES if pair_tiles else 0
     fp4_moe_grouped_gemm(x, expert_ids, topk_weights, T, topk, w, H, I, E, out, workspace, flags, h_dump)
     return out

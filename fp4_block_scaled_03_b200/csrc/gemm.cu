@@ -37,9 +37,7 @@
 // padded rows) x (BN columns of that expert's weights).  Every mbarrier wait
 // is bounded; on expiry the CTA records FP4_ERR_DEVICE_TIMEOUT, lets its
 // in-flight copies and MMAs finish, frees tensor memory and returns.
-#include <mutex>
-
-#include "common.cuh"
+#include "host.cuh"
 
 namespace fp4 {
 namespace {
@@ -148,10 +146,6 @@ __device__ __forceinline__ TileInfo tile_info(const Params &p, int t) {
     ti.out_row0 = mt * BM;
   }
   return ti;
-}
-
-__device__ __forceinline__ float silu_f32(float z) {
-  return __fdiv_rn(z, __fadd_rn(1.0f, expf(-z)));
 }
 
 template <int BN, int EPI, bool MX>
@@ -486,58 +480,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static std::once_flag once;
-  static EncodeTiledFn fn = nullptr;
-  std::call_once(once, [] {
-    void *ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  });
-  return fn;
-}
-
-// Packed-code matrix [rows][row_bytes] as a 2-D uint8 tensor map with a
-// 128-byte x box_rows box and 128-byte swizzle (zero fill out of bounds).
-bool make_code_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t row_bytes, uint32_t box_rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {row_bytes, rows};
-  cuuint64_t strides[1] = {row_bytes};
-  cuuint32_t box[2] = {128, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// fp32 matrix [rows][cols] as a 2-D tensor map with an 8-column x 32-row box
-// and 32-byte swizzle (the w2 epilogue's store staging layout).
-bool make_f32_store_map(CUtensorMap *m, void *base, uint64_t rows, uint64_t cols) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols * 4};
-  cuuint32_t box[2] = {8, 32};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-         CUDA_SUCCESS;
-}
-
-int sm_count() {
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  return sms;
-}
-
 template <int BN, int EPI, bool MX = false>
 fp4_status launch(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &ty, const Params &p, int grid,
                   cudaStream_t s) {
@@ -548,8 +490,6 @@ fp4_status launch(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMa
   FP4_HOST_CHECK(cudaGetLastError());
   return FP4_OK;
 }
-
-bool al16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 constexpr int kBN = 256;
 
@@ -612,6 +552,11 @@ fp4_status fp4_moe_w13(const uint8_t *a_codes, const uint8_t *a_sf, const float 
   if (!al16(a_codes) || !al16(a_sf) || !al16(w->w13_codes) || !al16(w->w13_sf) || !al16(h_codes) || !al16(h_sf) ||
       (h_dump && !al16(h_dump)))
     return FP4_ERR_ALIGNMENT;
+  if (!mx && (flags & FP4_MOE_PAIR_TILES)) {
+    if (((rows_cap + 255) / 256 + E) * (2 * I / 256) > (1LL << 31) - 1) return FP4_ERR_UNSUPPORTED_SHAPE;
+    return moe_pair_w13(a_codes, a_sf, a_g, w, H, I, E, counts, tile_offsets, rows_cap, h_codes, h_sf,
+                        (flags & FP4_DEBUG_DUMP_H) ? h_dump : nullptr, reinterpret_cast<cudaStream_t>(stream));
+  }
   const DeviceCtx *ctx = device_ctx();
   if (!ctx) return FP4_ERR_CUDA;
   CUtensorMap ta, tb;
@@ -647,6 +592,11 @@ fp4_status fp4_moe_w2(const uint8_t *h_codes, const uint8_t *h_sf, const fp4_moe
   if (H < 256 || H % 256 || I < 256 || I % 256 || E < 1 || E > 4096 || rows_cap < 1) return FP4_ERR_UNSUPPORTED_SHAPE;
   if ((int64_t)E * H > (1LL << 31) - 1 || rows_cap > (1LL << 31) - 1) return FP4_ERR_UNSUPPORTED_SHAPE;
   if (!al16(h_codes) || !al16(h_sf) || !al16(w->w2_codes) || !al16(w->w2_sf) || !al16(y)) return FP4_ERR_ALIGNMENT;
+  if (!mx && (flags & FP4_MOE_PAIR_TILES)) {
+    if (((rows_cap + 255) / 256 + E) * (H / 256) > (1LL << 31) - 1) return FP4_ERR_UNSUPPORTED_SHAPE;
+    return moe_pair_w2(h_codes, h_sf, w, H, I, E, counts, offsets, tile_offsets, perm, topk_weights, rows_cap, y,
+                       reinterpret_cast<cudaStream_t>(stream));
+  }
   const DeviceCtx *ctx = device_ctx();
   if (!ctx) return FP4_ERR_CUDA;
   CUtensorMap ta, tb;

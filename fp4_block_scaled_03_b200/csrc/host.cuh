@@ -1,0 +1,92 @@
+// Host-side helpers shared by the GEMM translation units: tensor-map
+// encoding through the driver entry point, the SM count, alignment checks,
+// and the CTA-pair grouped MoE launches (moe_pair.cu) that fp4_moe_w13 /
+// fp4_moe_w2 dispatch to.
+#pragma once
+
+#include <mutex>
+
+#include "common.cuh"
+
+namespace fp4 {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline EncodeTiledFn encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// Packed-code matrix [rows][row_bytes] as a 2-D uint8 tensor map with a
+// 128-byte x box_rows box and 128-byte swizzle (zero fill out of bounds).
+inline bool make_code_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t row_bytes, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {row_bytes, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// A tiled scale buffer of `bytes` (a multiple of 512) viewed as rows of 256
+// bytes, with a 256-byte x 8-row box: one box is the 2 KB of scales of a
+// 128-row slab over four K steps of 64 (one 256-element K stage).
+inline bool make_sf_map(CUtensorMap *m, const void *base, uint64_t bytes) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || bytes % 512) return false;
+  cuuint64_t dims[2] = {256, bytes / 256};
+  cuuint64_t strides[1] = {256};
+  cuuint32_t box[2] = {256, 8};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// fp32 matrix [rows][cols] as a 2-D tensor map with an 8-column x 32-row box
+// and 32-byte swizzle (the w2 epilogue's store staging layout).
+inline bool make_f32_store_map(CUtensorMap *m, void *base, uint64_t rows, uint64_t cols) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 4};
+  cuuint32_t box[2] = {8, 32};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+inline int sm_count() {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms;
+}
+
+inline bool al16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Grouped NVFP4 w13 / w2 on CTA pairs (moe_pair.cu).  Arguments are those of
+// fp4_moe_w13 / fp4_moe_w2, already validated by the caller.
+fp4_status moe_pair_w13(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_g, const fp4_moe_weights *w,
+                        int64_t H, int64_t I, int32_t E, const int32_t *counts, const int32_t *tile_offsets,
+                        int64_t rows_cap, uint8_t *h_codes, uint8_t *h_sf, float *h_dump, cudaStream_t stream);
+fp4_status moe_pair_w2(const uint8_t *h_codes, const uint8_t *h_sf, const fp4_moe_weights *w, int64_t H, int64_t I,
+                       int32_t E, const int32_t *counts, const int32_t *offsets, const int32_t *tile_offsets,
+                       const int32_t *perm, const float *topk_weights, int64_t rows_cap, float *y,
+                       cudaStream_t stream);
+
+}  // namespace fp4

@@ -75,14 +75,15 @@ fp4_status fp4_moe_grouped_gemm(const void *tokens_bf16, const int32_t *expert_i
                      I32(L.inv), ws + L.scratch, fp4_moe_route_scratch_bytes(T * topk, E), stream);
   if (st != FP4_OK) return st;
   const uint32_t fmt = flags & FP4_MOE_MX;
+  const uint32_t tiling = flags & FP4_MOE_PAIR_TILES;
   st = fp4_moe_quantize_gather(tokens_bf16, T, topk, H, E, I32(L.offsets), I32(L.tile_offsets), I32(L.inv),
                                ws + L.a_codes, ws + L.a_sf, L.rows_cap, g_x, ws + L.header, 256, fmt, stream);
   if (st != FP4_OK) return st;
   st = fp4_moe_w13(ws + L.a_codes, ws + L.a_sf, g_x, w, H, I, E, I32(L.counts), I32(L.tile_offsets), L.rows_cap,
-                   ws + L.h_codes, ws + L.h_sf, (flags & FP4_DEBUG_DUMP_H) | fmt, h_dump, stream);
+                   ws + L.h_codes, ws + L.h_sf, (flags & FP4_DEBUG_DUMP_H) | fmt | tiling, h_dump, stream);
   if (st != FP4_OK) return st;
   st = fp4_moe_w2(ws + L.h_codes, ws + L.h_sf, w, H, I, E, I32(L.counts), I32(L.offsets), I32(L.tile_offsets),
-                  I32(L.perm), topk_weights, L.rows_cap, reinterpret_cast<float *>(ws + L.y), fmt, stream);
+                  I32(L.perm), topk_weights, L.rows_cap, reinterpret_cast<float *>(ws + L.y), fmt | tiling, stream);
   if (st != FP4_OK) return st;
   return fp4_moe_combine(reinterpret_cast<const float *>(ws + L.y), I32(L.inv), T, topk, H, out_bf16, stream);
 }

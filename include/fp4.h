@@ -77,6 +77,7 @@ typedef enum { FP4_OUT_F32 = 0, FP4_OUT_BF16 = 1 } fp4_out_dtype;
 #define FP4_DEBUG_DUMP_H 0x4u        /* MoE w13 stage: also write fp32 h */
 #define FP4_GEMM_MX 0x8u             /* fp4_gemm: MXFP4 operands (UE8M0 per 32) */
 #define FP4_MOE_MX 0x10u             /* MoE layer / stages: MXFP4 weights, activations and h */
+#define FP4_MOE_PAIR_TILES 0x20u     /* MoE NVFP4 w13 / w2: CTA-pair tiles instead of 1-CTA row tiles */
 
 /* Human-readable name of a status code (static string). */
 const char *fp4_status_string(fp4_status s);
@@ -274,8 +275,14 @@ fp4_status fp4_moe_quantize_gather(const void *x_bf16, int64_t T, int32_t topk, 
 /* Grouped w13 GEMM + SwiGLU + NVFP4 re-quantize of h with h_g[e]:
  * a = gathered rows (codes [rows_cap][H/2], tiled sf), a_g = fp32[1] tensor
  * scale of x; writes h_codes [rows_cap][I/2] and tiled h_sf for [rows_cap, I]
- * (only rows that hold a routed row are written). h_dump (FP4_DEBUG_DUMP_H):
- * fp32 [rows_cap][I].  FP4_MOE_MX: MXFP4 operands and h (a_g unused). */
+ * (rows that hold a routed row; padding rows up to the next multiple of 16
+ * get zero codes and scales). h_dump (FP4_DEBUG_DUMP_H): fp32 [rows_cap][I].
+ * FP4_MOE_MX: MXFP4 operands and h (a_g unused).
+ * Tiling (results agree up to fp32 accumulation order): by default 1-CTA
+ * tiles of 128 routed rows (padded per expert to 128) x 256 weight rows;
+ * with FP4_MOE_PAIR_TILES (NVFP4 only; FP4_MOE_MX ignores it) CTA pairs
+ * (tcgen05 cta_group::2) with M = 256 weight rows x N = up to 256 routed
+ * rows rounded up to 16. */
 fp4_status fp4_moe_w13(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_g,
                        const fp4_moe_weights *w, int64_t H, int64_t I, int32_t E,
                        const int32_t *counts, const int32_t *tile_offsets, int64_t rows_cap,
@@ -284,7 +291,8 @@ fp4_status fp4_moe_w13(const uint8_t *a_codes, const uint8_t *a_sf, const float 
 
 /* Grouped w2 GEMM: y[offsets[e]+i] = w[perm[row]] * h_g[e]*w2_g[e] * (h . W2_e^T)
  * y: fp32 [T*topk][H] in routed order; topk_weights may be NULL.
- * FP4_MOE_MX: MXFP4 operands, y = w * (h . W2_e^T). */
+ * FP4_MOE_MX: MXFP4 operands, y = w * (h . W2_e^T).  Tiling and
+ * FP4_MOE_PAIR_TILES as for fp4_moe_w13. */
 fp4_status fp4_moe_w2(const uint8_t *h_codes, const uint8_t *h_sf, const fp4_moe_weights *w,
                       int64_t H, int64_t I, int32_t E, const int32_t *counts,
                       const int32_t *offsets, const int32_t *tile_offsets, const int32_t *perm,

@@ -62,6 +62,18 @@ def router(T, E, k, seed, zipf_s=0.0, device="cpu"):
     return ids, w, counts
 
 
+def router_fixed_counts(counts, seed, device="cpu"):
+    """Top-1 routing with prescribed per-expert row counts, tokens in a seeded
+    random order, weights uniform in [0.25, 1).  Returns the same triple as
+    router()."""
+    g = _gen(seed, device)
+    ids = torch.cat([torch.full((int(n),), e, dtype=torch.int32, device=device) for e, n in enumerate(counts)])
+    ids = ids[torch.randperm(ids.numel(), generator=g, device=device)].reshape(-1, 1)
+    w = (0.25 + 0.75 * torch.rand((ids.shape[0], 1), generator=g, device=device)).to(torch.float32)
+    c = torch.tensor([int(n) for n in counts], dtype=torch.int64, device=device)
+    return ids, w, c
+
+
 def random_codes(shape_bytes, seed, device="cpu"):
     """Uniform random packed FP4 bytes (every code equally likely)."""
     g = _gen(seed, device)

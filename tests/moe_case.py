@@ -19,14 +19,18 @@ class Case:
 
 
 def build(T, H, I, E, k, seed=0, zipf=0.0, h_g=1e-3, w_sigma=0.02, w_frac=0.005, w_factor=30.0, fmt="nv",
-          oracle_experts=None):
+          oracle_experts=None, counts=None):
     import fp4_block_scaled_03_b200 as fp4
 
     c = Case()
     c.T, c.H, c.I, c.E, c.k = T, H, I, E, k
     dev = "cuda"
     c.x = synth.activations_bf16((T, H), seed=seed, device=dev)
-    c.ids, c.w, c.counts = synth.router(T, E, k, seed=seed + 1, zipf_s=zipf, device=dev)
+    if counts is not None:  # prescribed top-1 routing
+        assert k == 1 and len(counts) == E and sum(counts) == T
+        c.ids, c.w, c.counts = synth.router_fixed_counts(counts, seed=seed + 1, device=dev)
+    else:
+        c.ids, c.w, c.counts = synth.router(T, E, k, seed=seed + 1, zipf_s=zipf, device=dev)
     w13 = synth.weights_bf16((E * 2 * I, H), w_sigma, w_frac, w_factor, seed=seed + 2, device=dev)
     w2 = synth.weights_bf16((E * H, I), w_sigma, w_frac, w_factor, seed=seed + 3, device=dev)
     c.w13_codes = torch.empty((E * 2 * I, H // 2), dtype=torch.uint8, device=dev)

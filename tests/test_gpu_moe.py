@@ -144,7 +144,14 @@ def _band_quantize_check(h_ref, tol, g, codes_gpu, sf_gpu):
     return int((~exact).sum()), int((~stable).sum()), ok
 
 
-def _run_stages(c, dump=True):
+TILINGS = ["pair", "rows"]
+
+
+def _tiling_flag(tiling):
+    return _lib().FP4_MOE_PAIR_TILES if tiling == "pair" else 0
+
+
+def _run_stages(c, dump=True, tiling="pair"):
     fp4 = _lib()
     T, H, I, E, k = c.T, c.H, c.I, c.E, c.k
     xc, xs, xg = fp4.quantize_nv(c.x)
@@ -157,14 +164,29 @@ def _run_stages(c, dump=True):
     h_s = torch.zeros(fp4.fp4_sf_tiled_bytes(cap, I), dtype=torch.uint8, device="cuda")
     h_d = torch.zeros((cap, I), dtype=torch.float32, device="cuda") if dump else None
     fp4.fp4_moe_w13(a_c, a_s, xg, c.weights, H, I, E, r["counts"], r["tile_offsets"], cap, h_c, h_s,
-                    fp4.FP4_DEBUG_DUMP_H if dump else 0, h_d)
+                    (fp4.FP4_DEBUG_DUMP_H if dump else 0) | _tiling_flag(tiling), h_d)
     return dict(r=r, cap=cap, h_c=h_c, h_s=h_s, h_d=h_d, xg=xg)
 
 
+@pytest.mark.parametrize("tiling", TILINGS)
 @pytest.mark.parametrize("T,H,I,E,k,zipf", [(200, 512, 256, 8, 2, 0.0), (700, 1024, 512, 6, 6, 1.1)])
-def test_w13_swiglu_requant(T, H, I, E, k, zipf):
+def test_w13_swiglu_requant(T, H, I, E, k, zipf, tiling):
     c = moe_case.build(T, H, I, E, k, seed=T, zipf=zipf)
-    out = _run_stages(c)
+    _check_w13(c, tiling)
+
+
+def test_w13_w2_chunk_edges():
+    """Experts holding 1, 16, 256, 257 and 530 routed rows: token chunks of
+    256 with tails of 1, 16, 1 and 18 rows (MMA N of 16 .. 256, one and two
+    128-row scale slabs), against the oracle, on the CTA-pair tiling."""
+    c = moe_case.build(1060, 512, 256, 5, 1, seed=21, counts=[1, 16, 256, 257, 530])
+    _check_w13(c, "pair")
+    _check_w2(c, "pair")
+
+
+def _check_w13(c, tiling):
+    T, H, I, E, k = c.T, c.H, c.I, c.E, c.k
+    out = _run_stages(c, tiling=tiling)
     assert _lib().fp4_get_device_status() == 0
     counts, offsets, perm, inv = MO.route(c.ids_np, E)
     toff = _tile_offsets_ref(counts)
@@ -193,10 +215,15 @@ def test_w13_swiglu_requant(T, H, I, E, k, zipf):
     assert total_diff <= 0.01 * (T * k * I // 16) + 8, total_diff
 
 
-def test_w2_weighted_rows():
-    fp4 = _lib()
+@pytest.mark.parametrize("tiling", TILINGS)
+def test_w2_weighted_rows(tiling):
     T, H, I, E, k = 260, 768, 512, 5, 3
-    c = moe_case.build(T, H, I, E, k, seed=77)
+    _check_w2(moe_case.build(T, H, I, E, k, seed=77), tiling)
+
+
+def _check_w2(c, tiling):
+    fp4 = _lib()
+    T, H, I, E, k = c.T, c.H, c.I, c.E, c.k
     r = _route_gpu(c.ids, T, k, E)
     cap = fp4.moe_rows_cap(T, k, E)
     h_c = synth.random_codes((cap, I // 2), seed=5, device="cuda")
@@ -204,7 +231,8 @@ def test_w2_weighted_rows():
     hg = torch.tensor(np.linspace(0.5, 2.0, E), dtype=torch.float32, device="cuda")
     wset = fp4.MoeWeightSet(c.w13_codes, c.w13_sf, c.w13_g, c.w2_codes, c.w2_sf, c.w2_g, hg)
     y = torch.full((T * k, H), np.nan, dtype=torch.float32, device="cuda")
-    fp4.fp4_moe_w2(h_c, h_s, wset, H, I, E, r["counts"], r["offsets"], r["tile_offsets"], r["perm"], c.w, cap, y)
+    fp4.fp4_moe_w2(h_c, h_s, wset, H, I, E, r["counts"], r["offsets"], r["tile_offsets"], r["perm"], c.w, cap, y,
+                   _tiling_flag(tiling))
     assert fp4.fp4_get_device_status() == 0
     yg = y.cpu().numpy().astype(np.float64)
     counts, offsets, perm, inv = MO.route(c.ids_np, E)
@@ -244,8 +272,9 @@ def test_combine_fixed_order():
     assert ok.all(), int((~ok).sum())
 
 
+@pytest.mark.parametrize("tiling", TILINGS)
 @pytest.mark.parametrize("T,H,I,E,k,zipf", [(256, 512, 256, 8, 2, 0.0), (1000, 1024, 512, 16, 6, 1.1)])
-def test_layer_end_to_end(T, H, I, E, k, zipf):
+def test_layer_end_to_end(T, H, I, E, k, zipf, tiling):
     """fp4_moe_grouped_gemm against the oracle layer.  Where every h block of
     a token's rows quantizes the same anywhere in the w13 error band, the
     output must be within 1 bf16 ulp (plus the w2 GEMM bound and the
@@ -253,7 +282,7 @@ def test_layer_end_to_end(T, H, I, E, k, zipf):
     rows it feeds, the most that one different decision there can move y."""
     fp4 = _lib()
     c = moe_case.build(T, H, I, E, k, seed=T + 3, zipf=zipf)
-    out = fp4.moe_layer(c.x, c.ids, c.w, c.weights, H, I, E)
+    out = fp4.moe_layer(c.x, c.ids, c.w, c.weights, H, I, E, pair_tiles=(tiling == "pair"))
     assert fp4.fp4_get_device_status() == 0
     counts, offsets, perm, inv = MO.route(c.ids_np, E)
     (xq, x_dq) = moe_case.oracle_x(c)
