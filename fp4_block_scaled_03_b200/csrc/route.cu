@@ -29,15 +29,19 @@ __global__ void route_count_kernel(const int32_t *__restrict__ ids, int64_t R, i
   for (int e = lane; e < E; e += 32) cnt[e] = 0;
   __syncwarp();
   const int64_t base = (int64_t)blockIdx.x * kChunk;
+  int idv[kChunk / 32];  // all of this lane's ids in flight at once
+#pragma unroll
   for (int step = 0; step < kChunk / 32; ++step) {
     const int64_t f = base + step * 32 + lane;
-    int id = -1;
-    if (f < R) {
-      id = ids[f];
-      if (id < 0 || id >= E) {
-        record_status(status, FP4_ERR_BAD_EXPERT);
-        id = -1;
-      }
+    idv[step] = (f < R) ? ids[f] : -1;
+  }
+#pragma unroll
+  for (int step = 0; step < kChunk / 32; ++step) {
+    const int64_t f = base + step * 32 + lane;
+    int id = idv[step];
+    if (f < R && (id < 0 || id >= E)) {
+      record_status(status, FP4_ERR_BAD_EXPERT);
+      id = -1;
     }
     const uint32_t grp = __match_any_sync(0xffffffffu, id);
     if (id >= 0 && (grp & lanemask_lt()) == 0) cnt[id] += __popc(grp);  // group leader
@@ -58,9 +62,20 @@ __global__ void route_scan_kernel(int32_t *__restrict__ chunk_counts, int nchunk
   int32_t local_rows = 0, local_tiles = 0;
   for (int e = e0; e < e0 + per && e < E; ++e) {
     int32_t run = 0;
-    for (int c = 0; c < nchunks; ++c) {
+    int c = 0;
+    for (; c + 8 <= nchunks; c += 8) {  // eight loads in flight, then their prefix
+      int32_t v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = chunk_counts[(int64_t)(c + i) * E + e];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        chunk_counts[(int64_t)(c + i) * E + e] = run;  // exclusive within the expert
+        run += v[i];
+      }
+    }
+    for (; c < nchunks; ++c) {
       int32_t v = chunk_counts[(int64_t)c * E + e];
-      chunk_counts[(int64_t)c * E + e] = run;  // exclusive within the expert
+      chunk_counts[(int64_t)c * E + e] = run;
       run += v;
     }
     counts[e] = run;
@@ -84,6 +99,7 @@ __global__ void route_scan_kernel(int32_t *__restrict__ chunk_counts, int nchunk
   for (int e = e0; e < e0 + per && e < E; ++e) {
     offsets[e] = row_base;
     tile_offsets[e] = tile_base;
+#pragma unroll 8
     for (int c = 0; c < nchunks; ++c) chunk_counts[(int64_t)c * E + e] += row_base;
     row_base += counts[e];
     tile_base += (counts[e] + 127) / 128;
@@ -104,13 +120,17 @@ __global__ void route_scatter_kernel(const int32_t *__restrict__ ids, int64_t R,
   for (int e = lane; e < E; e += 32) run[e] = chunk_base[(int64_t)blockIdx.x * E + e];
   __syncwarp();
   const int64_t base = (int64_t)blockIdx.x * kChunk;
+  int idv[kChunk / 32];
+#pragma unroll
   for (int step = 0; step < kChunk / 32; ++step) {
     const int64_t f = base + step * 32 + lane;
-    int id = -1;
-    if (f < R) {
-      id = ids[f];
-      if (id < 0 || id >= E) id = -1;
-    }
+    idv[step] = (f < R) ? ids[f] : -1;
+  }
+#pragma unroll
+  for (int step = 0; step < kChunk / 32; ++step) {
+    const int64_t f = base + step * 32 + lane;
+    int id = idv[step];
+    if (id < 0 || id >= E) id = -1;
     const uint32_t grp = __match_any_sync(0xffffffffu, id);
     int32_t pos = -1;
     if (id >= 0) pos = run[id] + __popc(grp & lanemask_lt());
