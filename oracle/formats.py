@@ -96,6 +96,18 @@ def e4m3_encode_pos(v):
     return _nearest_code(v.astype(np.float64), E4M3_VALUES)
 
 
+def e4m3_encode(v):
+    """fp32 array -> signed E4M3 byte codes (the MXFP8 element type): RNE ties
+    to even, saturating at +-448, sign bit copied from the input (so -0.0 and
+    negatives that round to zero give 0x80)."""
+    v = np.asarray(v, dtype=np.float32)
+    if np.any(np.isnan(v)):
+        raise ValueError("e4m3_encode: NaN input")
+    mag = _nearest_code(np.abs(v.astype(np.float64)), E4M3_VALUES)
+    sign = np.signbit(v).astype(np.uint8) << 7
+    return (mag | sign).astype(np.uint8)
+
+
 def ue8m0_decode(codes):
     """UE8M0 byte codes -> float64 2^(c-127); 255 -> NaN."""
     codes = np.asarray(codes, dtype=np.int64)

@@ -15,7 +15,7 @@ one bf16 ulp of RNE_bf16(C_ref).
 """
 import numpy as np
 
-from .quant import mxfp4_dequantize, nvfp4_dequantize
+from .quant import mxfp4_dequantize, mxfp8_dequantize, nvfp4_dequantize
 
 FP32_REL_TOL = 1e-4
 
@@ -33,6 +33,16 @@ def mxfp4_gemm_ref(a_packed, a_scales, b_packed, b_scales):
     a = mxfp4_dequantize(a_packed, a_scales)
     b = mxfp4_dequantize(b_packed, b_scales)
     return a @ b.T, np.abs(a) @ np.abs(b).T
+
+
+def w4a8_gemm_ref(a_codes, a_scales, b, b_scales, b_is_fp8=False):
+    """FP8 x FP4 ("DeepSeek-V4 FP4 QAT" §4.3: FP4 weights against FP8
+    activations): A MXFP8 (E4M3 codes [M,K], UE8M0 per 32), B MXFP4 (packed
+    [N,K/2], UE8M0 per 32) or, with b_is_fp8, MXFP8 like A.  fp64
+    C = A_dq @ B_dq^T and the bound matrix |A_dq| @ |B_dq|^T."""
+    a = mxfp8_dequantize(a_codes, a_scales)
+    bd = mxfp8_dequantize(b, b_scales) if b_is_fp8 else mxfp4_dequantize(b, b_scales)
+    return a @ bd.T, np.abs(a) @ np.abs(bd).T
 
 
 def bf16_ulp(x_bf16_as_f64):

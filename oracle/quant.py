@@ -34,6 +34,17 @@ of its 16-element halves (exactly representable while e - e_max + 8 >= -9);
 blocks whose codes are all (signed) zeros get scale 0; codes are unchanged.
 A tensor whose exponent span would need an E4M3 power below 2^-9 cannot be
 remapped losslessly and is reported as a range error.
+
+MXFP8 (the W4A8 activation format: "DeepSeek-V4 FP4 QAT" §4.3 recommends FP8
+activations against FP4 weights, and §4.2 keeps the power-of-two block scale
+of the MX format).  Reading: the MXFP4 rule above with the E4M3 element
+type, whose largest power of two is 2^8: per 32-block X = floor(log2 amax) - 8
+clamped to [-127, 127], scale byte X + 127 (0 for an all-zero block),
+element = E4M3_RNE_satfinite(x * 2^-X) with the input's sign bit.
+
+FP4 -> FP8 widening (same page §4.2, steps 3-4): every E2M1 value is exactly
+an E4M3 value, so each 4-bit code maps to the E4M3 byte of the same value and
+the UE8M0 block scales carry over unchanged; nothing is rounded.
 """
 import numpy as np
 
@@ -41,6 +52,7 @@ from .formats import (
     e2m1_decode,
     e2m1_encode,
     e4m3_decode,
+    e4m3_encode,
     e4m3_encode_pos,
     floor_log2_f32,
     pack_nibbles,
@@ -120,6 +132,40 @@ def mxfp4_dequantize(packed, scale_codes):
     rows, cols = codes.shape
     vals = e2m1_decode(codes).reshape(rows, cols // MX_BLOCK, MX_BLOCK)
     return (vals * ue8m0_decode(scale_codes)[:, :, None]).reshape(rows, cols)
+
+
+MXFP8_EMAX = 8  # floor(log2(448))
+
+
+def mxfp8_quantize(x):
+    """x: fp32 [rows, cols], cols % 32 == 0.
+    Returns (E4M3 codes uint8 [rows, cols], UE8M0 scale bytes [rows, cols/32])."""
+    x = np.asarray(x, dtype=np.float32)
+    rows, cols = x.shape
+    assert cols % MX_BLOCK == 0
+    xb = x.reshape(rows, cols // MX_BLOCK, MX_BLOCK)
+    amax = np.max(np.abs(xb), axis=2)
+    zero = amax == 0
+    X = np.zeros(amax.shape, dtype=np.int64)
+    X[~zero] = floor_log2_f32(amax[~zero]) - MXFP8_EMAX
+    X = np.clip(X, -127, 127)
+    scale_codes = np.where(zero, 0, X + 127).astype(np.uint8)
+    v = np.ldexp(xb.astype(np.float64), -X[:, :, None]).astype(np.float32)  # one RN to fp32
+    return e4m3_encode(v).reshape(rows, cols), scale_codes
+
+
+def mxfp8_dequantize(codes, scale_codes):
+    codes = np.asarray(codes, dtype=np.uint8)
+    rows, cols = codes.shape
+    vals = e4m3_decode(codes).reshape(rows, cols // MX_BLOCK, MX_BLOCK)
+    return (vals * ue8m0_decode(scale_codes)[:, :, None]).reshape(rows, cols)
+
+
+def e2m1_to_e4m3(packed):
+    """Packed E2M1 codes [rows, cols/2] -> E4M3 bytes [rows, cols] of the same
+    values (sign included): the E4M3 encoding of each decoded E2M1 value."""
+    codes = unpack_nibbles(packed)
+    return e4m3_encode(e2m1_decode(codes).astype(np.float32))
 
 
 class RemapRangeError(ValueError):

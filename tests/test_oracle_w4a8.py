@@ -1,0 +1,132 @@
+"""Pins of the W4A8 oracle (MXFP8 activations x MXFP4 weights) against
+things other than itself: ml_dtypes' float8_e4m3fn rounding, a brute-force
+nearest search over every E4M3 byte, a hand-written code table, exact integer
+products, and the lossless FP4 -> FP8 widening."""
+import os
+
+import ml_dtypes
+import numpy as np
+import pytest
+
+from oracle import formats as F
+from oracle import gemm as G
+from oracle import quant as Q
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+def _all_e4m3_finite():
+    """Every finite E4M3 byte and its value, decoded here by bit fields
+    (sign, 4-bit exponent with bias 7, 3-bit mantissa, subnormals m * 2^-9)."""
+    out = []
+    for b in range(256):
+        e, m, s = (b >> 3) & 15, b & 7, -1.0 if b & 0x80 else 1.0
+        if e == 15 and m == 7:
+            continue  # NaN
+        v = m * 2.0 ** -9 if e == 0 else (1 + m / 8) * 2.0 ** (e - 7)
+        out.append((b, s * v))
+    return out
+
+
+def test_e4m3_encode_matches_ml_dtypes_in_range():
+    rng = np.random.default_rng(3)
+    v = np.concatenate([rng.uniform(-463, 463, 20000), rng.standard_normal(20000) * 0.01,
+                        rng.standard_normal(5000) * 2.0 ** -8]).astype(np.float32)
+    ref = v.astype(ml_dtypes.float8_e4m3fn).view(np.uint8)
+    assert np.array_equal(F.e4m3_encode(v), ref)
+
+
+def test_e4m3_encode_brute_force_ties_and_saturation():
+    table = _all_e4m3_finite()
+    vals = np.array([v for _, v in table])
+    bytes_ = np.array([b for b, _ in table], dtype=np.uint8)
+    # every midpoint between neighbouring positive values, plus saturation and signed zeros
+    pos = np.sort(np.unique(np.abs(vals)))
+    mids = (pos[:-1] + pos[1:]) / 2
+    v = np.concatenate([mids, -mids, [460.0, 1000.0, -1000.0, -0.0, 0.0, -1e-30]]).astype(np.float32)
+    got = F.e4m3_encode(v)
+    for x, g in zip(v.astype(np.float64), got):
+        ax = min(abs(x), 448.0)  # satfinite
+        d = np.abs(np.abs(vals) - ax)
+        cand = [b for b, dv, val in zip(bytes_, d, vals) if dv == d.min() and (val > 0 or (val == 0 and not b & 0x80))]
+        # ties: the even mantissa; sign: the input's sign bit
+        best = min(cand, key=lambda b: (b & 1, b))
+        want = best | (0x80 if np.signbit(x) else 0)
+        assert g == want, (x, hex(g), hex(want))
+
+
+def test_e2m1_to_e4m3_golden_table():
+    rows = [l.split() for l in open(os.path.join(HERE, "golden", "e2m1_to_e4m3.txt")) if not l.startswith("#")]
+    codes = np.array([int(a) for a, _ in rows], dtype=np.uint8)
+    want = np.array([int(b, 16) for _, b in rows], dtype=np.uint8)
+    got = Q.e2m1_to_e4m3(F.pack_nibbles(codes.reshape(1, 16)))[0]
+    assert np.array_equal(got, want)
+    # the widening is value-exact, including the sign of zero
+    assert np.array_equal(F.e4m3_decode(want), F.e2m1_decode(codes))
+
+
+def test_mxfp8_scale_exponent_is_mxfp4_minus_six():
+    """Same block rule, element maxima 2^8 (E4M3) and 2^2 (E2M1)."""
+    x = (np.random.default_rng(5).standard_normal((16, 256)) * np.exp2(np.arange(16) - 8)[:, None]).astype(np.float32)
+    _, s4 = Q.mxfp4_quantize(x)
+    _, s8 = Q.mxfp8_quantize(x)
+    assert np.array_equal(s8.astype(int), s4.astype(int) - 6)
+
+
+@pytest.mark.parametrize("p", [-20, -3, 0, 5, 40])
+def test_mxfp8_power_of_two_amax(p):
+    rng = np.random.default_rng(p + 100)
+    x = (rng.uniform(-1, 1, (2, 32)) * 2.0 ** p).astype(np.float32)
+    x[:, 7] = 2.0 ** p  # amax exactly 2^p -> X = p - 8, that element codes to 2^8 = 0x78
+    c, s = Q.mxfp8_quantize(x)
+    assert np.all(s == p - 8 + 127)
+    assert np.all(c[:, 7] == 0x78)
+
+
+def test_mxfp8_brute_force_block():
+    table = _all_e4m3_finite()
+    rng = np.random.default_rng(11)
+    x = (rng.standard_normal((6, 64)) * 3).astype(np.float32)
+    x[0, :32] = 0.0
+    x[1, 5] = -0.0
+    c, s = Q.mxfp8_quantize(x)
+    assert s[0, 0] == 0 and np.all(c[0, :32] == 0)
+    for r in range(x.shape[0]):
+        for b in range(2):
+            blk = x[r, 32 * b:32 * b + 32].astype(np.float64)
+            amax = np.abs(blk).max()
+            if amax == 0:
+                continue
+            X = int(np.floor(np.log2(amax))) - 8
+            assert s[r, b] == X + 127
+            for j, v in enumerate(blk):
+                t = min(abs(v) * 2.0 ** -X, 448.0)
+                cands = sorted(table, key=lambda bv: (abs(abs(bv[1]) - t), bv[0] & 1))
+                best = [bv for bv in cands if bv[1] >= 0 and not bv[0] & 0x80][0][0]
+                assert c[r, 32 * b + j] == best | (0x80 if np.signbit(v) else 0)
+
+
+def test_w4a8_gemm_ref_integer_case_exact():
+    """Scales 2^0; A holds integer E4M3 values, B E2M1 values (halves); C is
+    exactly the integer product / 2."""
+    rng = np.random.default_rng(7)
+    M, N, K = 5, 7, 96
+    a_int = rng.integers(-16, 17, (M, K))
+    a_codes = F.e4m3_encode(a_int.astype(np.float32))
+    b_codes = rng.integers(0, 16, (N, K)).astype(np.uint8)
+    b_twice = np.rint(2 * F.e2m1_decode(b_codes)).astype(np.int64)
+    one = np.full((M, K // 32), 127, np.uint8)
+    C, bound = G.w4a8_gemm_ref(a_codes, one, F.pack_nibbles(b_codes), np.full((N, K // 32), 127, np.uint8))
+    assert np.array_equal(C * 2, (a_int @ b_twice.T).astype(np.float64))
+    assert np.all(bound >= np.abs(C))
+
+
+def test_w4a8_fp4_and_widened_fp8_weights_agree_exactly():
+    rng = np.random.default_rng(9)
+    a = rng.standard_normal((8, 128)).astype(np.float32)
+    w = (rng.standard_normal((12, 128)) * 0.02).astype(np.float32)
+    ac, as_ = Q.mxfp8_quantize(a)
+    wc, ws = Q.mxfp4_quantize(w)
+    C4, _ = G.w4a8_gemm_ref(ac, as_, wc, ws)
+    C8, _ = G.w4a8_gemm_ref(ac, as_, Q.e2m1_to_e4m3(wc), ws, b_is_fp8=True)
+    assert np.array_equal(C4, C8)
