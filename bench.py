@@ -1,12 +1,14 @@
 """Benchmark of the NVFP4 W4A4 routed-expert hot path on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload pro|flash|decode|dense4096|quant]
+    python bench.py [--gpus N] [--steps K] [--warmup W]
+                    [--workload pro|flash|flashmx|decode|pro64|dense4096|dense4096mx|dense4096w4a8|quant]
                     [--impl fp4|reference]
 
 A step is one pass of the whole hot path over one synthetic batch: dynamic
 NVFP4 quantize of the activations -> routing permute -> gather -> grouped
 w13 GEMM with SwiGLU + NVFP4 re-quantize -> grouped w2 GEMM -> combine
-(workloads pro / flash / decode), one quantize + dense GEMM (dense4096), or
+(workloads pro / flash / flashmx / decode / pro64), one quantize + dense GEMM
+(dense4096: NVFP4, dense4096mx: MXFP4, dense4096w4a8: MXFP8 x MXFP4), or
 one activation quantize (quant).  Inputs are resident in HBM before timing;
 weights (9.5 GB for pro) and activations exceed the 126 MB L2, so no flush
 is needed between steps.  Per-kernel times come from CUDA events recorded
@@ -535,7 +537,10 @@ def cpu_baseline_moe(b, n_tokens=1):
 
 
 # ---------------------------------------------------------------------------
-def run_dense(args, world, rank, peaks, mx=False):
+def run_dense(args, world, rank, peaks, mx=False, w4a8=False):
+    """Dense 4096^3 GEMM with the activation quantized on the device every
+    call: NVFP4 x NVFP4, MXFP4 x MXFP4 (mx), or W4A8 -- MXFP8 activations x
+    MXFP4 weights on kind::mxf8f6f4 (w4a8)."""
     import torch
 
     import fp4_block_scaled_03_b200 as fp4
@@ -544,13 +549,16 @@ def run_dense(args, world, rank, peaks, mx=False):
     M = N = K = 4096
     a_bf = synth.activations_bf16((M, K), seed=rank, device="cuda")
     b_bf = synth.weights_bf16((N, K), 0.02, 0.005, 30.0, seed=rank + 1, device="cuda")
+    mx = mx or w4a8
     if mx:
         b_c, b_sf = fp4.quantize_mx(b_bf, tiled=True)
         b_g = None
     else:
         b_c, b_sf, b_g = fp4.quantize_nv(b_bf, tiled=True)
-    a_c = torch.empty((M, K // 2), dtype=torch.uint8, device="cuda")
+    a_c = torch.empty((M, K if w4a8 else K // 2), dtype=torch.uint8, device="cuda")
     a_sf = torch.empty(fp4.fp4_sf_tiled_bytes(M, K) // (2 if mx else 1), dtype=torch.uint8, device="cuda")
+    a_fmt = fp4.FP4_MXFP8 if w4a8 else fp4.FP4_MX if mx else fp4.FP4_NV
+    g_flags = fp4.FP4_GEMM_A_MXFP8 if w4a8 else fp4.FP4_GEMM_MX if mx else 0
     a_g = torch.empty(1, dtype=torch.float32, device="cuda")
     ws = torch.empty(256, dtype=torch.uint8, device="cuda")
     c = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
@@ -559,12 +567,10 @@ def run_dense(args, world, rank, peaks, mx=False):
     def step(ev=None):
         if ev:
             ev[0].record()
-        fp4.fp4_quantize(fp4.FP4_MX if mx else fp4.FP4_NV, a_bf, M, K, K, a_c, a_sf, a_g, fp4.FP4_SCALE_LAYOUT_TILED,
-                         ws, 256)
+        fp4.fp4_quantize(a_fmt, a_bf, M, K, K, a_c, a_sf, a_g, fp4.FP4_SCALE_LAYOUT_TILED, ws, 256)
         if ev:
             ev[1].record()
-        fp4.fp4_gemm(a_c, a_sf, None if mx else a_g, b_c, b_sf, b_g, c, fp4.FP4_OUT_BF16, M, N, K,
-                     fp4.FP4_GEMM_MX if mx else 0)
+        fp4.fp4_gemm(a_c, a_sf, None if mx else a_g, b_c, b_sf, b_g, c, fp4.FP4_OUT_BF16, M, N, K, g_flags)
         if ev:
             ev[2].record()
 
@@ -591,18 +597,26 @@ def run_dense(args, world, rank, peaks, mx=False):
     ms = max_over_ranks(tot / args.steps, world)
     gms = g / args.steps
     flops = 2.0 * M * N * K
-    fp4_peak = 4.0 * peaks["bf16"]
+    # tensor peak of the instruction's own type: 4x (FP4) or 2x (FP8 x FP4 runs at the FP8 rate) the
+    # measured bf16 figure, the recipe's nominal dense ratios
+    ratio = 2.0 if w4a8 else 4.0
+    fp4_peak = ratio * peaks["bf16"]
+    name = ("Dense W4A8 (MXFP8 activations x MXFP4 weights, UE8M0/32)" if w4a8 else
+            "Dense MXFP4 (UE8M0/32) W4A4" if mx else "Dense NVFP4 W4A4")
+    kind = "mxf8f6f4" if w4a8 else "mxf4" if mx else "nvf4"
+    dtype = ("mxfp8 x mxfp4 (e4m3 x e2m1, ue8m0/32 scales, fp32 accumulate)" if w4a8 else
+             "mxfp4 (e2m1 x e2m1, ue8m0/32 scales, fp32 accumulate)" if mx else
+             "nvfp4 (e2m1 x e2m1, e4m3/16 scales, fp32 accumulate)")
     return {
         "metric": METRIC, "value": round(world * flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e2m1, e4m3/16 scales, fp32 accumulate)",
+        "scaling": "weak", "vs_baseline": None, "dtype": dtype,
         "data": "synthetic (seeded)",
-        "config": {"workload": ("Dense MXFP4 (UE8M0/32)" if mx else "Dense NVFP4") +
-                   " W4A4 GEMM 4096x4096x4096, activations quantized on device each call, bf16 out",
+        "config": {"workload": name + " GEMM 4096x4096x4096, activations quantized on device each call, bf16 out",
                    "l2": "flushed (256 MB write) before each timed step"},
-        "roofline": {"bound": "tensor", "kernel": "fp4_gemm_kernel<256, bf16, " + ("mxf4" if mx else "nvf4") + ">", "achieved": round(flops / (gms * 1e-3) / 1e12, 1),
+        "roofline": {"bound": "tensor", "kernel": "fp4_gemm_kernel<256, bf16, " + kind + ">", "achieved": round(flops / (gms * 1e-3) / 1e12, 1),
                      "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(flops / (gms * 1e-3) / 1e12 / fp4_peak, 4),
-                     "traffic": None, "peak_note": "4 x measured burst bf16 cuBLAS, of " + peaks["src"]},
+                     "traffic": None, "peak_note": "%dx measured burst bf16 cuBLAS, of %s" % (ratio, peaks["src"])},
         "stages_ms": {"quantize": round(q / args.steps, 4), "gemm": round(gms, 4)},
         "gpu_launches": 3 * args.steps, "clocks": clocks,
     }
@@ -704,7 +718,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="pro", choices=list(WORKLOADS) + ["dense4096", "dense4096mx", "quant"])
+    ap.add_argument("--workload", default="pro", choices=list(WORKLOADS) + ["dense4096", "dense4096mx", "dense4096w4a8", "quant"])
     ap.add_argument("--impl", default="fp4", choices=["fp4", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--pair-tiles", action="store_true",
@@ -727,8 +741,9 @@ def main():
         return
     elif args.workload in WORKLOADS:
         line = run_moe(args, world, rank, peaks)
-    elif args.workload in ("dense4096", "dense4096mx"):
-        line = run_dense(args, world, rank, peaks, mx=args.workload.endswith("mx"))
+    elif args.workload in ("dense4096", "dense4096mx", "dense4096w4a8"):
+        line = run_dense(args, world, rank, peaks, mx=args.workload.endswith("mx"),
+                         w4a8=args.workload.endswith("w4a8"))
     else:
         line = run_quant(args, world, rank, peaks)
     if rank == 0 and line is not None:

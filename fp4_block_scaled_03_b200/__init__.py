@@ -18,12 +18,14 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libfp4.so")
 
-FP4_NV, FP4_MX = 0, 1
+FP4_NV, FP4_MX, FP4_MXFP8 = 0, 1, 2
 FP4_OUT_F32, FP4_OUT_BF16 = 0, 1
 FP4_STATIC_GLOBAL_SCALE = 0x1
 FP4_SCALE_LAYOUT_TILED = 0x2
 FP4_DEBUG_DUMP_H = 0x4
 FP4_GEMM_MX = 0x8
+FP4_GEMM_A_MXFP8 = 0x40
+FP4_GEMM_B_MXFP8 = 0x80
 FP4_MOE_MX = 0x10
 FP4_MOE_PAIR_TILES = 0x20
 
@@ -76,6 +78,7 @@ _SIGS = {
     "fp4_quantize_workspace_size": (_SZ, []),
     "fp4_quantize": (ctypes.c_int, [ctypes.c_int, _P, _I64, _I64, _I64, _P, _P, _P, _U32, _P, _SZ, _P]),
     "fp4_mx_to_nv": (ctypes.c_int, [_P, _P, _I64, _I64, _I64, _P, _P, _U32, _P]),
+    "fp4_e2m1_to_e4m3": (ctypes.c_int, [_P, _I64, _I64, _P, _P]),
     "fp4_gemm": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, ctypes.c_int, _I64, _I64, _I64, _U32, _P]),
     "fp4_moe_workspace_size": (_SZ, [_I64, _I32, _I64, _I64, _I32]),
     "fp4_moe_grouped_gemm": (
@@ -137,6 +140,10 @@ def fp4_quantize(fmt, x, rows, cols, ld, codes, scales, global_scale, flags, wor
 def fp4_mx_to_nv(codes, mx_scales, rows, cols, num_tensors, nv_scales, nv_global, flags=0):
     _check(lib.fp4_mx_to_nv(_ptr(codes), _ptr(mx_scales), rows, cols, num_tensors, _ptr(nv_scales),
                             _ptr(nv_global), flags, _stream()), "fp4_mx_to_nv")
+
+
+def fp4_e2m1_to_e4m3(codes_e2m1, rows, cols, codes_e4m3):
+    _check(lib.fp4_e2m1_to_e4m3(_ptr(codes_e2m1), rows, cols, _ptr(codes_e4m3), _stream()), "fp4_e2m1_to_e4m3")
 
 
 def fp4_gemm(a_codes, a_sf, a_g, b_codes, b_sf, b_g, c, c_dtype, M, N, K, flags=0):
@@ -258,6 +265,28 @@ def quantize_mx(x, tiled=False):
     return codes, scales
 
 
+def quantize_mxfp8(x, tiled=False):
+    """MXFP8 (W4A8 activations): E4M3 codes [rows, cols] + UE8M0 scales."""
+    rows, cols = x.shape
+    dev = x.device
+    codes = torch.empty((rows, cols), dtype=torch.uint8, device=dev)
+    if tiled:
+        scales = _u8(fp4_sf_tiled_bytes(rows, cols) // 2, dev)
+    else:
+        scales = torch.empty((rows, cols // 32), dtype=torch.uint8, device=dev)
+    fp4_quantize(FP4_MXFP8, x, rows, cols, x.stride(0), codes, scales, None,
+                 FP4_SCALE_LAYOUT_TILED if tiled else 0, None, 0)
+    return codes, scales
+
+
+def e2m1_to_e4m3(codes):
+    """Packed E2M1 [rows, cols/2] -> E4M3 bytes [rows, cols] of the same values."""
+    rows, half = codes.shape
+    out = torch.empty((rows, half * 2), dtype=torch.uint8, device=codes.device)
+    fp4_e2m1_to_e4m3(codes, rows, half * 2, out)
+    return out
+
+
 def mx_to_nv(codes, mx_scales, num_tensors, tiled=False):
     total_rows, half = codes.shape
     rows, cols = total_rows // num_tensors, half * 2
@@ -270,10 +299,13 @@ def mx_to_nv(codes, mx_scales, num_tensors, tiled=False):
     return nv, g
 
 
-def gemm(a_codes, a_sf, a_g, b_codes, b_sf, b_g, M, N, K, out_dtype=torch.float32, mx=False):
+def gemm(a_codes, a_sf, a_g, b_codes, b_sf, b_g, M, N, K, out_dtype=torch.float32, mx=False, w4a8=False,
+         b_fp8=False):
+    """mx: MXFP4 x MXFP4.  w4a8: MXFP8 A x MXFP4 B (or MXFP8 B with b_fp8)."""
     c = torch.empty((M, N), dtype=out_dtype, device=a_codes.device)
+    flags = (FP4_GEMM_MX if mx else 0) | (FP4_GEMM_A_MXFP8 if w4a8 else 0) | (FP4_GEMM_B_MXFP8 if b_fp8 else 0)
     fp4_gemm(a_codes, a_sf, a_g, b_codes, b_sf, b_g, c, FP4_OUT_F32 if out_dtype == torch.float32 else FP4_OUT_BF16,
-             M, N, K, FP4_GEMM_MX if mx else 0)
+             M, N, K, flags)
     return c
 
 

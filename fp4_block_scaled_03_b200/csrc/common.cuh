@@ -314,6 +314,28 @@ __host__ __device__ constexpr uint32_t idesc_mxf4(uint32_t M, uint32_t N) {
   return (1u << 7) | (1u << 10) | ((N >> 3) << 17) | (1u << 23) | ((M >> 4) << 24);
 }
 
+// Instruction descriptor of kind::mxf8f6f4 (W4A8): A and B element formats
+// (0 = E4M3, 5 = E2M1), UE8M0 scales (bit 23), both K-major, fp32
+// accumulation, M x N tile; K is 32 elements per instruction.
+__host__ __device__ constexpr uint32_t idesc_mxf8f6f4(uint32_t M, uint32_t N, uint32_t a_fmt, uint32_t b_fmt) {
+  return (a_fmt << 7) | (b_fmt << 10) | ((N >> 3) << 17) | (1u << 23) | ((M >> 4) << 24);
+}
+
+// FP8 x FP4 (or FP8) with UE8M0 scales per 32: D (+)= A . B^T over K = 32.
+// A sub-byte B operand sits in shared memory one element per byte (the
+// tensor map's 16U4_ALIGN16B unpacking); the scale addresses carry in bits
+// 30-31, and idesc in its scale-ID fields, the byte of the 32-bit TMEM scale
+// column that holds this K step's scale.
+__device__ __forceinline__ void mma_mxf8f6f4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
 // Copy a 32-line x 16-byte scale tile from shared memory into 4 TMEM columns,
 // replicated to all four 32-lane quarters.
 __device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint64_t sdesc) {

@@ -79,7 +79,10 @@ struct Params {
   int m_tiles;       // dense only
   int k_stages;      // ceil(K / 256)
   int kw;            // K / 64 (MMA K steps per row)
-  int kw_sf;         // scale words (4 scales) per row: K / 64 (NVFP4) or K / 128 (MXFP4)
+  int kw_sf;         // scale words (4 scales) per row: K / 64 (NVFP4) or K / 128 (MXFP4, W4A8)
+  int b_fmt;         // W4A8: B element format in the instruction descriptor (5 E2M1, 0 E4M3)
+  uint32_t b_tx;     // W4A8: bytes a B stage load completes on its barrier (the packed global bytes
+                     // when TMA unpacks E2M1 into one byte per element)
   const uint8_t *a_sf;
   const uint8_t *b_sf;
   int64_t b_sf_rows;  // rows covered by b's tiled scale buffer (padded to 128)
@@ -148,13 +151,19 @@ __device__ __forceinline__ TileInfo tile_info(const Params &p, int t) {
   return ti;
 }
 
-template <int BN, int EPI, bool MX>
+// KIND: 0 NVFP4 x NVFP4 (kind::mxf4nvf4, E4M3 scale per 16); 1 MXFP4 x MXFP4
+// (kind::mxf4, UE8M0 per 32); 2 W4A8, MXFP8 A x MXFP4 or MXFP8 B
+// (kind::mxf8f6f4, UE8M0 per 32, 128 K-elements per stage).
+template <int BN, int EPI, int KIND>
 __global__ void __launch_bounds__(kThreads, 1)
     fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmY, const Params p) {
   using C = Cfg<BN, EPI>;
   constexpr bool kGrouped = (EPI == EPI_W13 || EPI == EPI_W2);
-  constexpr int WPS = MX ? 2 : 4;   // scale words per row per 256-element stage
+  constexpr bool MX = KIND != 0;  // power-of-two block scales, no tensor scales
+  // scale words (512-byte tiles) per 128-row slab per stage: one per K step of
+  // 64 (NVFP4), per two K steps (MXFP4), or one for the stage's 4 x 32 (W4A8)
+  constexpr int WPS = KIND == 0 ? 4 : KIND == 1 ? 2 : 1;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *smA = smem;
@@ -218,12 +227,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kt = 0; kt < p.k_stages; ++kt) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, &s_abort, p.status, lim)) { ok = false; break; }
           const int nk = min(4, p.kw - kt * 4);
-          const int nw = MX ? (nk + 1) / 2 : nk;  // scale words this stage
+          const int nw = KIND == 0 ? nk : KIND == 1 ? (nk + 1) / 2 : 1;  // scale words this stage
           const uint32_t sf_bytes = (uint32_t)nw * 512u;
           int halves = 0;
           for (int h = 0; h < C::HALVES; ++h)
             if ((int64_t)(b_slab0 + h) * 128 < p.b_sf_rows) ++halves;
-          const uint32_t bytes = C::A_BYTES + C::B_BYTES + sf_bytes * (1 + halves);
+          const uint32_t bytes = C::A_BYTES + (KIND == 2 ? p.b_tx : (uint32_t)C::B_BYTES) + sf_bytes * (1 + halves);
           mbar_arrive_expect_tx(&full[stage], bytes);
           tma_load_2d(smA + stage * C::A_BYTES, &tmA, &full[stage], kt * BK_BYTES, ti.a_row0);
           tma_load_2d(smB + stage * C::B_BYTES, &tmB, &full[stage], kt * BK_BYTES, ti.b_row0);
@@ -253,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait(&full[stage], phase, &s_abort, p.status, lim)) { ok = false; break; }
           tc_fence_after();
           const int nk = min(4, p.kw - kt * 4);
-          const int nw = MX ? (nk + 1) / 2 : nk;
+          const int nw = KIND == 0 ? nk : KIND == 1 ? (nk + 1) / 2 : 1;
           const uint32_t ta = tmem + C::SF_COL0 + stage * C::SF_SLOT_COLS;
           const uint32_t tb = ta + 16;
           // descriptors of the first 512-byte scale tile; tile i is +i*512 bytes (+i*32 in 16-byte units)
@@ -281,7 +290,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = MX ? idesc_mxf4(BM, BN) : idesc_mxf4nvf4(BM, BN);
+      const uint32_t idesc = KIND == 0 ? idesc_mxf4nvf4(BM, BN)
+                             : KIND == 1 ? idesc_mxf4(BM, BN)
+                                         : idesc_mxf8f6f4(BM, BN, 0u /*E4M3*/, (uint32_t)p.b_fmt);
       int stage = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true, any_mma = false;
@@ -302,7 +313,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             if (j < nk) {
-              if (MX) {  // K step j: scale word j/2, bytes 2*(j%2) and 2*(j%2)+1
+              if (KIND == 2) {  // K step j (32 elements): byte j of the stage's scale word
+                const uint32_t byte = (uint32_t)j;
+                mma_mxf8f6f4(t_acc, ad + (uint64_t)(j * 2), bd + (uint64_t)(j * 2), idesc | (byte << 29) | (byte << 4),
+                             ta | (byte << 30), tb | (byte << 30), (kt > 0 || j > 0) ? 1u : 0u);
+              } else if (MX) {  // K step j: scale word j/2, bytes 2*(j%2) and 2*(j%2)+1
                 const uint32_t byte = 2u * (uint32_t)(j & 1);
                 const uint32_t w = (uint32_t)(j >> 1);
                 mma_mxf4(t_acc, ad + (uint64_t)(j * 2), bd + (uint64_t)(j * 2), idesc | (byte << 29) | (byte << 4),
@@ -363,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (EPI == EPI_W2 && p.topk_w) scale = MX ? p.topk_w[p.perm[ti.out_row0 + row]]
                                                 : __fmul_rn(alpha, p.topk_w[p.perm[ti.out_row0 + row]]);
       const int colh = ti.n0 + half * HC;
-      if constexpr (EPI == EPI_W13 && MX) {
+      if constexpr (EPI == EPI_W13 && KIND == 1) {
         // MXFP4 h: one 32-element block per pair of 32-column chunks (16 gate +
         // 16 up columns each), quantized with its own power-of-two scale
 #pragma unroll
@@ -480,11 +495,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-template <int BN, int EPI, bool MX = false>
+template <int BN, int EPI, int KIND = 0>
 fp4_status launch(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &ty, const Params &p, int grid,
                   cudaStream_t s) {
   using C = Cfg<BN, EPI>;
-  auto kern = fp4_gemm_kernel<BN, EPI, MX>;
+  auto kern = fp4_gemm_kernel<BN, EPI, KIND>;
   FP4_HOST_CHECK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
   kern<<<grid, kThreads, C::SMEM_BYTES, s>>>(ta, tb, ty, p);
   FP4_HOST_CHECK(cudaGetLastError());
@@ -503,24 +518,39 @@ extern "C" {
 fp4_status fp4_gemm(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_g, const uint8_t *b_codes,
                     const uint8_t *b_sf, const float *b_g, void *c, fp4_out_dtype c_dtype, int64_t M, int64_t N,
                     int64_t K, uint32_t flags, fp4_stream_t stream) {
-  const bool mx = flags & FP4_GEMM_MX;
+  const bool w4a8 = flags & FP4_GEMM_A_MXFP8;
+  const bool b_fp8 = flags & FP4_GEMM_B_MXFP8;
+  const bool mx = (flags & FP4_GEMM_MX) || w4a8;
   if (!a_codes || !a_sf || !b_codes || !b_sf || !c || (!mx && (!a_g || !b_g))) return FP4_ERR_INVALID_ARG;
   if (c_dtype != FP4_OUT_F32 && c_dtype != FP4_OUT_BF16) return FP4_ERR_INVALID_ARG;
+  if (b_fp8 && !w4a8) return FP4_ERR_INVALID_ARG;
   if (M < 1 || N < 1 || K < 64 || K % 64 || N % 8 || (mx && K % 128)) return FP4_ERR_UNSUPPORTED_SHAPE;
   if (M > (1LL << 30) || N > (1LL << 30) || K > (1LL << 30)) return FP4_ERR_UNSUPPORTED_SHAPE;
   if (!al16(a_codes) || !al16(b_codes) || !al16(a_sf) || !al16(b_sf) || !al16(c)) return FP4_ERR_ALIGNMENT;
+  if (w4a8 && !b_fp8 && (reinterpret_cast<uintptr_t>(b_codes) & 31u)) return FP4_ERR_ALIGNMENT;
   const DeviceCtx *ctx = device_ctx();
   if (!ctx) return FP4_ERR_CUDA;
   CUtensorMap ta, tb;
-  if (!make_code_map(&ta, a_codes, (uint64_t)M, (uint64_t)K / 2, BM)) return FP4_ERR_CUDA;
-  if (!make_code_map(&tb, b_codes, (uint64_t)N, (uint64_t)K / 2, kBN)) return FP4_ERR_CUDA;
+  if (w4a8) {  // A: one E4M3 byte per element, 128 elements per stage row
+    if (!make_code_map(&ta, a_codes, (uint64_t)M, (uint64_t)K, BM)) return FP4_ERR_CUDA;
+    if (b_fp8) {
+      if (!make_code_map(&tb, b_codes, (uint64_t)N, (uint64_t)K, kBN)) return FP4_ERR_CUDA;
+    } else if (!make_u4_unpack_map(&tb, b_codes, (uint64_t)N, (uint64_t)K, kBN)) {
+      return FP4_ERR_CUDA;
+    }
+  } else {
+    if (!make_code_map(&ta, a_codes, (uint64_t)M, (uint64_t)K / 2, BM)) return FP4_ERR_CUDA;
+    if (!make_code_map(&tb, b_codes, (uint64_t)N, (uint64_t)K / 2, kBN)) return FP4_ERR_CUDA;
+  }
   Params p = {};
   p.M = (int)M; p.N = (int)N; p.K = (int)K;
   p.n_tiles = (int)((N + kBN - 1) / kBN);
   p.m_tiles = (int)((M + BM - 1) / BM);
-  p.k_stages = (int)((K + 255) / 256);
-  p.kw = (int)(K / 64);
+  p.k_stages = w4a8 ? (int)(K / 128) : (int)((K + 255) / 256);
+  p.kw = w4a8 ? (int)(K / 32) : (int)(K / 64);  // MMA K steps per row
   p.kw_sf = mx ? (int)(K / 128) : (int)(K / 64);
+  p.b_fmt = b_fp8 ? 0 : 5;
+  p.b_tx = b_fp8 ? (uint32_t)kBN * 128u : (uint32_t)kBN * 64u;
   p.a_sf = a_sf; p.b_sf = b_sf;
   p.b_sf_rows = ((N + 127) / 128) * 128;
   p.a_g = a_g; p.b_g = b_g; p.c = c;
@@ -530,9 +560,13 @@ fp4_status fp4_gemm(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_
   if (tiles > 2147483647LL) return FP4_ERR_UNSUPPORTED_SHAPE;
   const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (w4a8) {
+    if (c_dtype == FP4_OUT_F32) return launch<kBN, EPI_F32, 2>(ta, tb, tb, p, grid, s);
+    return launch<kBN, EPI_BF16, 2>(ta, tb, tb, p, grid, s);
+  }
   if (mx) {
-    if (c_dtype == FP4_OUT_F32) return launch<kBN, EPI_F32, true>(ta, tb, tb, p, grid, s);
-    return launch<kBN, EPI_BF16, true>(ta, tb, tb, p, grid, s);
+    if (c_dtype == FP4_OUT_F32) return launch<kBN, EPI_F32, 1>(ta, tb, tb, p, grid, s);
+    return launch<kBN, EPI_BF16, 1>(ta, tb, tb, p, grid, s);
   }
   if (c_dtype == FP4_OUT_F32) return launch<kBN, EPI_F32>(ta, tb, tb, p, grid, s);
   return launch<kBN, EPI_BF16>(ta, tb, tb, p, grid, s);
@@ -577,7 +611,7 @@ fp4_status fp4_moe_w13(const uint8_t *a_codes, const uint8_t *a_sf, const float 
   p.h_dump = (flags & FP4_DEBUG_DUMP_H) ? h_dump : nullptr;
   p.status = ctx->status;
   p.wait_limit = ctx->wait_limit_ns;
-  if (mx) return launch<kBN, EPI_W13, true>(ta, tb, tb, p, sm_count(), reinterpret_cast<cudaStream_t>(stream));
+  if (mx) return launch<kBN, EPI_W13, 1>(ta, tb, tb, p, sm_count(), reinterpret_cast<cudaStream_t>(stream));
   return launch<kBN, EPI_W13>(ta, tb, tb, p, sm_count(), reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -617,7 +651,7 @@ fp4_status fp4_moe_w2(const uint8_t *h_codes, const uint8_t *h_sf, const fp4_moe
   p.wait_limit = ctx->wait_limit_ns;
   CUtensorMap ty;
   if (!make_f32_store_map(&ty, y, (uint64_t)rows_cap, (uint64_t)H)) return FP4_ERR_CUDA;
-  if (mx) return launch<kBN, EPI_W2, true>(ta, tb, ty, p, sm_count(), reinterpret_cast<cudaStream_t>(stream));
+  if (mx) return launch<kBN, EPI_W2, 1>(ta, tb, ty, p, sm_count(), reinterpret_cast<cudaStream_t>(stream));
   return launch<kBN, EPI_W2>(ta, tb, ty, p, sm_count(), reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -41,6 +41,23 @@ inline bool make_code_map(CUtensorMap *m, const void *base, uint64_t rows, uint6
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Packed E2M1 matrix [rows][cols] (cols 4-bit elements per row, cols / 2
+// bytes) as a 2-D tensor map that unpacks into shared memory one element per
+// byte (16U4_ALIGN16B: each 8 bytes of 16 codes followed by 8 bytes of gap),
+// a 128-element x box_rows box and 128-byte swizzle.  Needs a 32-byte
+// aligned base, cols % 128 == 0 and a row stride that is a multiple of 32.
+inline bool make_u4_unpack_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || cols % 128 || (reinterpret_cast<uintptr_t>(base) & 31u)) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols / 2};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<void *>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // A tiled scale buffer of `bytes` (a multiple of 512) viewed as rows of 256
 // bytes, with a 256-byte x 8-row box: one box is the 2 KB of scales of a
 // 128-row slab over four K steps of 64 (one 256-element K stage).

@@ -244,6 +244,93 @@ __global__ void __launch_bounds__(128) mxfp4_quantize_gather_kernel(
   }
 }
 
+// Four fp32 -> 32 bits of E4M3 bytes (element 0 in the lowest byte), round to
+// nearest even, saturating at +-448, sign kept.  The cvt writes its first
+// source to the high byte of each 16-bit pair.
+__device__ __forceinline__ uint32_t pack4_e4m3(float a, float b, float c, float d) {
+  uint16_t lo, hi;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(b), "f"(a));
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(d), "f"(c));
+  return (uint32_t)lo | ((uint32_t)hi << 16);
+}
+
+// ---- MXFP8 quantize (W4A8 activations): one thread per 32-element block ----
+// Same block rule as MXFP4 with E4M3 elements: X = clamp(floor(log2 amax) - 8),
+// element = E4M3_RNE_satfinite(x * 2^-X).
+template <bool kTiled>
+__global__ void __launch_bounds__(kThreads) mxfp8_quantize_kernel(const uint16_t *__restrict__ x, int64_t rows,
+                                                                  int64_t cols, int64_t ld,
+                                                                  uint8_t *__restrict__ codes,
+                                                                  uint8_t *__restrict__ scales) {
+  const int64_t nb = cols / 32;
+  const int64_t total = rows * nb;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = i / nb, b = i - r * nb;
+    const uint4 *src = reinterpret_cast<const uint4 *>(x + r * ld + b * 32);
+    uint32_t w[16];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint4 v = __ldcs(src + q);
+      w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
+    }
+    uint32_t amax = 0;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) amax = max(amax, max(w[j] & 0x7FFFu, (w[j] >> 16) & 0x7FFFu));
+    int X = 0;
+    uint32_t scale = 0;
+    if (amax) {
+      const int e = (int)(amax >> 7);
+      const int fl = e ? e - 127 : (31 - __clz((int)(amax & 0x7Fu))) - 133;
+      X = min(max(fl - 8, -127), 127);
+      scale = (uint32_t)(X + 127);
+    }
+    const float p = __uint_as_float((uint32_t)(127 - X) << 23);  // 2^-X, X in [-127, 119] for bf16 input
+    uint32_t out[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t w0 = w[2 * j], w1 = w[2 * j + 1];
+      out[j] = pack4_e4m3(__fmul_rn(bf16_bits_to_f32(w0 & 0xFFFFu), p), __fmul_rn(bf16_bits_to_f32(w0 >> 16), p),
+                          __fmul_rn(bf16_bits_to_f32(w1 & 0xFFFFu), p), __fmul_rn(bf16_bits_to_f32(w1 >> 16), p));
+    }
+    uint4 *dst = reinterpret_cast<uint4 *>(codes + r * cols + b * 32);
+    dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
+    dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+    if (kTiled)  // the MX tile layout (32-element blocks, 4 per row per 128 columns)
+      scales[sf_tiled_offset(r, b, cols / 128)] = (uint8_t)scale;
+    else
+      scales[i] = (uint8_t)scale;
+  }
+}
+
+// ---- FP4 -> FP8 widening: E2M1 code -> the E4M3 byte of the same value ------
+// Magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6 are E4M3 bytes 00 30 38 3C 40 44 48 4C;
+// the sign bit moves from bit 3 to bit 7.  One thread per 32 elements.
+__device__ __forceinline__ uint32_t widen4(uint32_t nib4) {  // four codes in the low 16 bits -> four bytes
+  const uint32_t sel = (nib4 & 0x7u) | ((nib4 >> 4 & 0x7u) << 4) | ((nib4 >> 8 & 0x7u) << 8) |
+                       ((nib4 >> 12 & 0x7u) << 12);
+  const uint32_t mag = __byte_perm(0x3C383000u, 0x4C484440u, sel);
+  const uint32_t sgn = ((nib4 & 0x8u) << 4) | ((nib4 & 0x80u) << 8) | ((nib4 & 0x800u) << 12) |
+                       ((nib4 & 0x8000u) << 16);
+  return mag | sgn;
+}
+
+__global__ void __launch_bounds__(kThreads) e2m1_to_e4m3_kernel(const uint8_t *__restrict__ in, int64_t n32,
+                                                                uint8_t *__restrict__ out) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n32; i += (int64_t)gridDim.x * blockDim.x) {
+    const uint4 v = __ldcs(reinterpret_cast<const uint4 *>(in) + i);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      o[2 * q] = widen4(w[q] & 0xFFFFu);
+      o[2 * q + 1] = widen4(w[q] >> 16);
+    }
+    uint4 *d = reinterpret_cast<uint4 *>(out) + 2 * i;
+    d[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    d[1] = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+}
+
 // ---- MXFP4 quantize: one thread per 32-element block -----------------------
 template <bool kTiled>
 __global__ void __launch_bounds__(kThreads) mxfp4_quantize_kernel(const uint16_t *__restrict__ x, int64_t rows,
@@ -371,7 +458,7 @@ fp4_status fp4_quantize(fp4_format fmt, const void *x_bf16, int64_t rows, int64_
                         uint8_t *scales, float *global_scale, uint32_t flags, void *workspace, size_t ws_bytes,
                         fp4_stream_t stream) {
   if (!x_bf16 || !codes || !scales || rows < 0 || cols <= 0 || ld < cols) return FP4_ERR_INVALID_ARG;
-  if (fmt != FP4_NV && fmt != FP4_MX) return FP4_ERR_INVALID_ARG;
+  if (fmt != FP4_NV && fmt != FP4_MX && fmt != FP4_MXFP8) return FP4_ERR_INVALID_ARG;
   if (!aligned16(x_bf16) || !aligned16(codes) || (ld * 2) % 16) return FP4_ERR_ALIGNMENT;
   const DeviceCtx *ctx = device_ctx();
   if (!ctx) return FP4_ERR_CUDA;
@@ -379,6 +466,15 @@ fp4_status fp4_quantize(fp4_format fmt, const void *x_bf16, int64_t rows, int64_
   if (rows == 0) return FP4_OK;
   const uint16_t *x = static_cast<const uint16_t *>(x_bf16);
   const bool tiled = flags & FP4_SCALE_LAYOUT_TILED;
+  if (fmt == FP4_MXFP8) {
+    if (cols % 32 || (tiled && cols % 128)) return FP4_ERR_UNSUPPORTED_SHAPE;
+    if (tiled)
+      mxfp8_quantize_kernel<true><<<grid_for(rows * (cols / 32)), kThreads, 0, s>>>(x, rows, cols, ld, codes, scales);
+    else
+      mxfp8_quantize_kernel<false><<<grid_for(rows * (cols / 32)), kThreads, 0, s>>>(x, rows, cols, ld, codes, scales);
+    FP4_HOST_CHECK(cudaGetLastError());
+    return FP4_OK;
+  }
   if (fmt == FP4_MX) {
     if (cols % 32 || (tiled && cols % 128)) return FP4_ERR_UNSUPPORTED_SHAPE;
     if (tiled)
@@ -407,6 +503,19 @@ fp4_status fp4_quantize(fp4_format fmt, const void *x_bf16, int64_t rows, int64_
     nvfp4_quantize_kernel<true><<<grid, kThreads, 0, s>>>(x, rows, cols, ld, codes, scales, amax, global_scale, g_in);
   else
     nvfp4_quantize_kernel<false><<<grid, kThreads, 0, s>>>(x, rows, cols, ld, codes, scales, amax, global_scale, g_in);
+  FP4_HOST_CHECK(cudaGetLastError());
+  return FP4_OK;
+}
+
+fp4_status fp4_e2m1_to_e4m3(const uint8_t *codes_e2m1, int64_t rows, int64_t cols, uint8_t *codes_e4m3,
+                            fp4_stream_t stream) {
+  if (!codes_e2m1 || !codes_e4m3 || rows < 0 || cols <= 0) return FP4_ERR_INVALID_ARG;
+  if (cols % 32) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(codes_e2m1) || !aligned16(codes_e4m3)) return FP4_ERR_ALIGNMENT;
+  if (rows == 0) return FP4_OK;
+  const int64_t n32 = rows * (cols / 32);
+  e2m1_to_e4m3_kernel<<<grid_for(n32), kThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(codes_e2m1, n32,
+                                                                                             codes_e4m3);
   FP4_HOST_CHECK(cudaGetLastError());
   return FP4_OK;
 }

@@ -67,7 +67,7 @@ typedef enum {
   FP4_ERR_CUDA = 8               /* a CUDA runtime/driver call failed */
 } fp4_status;
 
-typedef enum { FP4_NV = 0, FP4_MX = 1 } fp4_format;
+typedef enum { FP4_NV = 0, FP4_MX = 1, FP4_MXFP8 = 2 } fp4_format;
 
 typedef enum { FP4_OUT_F32 = 0, FP4_OUT_BF16 = 1 } fp4_out_dtype;
 
@@ -78,6 +78,8 @@ typedef enum { FP4_OUT_F32 = 0, FP4_OUT_BF16 = 1 } fp4_out_dtype;
 #define FP4_GEMM_MX 0x8u             /* fp4_gemm: MXFP4 operands (UE8M0 per 32) */
 #define FP4_MOE_MX 0x10u             /* MoE layer / stages: MXFP4 weights, activations and h */
 #define FP4_MOE_PAIR_TILES 0x20u     /* MoE NVFP4 w13 / w2: CTA-pair tiles instead of 1-CTA row tiles */
+#define FP4_GEMM_A_MXFP8 0x40u       /* fp4_gemm: W4A8 -- A is MXFP8 (E4M3, UE8M0 per 32), B MXFP4 */
+#define FP4_GEMM_B_MXFP8 0x80u       /* fp4_gemm with FP4_GEMM_A_MXFP8: B is MXFP8 too */
 
 /* Human-readable name of a status code (static string). */
 const char *fp4_status_string(fp4_status s);
@@ -108,11 +110,25 @@ size_t fp4_quantize_workspace_size(void);
  *   FP4_SCALE_LAYOUT_TILED (cols % 128 == 0) the tiled layout with 32-element
  *   blocks (n_ksteps = cols/128; size fp4_sf_tiled_bytes(rows, cols) / 2).
  *   global_scale and workspace are ignored.
+ * FP4_MXFP8 (cols % 32 == 0) [QAT §4.2-4.3: FP8 activations for W4A8]: the
+ *   FP4_MX rule with E4M3 elements, X = clamp(floor(log2 amax)-8, -127, 127),
+ *   element = E4M3_RNE_satfinite(x * 2^-X) with the input's sign.  codes:
+ *   uint8 [rows][cols] (one E4M3 byte per element); scales as FP4_MX.
  * Alignment: x, codes, workspace 16-byte aligned; ld*2 % 16 == 0.
  */
 fp4_status fp4_quantize(fp4_format fmt, const void *x_bf16, int64_t rows, int64_t cols, int64_t ld,
                         uint8_t *codes, uint8_t *scales, float *global_scale, uint32_t flags,
                         void *workspace, size_t ws_bytes, fp4_stream_t stream);
+
+/*
+ * fp4_e2m1_to_e4m3 -- lossless FP4 -> FP8 widening [QAT §4.2]: packed E2M1
+ * codes uint8 [rows][cols/2] -> E4M3 bytes uint8 [rows][cols] holding the
+ * same values (sign included; code 8, -0, gives 0x80).  Block scales are not
+ * touched: an MXFP4 tensor's UE8M0 scales serve the widened MXFP8 tensor as
+ * they are.  cols % 32 == 0; both pointers 16-byte aligned.  Asynchronous.
+ */
+fp4_status fp4_e2m1_to_e4m3(const uint8_t *codes_e2m1, int64_t rows, int64_t cols, uint8_t *codes_e4m3,
+                            fp4_stream_t stream);
 
 /*
  * fp4_mx_to_nv -- lossless MXFP4 -> NVFP4 scale remap [NVFP4 §一 point 2, §六].
@@ -145,6 +161,12 @@ fp4_status fp4_mx_to_nv(const uint8_t *codes, const uint8_t *mx_scales, int64_t 
  * scales per 32 elements in the tiled layout with 32-element blocks (from
  * fp4_quantize(FP4_MX, FP4_SCALE_LAYOUT_TILED)); a_g/b_g are ignored (may be
  * NULL); C = A_dq . B_dq^T; K % 128 == 0.
+ * With flags & FP4_GEMM_A_MXFP8: W4A8 [QAT §4.3, FP8 activations x FP4
+ * weights] on tcgen05 kind::mxf8f6f4 -- A is MXFP8 (a_codes uint8 [M][K], one
+ * E4M3 byte per element, from fp4_quantize(FP4_MXFP8, tiled)); B is MXFP4
+ * (b_codes packed [N][K/2], 32-byte aligned) or, with FP4_GEMM_B_MXFP8,
+ * MXFP8 like A; a_sf/b_sf are tiled UE8M0 scales as for FP4_GEMM_MX; a_g/b_g
+ * are ignored; C = A_dq . B_dq^T; K % 128 == 0.
  */
 fp4_status fp4_gemm(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_g,
                     const uint8_t *b_codes, const uint8_t *b_sf, const float *b_g, void *c,

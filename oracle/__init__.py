@@ -15,13 +15,16 @@ Sources (cited by page title and section):
   * "DeepSeek-V4 architecture" page, §6.3 (1x32 MX tiles) and §5.1 (SwiGLU
     feed-forward layers); §2.1 (Pro shape: 384 experts, 6 active).
   * "DeepSeek-V4 FP4 QAT" page, §3.1 (simplified MoE forward: per-token
-    top-k experts, outputs summed).
+    top-k experts, outputs summed); §4.2 (FP4 -> FP8 widening without loss)
+    and §4.3 (FP8 activations against FP4 weights: W4A8).
 
 Modules:
   formats  -- E2M1 / E4M3 / UE8M0 encoders and decoders (brute-force nearest)
-  quant    -- NVFP4 and MXFP4 quantizers, dequantizers, MXFP4->NVFP4 remap
+  quant    -- NVFP4, MXFP4 and MXFP8 quantizers, dequantizers, MXFP4->NVFP4
+              remap, E2M1 -> E4M3 widening
   layouts  -- the tensor-core scale-factor tile layout (permutation only)
-  gemm     -- fp64 dequantize-then-matmul GEMM and its error bound
+  gemm     -- fp64 dequantize-then-matmul GEMMs (NVFP4, MXFP4, W4A8) and
+              their error bound
   moe      -- routing (stable sort), SwiGLU expert FFN, combine
 
 Parity pins: every function here is checked by ``tests/test_oracle_*.py``

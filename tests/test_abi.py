@@ -81,6 +81,14 @@ def test_host_validation_without_gpu():
     assert L.fp4_moe_gather(A, A, 8, 2, 256, 4, A, A, A, A, A, 16, None) == 6
     # MX->NV: cols not a multiple of 32
     assert L.fp4_mx_to_nv(A, A, 4, 48, 1, A, A, 0, None) == 3
+    # FP4 -> FP8 widening: cols % 32, misaligned output, null input
+    assert L.fp4_e2m1_to_e4m3(A, 4, 48, A, None) == 3
+    assert L.fp4_e2m1_to_e4m3(A, 4, 64, A + 8, None) == 2
+    assert L.fp4_e2m1_to_e4m3(None, 4, 64, A, None) == 1
+    # W4A8 GEMM: B_MXFP8 needs A_MXFP8; K % 128; packed FP4 B must be 32-byte aligned
+    assert L.fp4_gemm(A, A, None, A, A, None, A, 0, 128, 256, 512, 0x80, None) == 1
+    assert L.fp4_gemm(A, A, None, A, A, None, A, 0, 128, 256, 576, 0x40, None) == 3
+    assert L.fp4_gemm(A, A, None, A + 16, A, None, A, 0, 128, 256, 512, 0x40, None) == 2
 
 
 def test_package_fails_loudly_without_library(tmp_path, monkeypatch):
