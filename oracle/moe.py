@@ -21,7 +21,8 @@ caller's top-k weight (1.0 when none is given) and sums slots in order 0..k-1.
 import numpy as np
 
 from .formats import f64_to_bf16_rne
-from .quant import mxfp4_dequantize, mxfp4_quantize, nvfp4_dequantize, nvfp4_quantize
+from .quant import (mxfp4_dequantize, mxfp4_quantize, mxfp8_dequantize, mxfp8_quantize, nvfp4_dequantize,
+                    nvfp4_quantize)
 
 
 def route(expert_ids, num_experts):
@@ -88,6 +89,20 @@ def expert_ffn_ref_mx(x_dq_rows, w1_dq, w3_dq, w2_dq):
     h = swiglu(gate, up)
     h_codes, h_sc = mxfp4_quantize(h.astype(np.float32))
     h_dq = mxfp4_dequantize(h_codes, h_sc)
+    y = h_dq @ w2_dq.T
+    return dict(gate=gate, up=up, h=h, h_codes=h_codes, h_sc=h_sc, h_dq=h_dq, y=y)
+
+
+def expert_ffn_ref_w4a8(x_dq_rows, w1_dq, w3_dq, w2_dq):
+    """W4A8 variant ("DeepSeek-V4 FP4 QAT" §4.3: FP8 activations, FP4
+    weights): x_dq_rows are the dequantized MXFP8 activations, the weights
+    dequantized MXFP4; h is re-quantized to MXFP8 (E4M3 elements, one
+    power-of-two scale per 32) from h rounded once to fp32."""
+    gate = x_dq_rows @ w1_dq.T
+    up = x_dq_rows @ w3_dq.T
+    h = swiglu(gate, up)
+    h_codes, h_sc = mxfp8_quantize(h.astype(np.float32))
+    h_dq = mxfp8_dequantize(h_codes, h_sc)
     y = h_dq @ w2_dq.T
     return dict(gate=gate, up=up, h=h, h_codes=h_codes, h_sc=h_sc, h_dq=h_dq, y=y)
 

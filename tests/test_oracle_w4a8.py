@@ -130,3 +130,23 @@ def test_w4a8_fp4_and_widened_fp8_weights_agree_exactly():
     C4, _ = G.w4a8_gemm_ref(ac, as_, wc, ws)
     C8, _ = G.w4a8_gemm_ref(ac, as_, Q.e2m1_to_e4m3(wc), ws, b_is_fp8=True)
     assert np.array_equal(C4, C8)
+
+
+def test_expert_ffn_w4a8_requantizes_h_to_mxfp8():
+    from oracle import moe as M
+
+    rng = np.random.default_rng(4)
+    x = rng.standard_normal((5, 64))
+    w1, w3 = rng.standard_normal((32, 64)) * 0.1, rng.standard_normal((32, 64)) * 0.1
+    w2 = rng.standard_normal((64, 32)) * 0.1
+    r = M.expert_ffn_ref_w4a8(x, w1, w3, w2)
+    # silu in closed form, then one RN of h to fp32 before the MXFP8 encode
+    np.testing.assert_allclose(r["h"], (r["gate"] / (1 + np.exp(-r["gate"]))) * r["up"], rtol=1e-15)
+    hc, hs = Q.mxfp8_quantize(r["h"].astype(np.float32))
+    assert np.array_equal(hc, r["h_codes"]) and np.array_equal(hs, r["h_sc"])
+    # each element of h_dq is within 64 * 2^X of h: half the largest E4M3 spacing (32 * 2^X in the top
+    # octave, 256..448 before scaling) or the saturation of [448, 512) * 2^X to 448 * 2^X
+    X = np.repeat(hs.astype(np.int64) - 127, 32, axis=1)
+    err = np.abs(r["h_dq"] - r["h"].astype(np.float32))
+    assert np.all(err <= 64.0 * np.exp2(X))
+    np.testing.assert_allclose(r["y"], r["h_dq"] @ w2.T, rtol=1e-15)
