@@ -43,6 +43,8 @@ WORKLOADS = {
     "decode": (64, 7168, 2048, 384, 6, 1.1, 0.01, "Pro-shaped MoE layer at 64 decode tokens (weight-read bound)"),
     "flashmx": (4096, 4096, 2048, 256, 6, 0.0, 0.02,
                 "Flash-shaped MoE layer run natively in MXFP4 (UE8M0/32 weights, activations and h; no remap)"),
+    "flashw4a8": (4096, 4096, 2048, 256, 6, 0.0, 0.02,
+                  "Flash-shaped MoE layer in W4A8: MXFP4 weights (UE8M0/32) x MXFP8 activations and h (E4M3, UE8M0/32)"),
     "pro64": (4096, 7168, 2048, 64, 6, 1.1, 0.01,
               "Pro-shaped expert matrices, 64 experts, 4096 tokens, top-6, Zipf 1.1 (profiling size)"),
 }
@@ -187,8 +189,9 @@ class MoeBench:
         import synth
 
         self.fp4 = fp4
-        self.mx = name.endswith("mx")
-        self.flags = fp4.FP4_MOE_MX if self.mx else 0
+        self.w4a8 = name.endswith("w4a8")  # MXFP4 weights, MXFP8 activations and h
+        self.mx = name.endswith("mx") or self.w4a8  # power-of-two scales, no tensor scales
+        self.flags = fp4.FP4_MOE_W4A8 if self.w4a8 else fp4.FP4_MOE_MX if self.mx else 0
         # NVFP4 grouped GEMMs on 1-CTA row tiles unless CTA pairs are asked for (MXFP4 always row tiles)
         self.pair = pair_tiles and not self.mx
         if self.pair:
@@ -248,9 +251,10 @@ class MoeBench:
         self.counts_d, self.offs, self.toffs = i32(E), i32(E + 1), i32(E + 1)
         self.perm, self.inv = i32(R), i32(R)
         self.scratch = u8(fp4.fp4_moe_route_scratch_bytes(R, E))
-        self.a_c = torch.empty((cap, H // 2), dtype=torch.uint8, device=d)
+        cpb = 1 if self.w4a8 else 2  # codes per byte of the gathered x and of h
+        self.a_c = torch.empty((cap, H // cpb), dtype=torch.uint8, device=d)
         self.a_s = u8(fp4.fp4_sf_tiled_bytes(cap, H))  # (an MX run uses the first half)
-        self.h_c = torch.empty((cap, I // 2), dtype=torch.uint8, device=d)
+        self.h_c = torch.empty((cap, I // cpb), dtype=torch.uint8, device=d)
         self.h_s = u8(fp4.fp4_sf_tiled_bytes(cap, I))
         self.y = torch.empty((R, H), dtype=torch.float32, device=d)
         self.out = torch.empty((T, H), dtype=torch.bfloat16, device=d)
@@ -367,13 +371,17 @@ def run_moe(args, world, rank, peaks):
             stage[j] += evs[i][j].elapsed_time(evs[i][j + 1]) / args.steps
     flops = b.flops()
     value = world * flops / (ms * 1e-3) / 1e12
-    fp4_peak = 4.0 * peaks["bf16_sus"]
+    # FP4 x FP4 runs at 4x the bf16 rate, FP8 x FP4 (W4A8) at the FP8 rate, 2x (the recipe's nominal ratios)
+    ratio = 2.0 if b.w4a8 else 4.0
+    fp4_peak = ratio * peaks["bf16_sus"]
     # dominant kernel: the grouped w13 GEMM (2/3 of the layer's FLOPs)
     w13_flops = 2.0 * 2 * b.I * b.H * b.R
     w13_tf = w13_flops / (stage[2] * 1e-3) / 1e12
     # algorithmic bytes of the w13 launch: touched experts' w13 weights, the gathered rows, h out
     n_touched = int((b.counts > 0).sum().item())
-    w13_bytes = n_touched * 2 * b.I * b.H * 0.5625 + b.R * b.H * 0.5625 + b.R * b.I * 0.5625
+    act_b = 1.03125 if b.w4a8 else 0.5625  # bytes per activation / h element (codes + scales)
+    w_b = 0.53125 if b.mx else 0.5625  # bytes per weight element
+    w13_bytes = n_touched * 2 * b.I * b.H * w_b + b.R * b.H * act_b + b.R * b.I * act_b
     w2_tf = (2.0 * b.I * b.H * b.R) / (stage[3] * 1e-3) / 1e12
     q_bytes = b.T * b.H * 2.0 + b.R * b.H * 0.5625  # read x once, write every routed row
     q_gbs = q_bytes / (stage[1] * 1e-3) / 1e9
@@ -391,7 +399,8 @@ def run_moe(args, world, rank, peaks):
     ids_d = [torch.empty_like(b.ids) for _ in range(nb)]
     w_d = [torch.empty_like(b.w) for _ in range(nb)]
     out_d = [torch.empty((b.T, b.H), dtype=torch.bfloat16, device="cuda") for _ in range(nb)]
-    ws = torch.empty(fp4.fp4_moe_workspace_size(b.T, b.k, b.H, b.I, b.E), dtype=torch.uint8, device="cuda")
+    ws = torch.empty(fp4.fp4_moe_workspace_size_flags(b.T, b.k, b.H, b.I, b.E, b.flags), dtype=torch.uint8,
+                     device="cuda")
     s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
     ev_in = [torch.cuda.Event() for _ in range(nb)]
     ev_cmp = [torch.cuda.Event() for _ in range(nb)]
@@ -447,7 +456,9 @@ def run_moe(args, world, rank, peaks):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "nvfp4 (e2m1 x e2m1, e4m3/16 scales, fp32 accumulate)",
+        "dtype": ("mxfp8 x mxfp4 (e4m3 activations x e2m1 weights, ue8m0/32 scales, fp32 accumulate)" if b.w4a8 else
+                  "mxfp4 (e2m1 x e2m1, ue8m0/32 scales, fp32 accumulate)" if b.mx else
+                  "nvfp4 (e2m1 x e2m1, e4m3/16 scales, fp32 accumulate)"),
         "data": "synthetic (seeded): bf16 N(0,1) activations, N(0,sigma)+0.5% x30 outlier weights, Gaussian router"
                 " logits + Zipf popularity",
         "config": {"workload": b.desc, "tokens": b.T, "hidden": b.H, "intermediate": b.I, "experts": b.E,
@@ -462,7 +473,8 @@ def run_moe(args, world, rank, peaks):
                      "algorithmic_bytes": w13_bytes,
                      "frac_of_max_flops_bytes": round(max(w13_flops / (fp4_peak * 1e12), w13_bytes / (peaks["hbm"] * 1e9))
                                                       / (stage[2] * 1e-3), 4),
-                     "peak_note": "4 x measured sustained bf16 cuBLAS (nominal fp4/bf16 ratio), of " + peaks["src"]},
+                     "peak_note": "%dx measured sustained bf16 cuBLAS (nominal %s/bf16 ratio), of %s"
+                                  % (ratio, "fp8" if b.w4a8 else "fp4", peaks["src"])},
         "stages_ms": {n: round(v, 4) for n, v in zip(["route", "quantize_gather", "w13", "w2", "combine"], stage)},
         "w2": {"achieved_tflops": round(w2_tf, 1), "frac": round(w2_tf / fp4_peak, 4),
                "traffic": measured_traffic(args.workload, b.kernel_name("w2"))},
@@ -518,15 +530,24 @@ def cpu_baseline_moe(b, n_tokens=1):
         return Q.nvfp4_dequantize(*Q.nvfp4_quantize(w))
 
     t0 = time.perf_counter()
-    x_dq = Q.mxfp4_dequantize(*Q.mxfp4_quantize(xs)) if b.mx else Q.nvfp4_dequantize(*Q.nvfp4_quantize(xs, g=g))
+    if b.w4a8:
+        x_dq = Q.mxfp8_dequantize(*Q.mxfp8_quantize(xs))
+    elif b.mx:
+        x_dq = Q.mxfp4_dequantize(*Q.mxfp4_quantize(xs))
+    else:
+        x_dq = Q.nvfp4_dequantize(*Q.nvfp4_quantize(xs, g=g))
     dq = {e: (MO.deinterleave_w13(deq(wb[e][0])), deq(wb[e][1])) for e in experts}
     out = np.zeros((n_tokens, b.H))
     for t in range(n_tokens):
         for s in range(b.k):
             e = int(ids[t, s])
             (w1d, w3d), w2d = dq[e]
-            r = (MO.expert_ffn_ref_mx(x_dq[t:t + 1], w1d, w3d, w2d) if b.mx
-                 else MO.expert_ffn_ref(x_dq[t:t + 1], w1d, w3d, w2d, hg[e]))
+            if b.w4a8:
+                r = MO.expert_ffn_ref_w4a8(x_dq[t:t + 1], w1d, w3d, w2d)
+            elif b.mx:
+                r = MO.expert_ffn_ref_mx(x_dq[t:t + 1], w1d, w3d, w2d)
+            else:
+                r = MO.expert_ffn_ref(x_dq[t:t + 1], w1d, w3d, w2d, hg[e])
             out[t] += wts[t, s] * r["y"][0]
     dt = time.perf_counter() - t0
     flops = 2.0 * 3 * b.H * b.I * b.k * n_tokens

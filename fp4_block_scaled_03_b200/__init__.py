@@ -26,6 +26,7 @@ FP4_DEBUG_DUMP_H = 0x4
 FP4_GEMM_MX = 0x8
 FP4_GEMM_A_MXFP8 = 0x40
 FP4_GEMM_B_MXFP8 = 0x80
+FP4_MOE_W4A8 = 0x100
 FP4_MOE_MX = 0x10
 FP4_MOE_PAIR_TILES = 0x20
 
@@ -81,6 +82,7 @@ _SIGS = {
     "fp4_e2m1_to_e4m3": (ctypes.c_int, [_P, _I64, _I64, _P, _P]),
     "fp4_gemm": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, ctypes.c_int, _I64, _I64, _I64, _U32, _P]),
     "fp4_moe_workspace_size": (_SZ, [_I64, _I32, _I64, _I64, _I32]),
+    "fp4_moe_workspace_size_flags": (_SZ, [_I64, _I32, _I64, _I64, _I32, _U32]),
     "fp4_moe_grouped_gemm": (
         ctypes.c_int,
         [_P, _P, _P, _I64, _I32, ctypes.POINTER(MoeWeights), _I64, _I64, _I32, _P, _P, _SZ, _U32, _P, _P],
@@ -222,6 +224,10 @@ def fp4_moe_workspace_size(T, topk, H, I, E):
     return lib.fp4_moe_workspace_size(T, topk, H, I, E)
 
 
+def fp4_moe_workspace_size_flags(T, topk, H, I, E, flags):
+    return lib.fp4_moe_workspace_size_flags(T, topk, H, I, E, flags)
+
+
 def fp4_moe_route_scratch_bytes(R, E):
     return lib.fp4_moe_route_scratch_bytes(R, E)
 
@@ -327,14 +333,16 @@ def moe_rows_cap(T, topk, E):
 
 
 def moe_layer(x, expert_ids, topk_weights, w, H, I, E, workspace=None, out=None, h_dump=None, mx=False,
-              pair_tiles=False):
+              pair_tiles=False, w4a8=False):
+    """mx: MXFP4 weights, activations and h.  w4a8: MXFP4 weights with MXFP8
+    activations and h (FP8 x FP4 grouped GEMMs)."""
     T, topk = expert_ids.shape
     dev = x.device
+    flags = (FP4_DEBUG_DUMP_H if h_dump is not None else 0) | (FP4_MOE_MX if mx else 0)
+    flags |= (FP4_MOE_PAIR_TILES if pair_tiles else 0) | (FP4_MOE_W4A8 if w4a8 else 0)
     if workspace is None:
-        workspace = _u8(fp4_moe_workspace_size(T, topk, H, I, E), dev)
+        workspace = _u8(fp4_moe_workspace_size_flags(T, topk, H, I, E, flags), dev)
     if out is None:
         out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
-    flags = (FP4_DEBUG_DUMP_H if h_dump is not None else 0) | (FP4_MOE_MX if mx else 0)
-    flags |= FP4_MOE_PAIR_TILES if pair_tiles else 0
     fp4_moe_grouped_gemm(x, expert_ids, topk_weights, T, topk, w, H, I, E, out, workspace, flags, h_dump)
     return out

@@ -137,6 +137,41 @@ __device__ __forceinline__ uint32_t mxfp4_block32(const float *x, uint32_t *code
   return scale;
 }
 
+// Four fp32 -> 32 bits of E4M3 bytes (element 0 in the lowest byte), round to
+// nearest even, saturating at +-448, sign kept.  The cvt writes its first
+// source to the high byte of each 16-bit pair.
+__device__ __forceinline__ uint32_t pack4_e4m3(float a, float b, float c, float d) {
+  uint16_t lo, hi;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(b), "f"(a));
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(d), "f"(c));
+  return (uint32_t)lo | ((uint32_t)hi << 16);
+}
+
+// MXFP8 quantization of one 32-element block held in fp32 registers (the
+// MXFP4 rule with E4M3 elements): X = clamp(floor(log2 amax) - 8, -127, 127),
+// byte X + 127 (0 for an all-zero block), element = E4M3_RNE_satfinite(x * 2^-X).
+// Returns the scale byte and writes 32 E4M3 bytes (eight words).
+__device__ __forceinline__ uint32_t mxfp8_block32(const float *x, uint32_t *codes8) {
+  float a = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) a = fmaxf(a, fabsf(x[i]));
+  int X = 0;
+  uint32_t scale = 0;
+  if (a > 0.0f) {
+    const uint32_t bits = __float_as_uint(a);
+    const int e = (int)(bits >> 23);
+    const int fl = e ? e - 127 : (31 - __clz((int)(bits & 0x7FFFFFu))) - 149;  // exact floor(log2 a)
+    X = min(max(fl - 8, -127), 127);
+    scale = (uint32_t)(X + 127);
+  }
+  const float p = __uint_as_float((uint32_t)(127 - X) << 23);  // 2^-X (X <= 119 for finite fp32)
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+    codes8[q] = pack4_e4m3(__fmul_rn(x[4 * q], p), __fmul_rn(x[4 * q + 1], p), __fmul_rn(x[4 * q + 2], p),
+                           __fmul_rn(x[4 * q + 3], p));
+  return scale;
+}
+
 // ---------------------------------------------------------------------------
 // shared memory, mbarriers, TMA
 // ---------------------------------------------------------------------------

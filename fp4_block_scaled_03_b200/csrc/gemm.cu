@@ -378,9 +378,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (EPI == EPI_W2 && p.topk_w) scale = MX ? p.topk_w[p.perm[ti.out_row0 + row]]
                                                 : __fmul_rn(alpha, p.topk_w[p.perm[ti.out_row0 + row]]);
       const int colh = ti.n0 + half * HC;
-      if constexpr (EPI == EPI_W13 && KIND == 1) {
-        // MXFP4 h: one 32-element block per pair of 32-column chunks (16 gate +
-        // 16 up columns each), quantized with its own power-of-two scale
+      if constexpr (EPI == EPI_W13 && KIND >= 1) {
+        // MXFP4 h (KIND 1) or MXFP8 h (KIND 2, W4A8): one 32-element block per
+        // pair of 32-column chunks (16 gate + 16 up columns each), quantized
+        // with its own power-of-two scale
 #pragma unroll
         for (int cp = 0; cp < HC / 64; ++cp) {
           const int col0 = colh + cp * 64;
@@ -395,9 +396,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const int hc = col0 / 2;  // a multiple of 32
           const int64_t prow = (int64_t)ti.a_row0 + row;
-          uint32_t cq[4];
-          const uint32_t sc = mxfp4_block32(h, cq);
-          *reinterpret_cast<uint4 *>(p.h_codes + prow * (p.I / 2) + hc / 2) = make_uint4(cq[0], cq[1], cq[2], cq[3]);
+          uint32_t sc;
+          if constexpr (KIND == 2) {
+            uint32_t c8[8];
+            sc = mxfp8_block32(h, c8);
+            uint4 *dst = reinterpret_cast<uint4 *>(p.h_codes + prow * p.I + hc);
+            dst[0] = make_uint4(c8[0], c8[1], c8[2], c8[3]);
+            dst[1] = make_uint4(c8[4], c8[5], c8[6], c8[7]);
+          } else {
+            uint32_t cq[4];
+            sc = mxfp4_block32(h, cq);
+            *reinterpret_cast<uint4 *>(p.h_codes + prow * (p.I / 2) + hc / 2) = make_uint4(cq[0], cq[1], cq[2], cq[3]);
+          }
           p.h_sf[sf_tiled_offset(prow, hc / 32, p.I / 128)] = (uint8_t)sc;
           if (p.h_dump) {
             float4 *d = reinterpret_cast<float4 *>(p.h_dump + prow * p.I + hc);
@@ -578,13 +588,14 @@ fp4_status fp4_moe_w13(const uint8_t *a_codes, const uint8_t *a_sf, const float 
                        fp4_stream_t stream) {
   if (!a_codes || !a_sf || !w || !w->w13_codes || !w->w13_sf || !counts || !tile_offsets || !h_codes || !h_sf)
     return FP4_ERR_INVALID_ARG;
-  if (!(flags & FP4_MOE_MX) && (!a_g || !w->w13_g || !w->h_g)) return FP4_ERR_INVALID_ARG;
+  const bool w4a8 = flags & FP4_MOE_W4A8;  // MXFP8 activations and h, MXFP4 weights
+  const bool mx = (flags & FP4_MOE_MX) || w4a8;
+  if (!mx && (!a_g || !w->w13_g || !w->h_g)) return FP4_ERR_INVALID_ARG;
   if ((flags & FP4_DEBUG_DUMP_H) && !h_dump) return FP4_ERR_INVALID_ARG;
-  const bool mx = flags & FP4_MOE_MX;
   if (H < 256 || H % 256 || I < 256 || I % 256 || E < 1 || E > 4096 || rows_cap < 1) return FP4_ERR_UNSUPPORTED_SHAPE;
   if ((int64_t)E * 2 * I > (1LL << 31) - 1 || rows_cap > (1LL << 31) - 1) return FP4_ERR_UNSUPPORTED_SHAPE;
   if (!al16(a_codes) || !al16(a_sf) || !al16(w->w13_codes) || !al16(w->w13_sf) || !al16(h_codes) || !al16(h_sf) ||
-      (h_dump && !al16(h_dump)))
+      (h_dump && !al16(h_dump)) || (w4a8 && (reinterpret_cast<uintptr_t>(w->w13_codes) & 31u)))
     return FP4_ERR_ALIGNMENT;
   if (!mx && (flags & FP4_MOE_PAIR_TILES)) {
     if (((rows_cap + 255) / 256 + E) * (2 * I / 256) > (1LL << 31) - 1) return FP4_ERR_UNSUPPORTED_SHAPE;
@@ -594,14 +605,21 @@ fp4_status fp4_moe_w13(const uint8_t *a_codes, const uint8_t *a_sf, const float 
   const DeviceCtx *ctx = device_ctx();
   if (!ctx) return FP4_ERR_CUDA;
   CUtensorMap ta, tb;
-  if (!make_code_map(&ta, a_codes, (uint64_t)rows_cap, (uint64_t)H / 2, BM)) return FP4_ERR_CUDA;
-  if (!make_code_map(&tb, w->w13_codes, (uint64_t)E * 2 * I, (uint64_t)H / 2, kBN)) return FP4_ERR_CUDA;
+  if (w4a8) {  // A: one E4M3 byte per element; B: packed E2M1 unpacked by the TMA
+    if (!make_code_map(&ta, a_codes, (uint64_t)rows_cap, (uint64_t)H, BM)) return FP4_ERR_CUDA;
+    if (!make_u4_unpack_map(&tb, w->w13_codes, (uint64_t)E * 2 * I, (uint64_t)H, kBN)) return FP4_ERR_CUDA;
+  } else {
+    if (!make_code_map(&ta, a_codes, (uint64_t)rows_cap, (uint64_t)H / 2, BM)) return FP4_ERR_CUDA;
+    if (!make_code_map(&tb, w->w13_codes, (uint64_t)E * 2 * I, (uint64_t)H / 2, kBN)) return FP4_ERR_CUDA;
+  }
   Params p = {};
   p.N = (int)(2 * I); p.K = (int)H;
   p.n_tiles = (int)(2 * I / kBN);
-  p.k_stages = (int)(H / 256);
-  p.kw = (int)(H / 64);
+  p.k_stages = w4a8 ? (int)(H / 128) : (int)(H / 256);
+  p.kw = w4a8 ? (int)(H / 32) : (int)(H / 64);
   p.kw_sf = mx ? (int)(H / 128) : p.kw;
+  p.b_fmt = 5;
+  p.b_tx = (uint32_t)kBN * 64u;
   p.a_sf = a_sf; p.b_sf = w->w13_sf;
   p.b_sf_rows = (int64_t)E * 2 * I;
   p.a_g = a_g;
@@ -611,6 +629,7 @@ fp4_status fp4_moe_w13(const uint8_t *a_codes, const uint8_t *a_sf, const float 
   p.h_dump = (flags & FP4_DEBUG_DUMP_H) ? h_dump : nullptr;
   p.status = ctx->status;
   p.wait_limit = ctx->wait_limit_ns;
+  if (w4a8) return launch<kBN, EPI_W13, 2>(ta, tb, tb, p, sm_count(), reinterpret_cast<cudaStream_t>(stream));
   if (mx) return launch<kBN, EPI_W13, 1>(ta, tb, tb, p, sm_count(), reinterpret_cast<cudaStream_t>(stream));
   return launch<kBN, EPI_W13>(ta, tb, tb, p, sm_count(), reinterpret_cast<cudaStream_t>(stream));
 }
@@ -619,13 +638,15 @@ fp4_status fp4_moe_w2(const uint8_t *h_codes, const uint8_t *h_sf, const fp4_moe
                       int32_t E, const int32_t *counts, const int32_t *offsets, const int32_t *tile_offsets,
                       const int32_t *perm, const float *topk_weights, int64_t rows_cap, float *y, uint32_t flags,
                       fp4_stream_t stream) {
-  const bool mx = flags & FP4_MOE_MX;
+  const bool w4a8 = flags & FP4_MOE_W4A8;
+  const bool mx = (flags & FP4_MOE_MX) || w4a8;
   if (!h_codes || !h_sf || !w || !w->w2_codes || !w->w2_sf || !counts || !offsets || !tile_offsets || !perm || !y)
     return FP4_ERR_INVALID_ARG;
   if (!mx && (!w->w2_g || !w->h_g)) return FP4_ERR_INVALID_ARG;
   if (H < 256 || H % 256 || I < 256 || I % 256 || E < 1 || E > 4096 || rows_cap < 1) return FP4_ERR_UNSUPPORTED_SHAPE;
   if ((int64_t)E * H > (1LL << 31) - 1 || rows_cap > (1LL << 31) - 1) return FP4_ERR_UNSUPPORTED_SHAPE;
   if (!al16(h_codes) || !al16(h_sf) || !al16(w->w2_codes) || !al16(w->w2_sf) || !al16(y)) return FP4_ERR_ALIGNMENT;
+  if (w4a8 && (reinterpret_cast<uintptr_t>(w->w2_codes) & 31u)) return FP4_ERR_ALIGNMENT;
   if (!mx && (flags & FP4_MOE_PAIR_TILES)) {
     if (((rows_cap + 255) / 256 + E) * (H / 256) > (1LL << 31) - 1) return FP4_ERR_UNSUPPORTED_SHAPE;
     return moe_pair_w2(h_codes, h_sf, w, H, I, E, counts, offsets, tile_offsets, perm, topk_weights, rows_cap, y,
@@ -634,14 +655,21 @@ fp4_status fp4_moe_w2(const uint8_t *h_codes, const uint8_t *h_sf, const fp4_moe
   const DeviceCtx *ctx = device_ctx();
   if (!ctx) return FP4_ERR_CUDA;
   CUtensorMap ta, tb;
-  if (!make_code_map(&ta, h_codes, (uint64_t)rows_cap, (uint64_t)I / 2, BM)) return FP4_ERR_CUDA;
-  if (!make_code_map(&tb, w->w2_codes, (uint64_t)E * H, (uint64_t)I / 2, kBN)) return FP4_ERR_CUDA;
+  if (w4a8) {
+    if (!make_code_map(&ta, h_codes, (uint64_t)rows_cap, (uint64_t)I, BM)) return FP4_ERR_CUDA;
+    if (!make_u4_unpack_map(&tb, w->w2_codes, (uint64_t)E * H, (uint64_t)I, kBN)) return FP4_ERR_CUDA;
+  } else {
+    if (!make_code_map(&ta, h_codes, (uint64_t)rows_cap, (uint64_t)I / 2, BM)) return FP4_ERR_CUDA;
+    if (!make_code_map(&tb, w->w2_codes, (uint64_t)E * H, (uint64_t)I / 2, kBN)) return FP4_ERR_CUDA;
+  }
   Params p = {};
   p.N = (int)H; p.K = (int)I;
   p.n_tiles = (int)(H / kBN);
-  p.k_stages = (int)(I / 256);
-  p.kw = (int)(I / 64);
+  p.k_stages = w4a8 ? (int)(I / 128) : (int)(I / 256);
+  p.kw = w4a8 ? (int)(I / 32) : (int)(I / 64);
   p.kw_sf = mx ? (int)(I / 128) : p.kw;
+  p.b_fmt = 5;
+  p.b_tx = (uint32_t)kBN * 64u;
   p.a_sf = h_sf; p.b_sf = w->w2_sf;
   p.b_sf_rows = (int64_t)E * H;
   p.E = E; p.counts = counts; p.offsets = offsets; p.tile_offsets = tile_offsets;
@@ -651,6 +679,7 @@ fp4_status fp4_moe_w2(const uint8_t *h_codes, const uint8_t *h_sf, const fp4_moe
   p.wait_limit = ctx->wait_limit_ns;
   CUtensorMap ty;
   if (!make_f32_store_map(&ty, y, (uint64_t)rows_cap, (uint64_t)H)) return FP4_ERR_CUDA;
+  if (w4a8) return launch<kBN, EPI_W2, 2>(ta, tb, ty, p, sm_count(), reinterpret_cast<cudaStream_t>(stream));
   if (mx) return launch<kBN, EPI_W2, 1>(ta, tb, ty, p, sm_count(), reinterpret_cast<cudaStream_t>(stream));
   return launch<kBN, EPI_W2>(ta, tb, ty, p, sm_count(), reinterpret_cast<cudaStream_t>(stream));
 }

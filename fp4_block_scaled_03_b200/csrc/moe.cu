@@ -20,7 +20,8 @@ struct MoeLayout {
 
 size_t up256(size_t v) { return (v + 255) & ~size_t(255); }
 
-MoeLayout moe_layout(int64_t T, int32_t topk, int64_t H, int64_t I, int32_t E) {
+// codes_per_byte: 2 for FP4 activations and h, 1 for FP8 (W4A8).
+MoeLayout moe_layout(int64_t T, int32_t topk, int64_t H, int64_t I, int32_t E, int codes_per_byte) {
   MoeLayout L;
   const int64_t R = T * topk;
   L.rows_cap = ((R + 127LL * E + 127) / 128) * 128;
@@ -37,9 +38,9 @@ MoeLayout moe_layout(int64_t T, int32_t topk, int64_t H, int64_t I, int32_t E) {
   L.perm = take((size_t)R * 4);
   L.inv = take((size_t)R * 4);
   L.scratch = take(fp4_moe_route_scratch_bytes(R, E));
-  L.a_codes = take((size_t)(L.rows_cap * H / 2));
+  L.a_codes = take((size_t)(L.rows_cap * H / codes_per_byte));
   L.a_sf = take(fp4_sf_tiled_bytes(L.rows_cap, H));
-  L.h_codes = take((size_t)(L.rows_cap * I / 2));
+  L.h_codes = take((size_t)(L.rows_cap * I / codes_per_byte));
   L.h_sf = take(fp4_sf_tiled_bytes(L.rows_cap, I));
   L.y = take((size_t)R * (size_t)H * 4);
   L.total = off;
@@ -52,7 +53,12 @@ extern "C" {
 
 size_t fp4_moe_workspace_size(int64_t T, int32_t topk, int64_t H, int64_t I, int32_t E) {
   if (T < 0 || topk < 1 || H <= 0 || I <= 0 || E < 1) return 0;
-  return moe_layout(T, topk, H, I, E).total;
+  return moe_layout(T, topk, H, I, E, 2).total;
+}
+
+size_t fp4_moe_workspace_size_flags(int64_t T, int32_t topk, int64_t H, int64_t I, int32_t E, uint32_t flags) {
+  if (T < 0 || topk < 1 || H <= 0 || I <= 0 || E < 1) return 0;
+  return moe_layout(T, topk, H, I, E, (flags & FP4_MOE_W4A8) ? 1 : 2).total;
 }
 
 fp4_status fp4_moe_grouped_gemm(const void *tokens_bf16, const int32_t *expert_ids, const float *topk_weights,
@@ -63,7 +69,7 @@ fp4_status fp4_moe_grouped_gemm(const void *tokens_bf16, const int32_t *expert_i
   if (T < 0 || topk < 1 || topk > 16 || E < 1 || E > 4096) return FP4_ERR_UNSUPPORTED_SHAPE;
   if (H < 256 || H % 256 || I < 256 || I % 256) return FP4_ERR_UNSUPPORTED_SHAPE;
   if (reinterpret_cast<uintptr_t>(workspace) & 255u) return FP4_ERR_ALIGNMENT;
-  const MoeLayout L = moe_layout(T, topk, H, I, E);
+  const MoeLayout L = moe_layout(T, topk, H, I, E, (flags & FP4_MOE_W4A8) ? 1 : 2);
   if (ws_bytes < L.total) return FP4_ERR_WORKSPACE;
   if ((flags & FP4_DEBUG_DUMP_H) && !h_dump) return FP4_ERR_INVALID_ARG;
   if (T == 0) return FP4_OK;
@@ -74,7 +80,7 @@ fp4_status fp4_moe_grouped_gemm(const void *tokens_bf16, const int32_t *expert_i
   st = fp4_moe_route(expert_ids, T, topk, E, I32(L.counts), I32(L.offsets), I32(L.tile_offsets), I32(L.perm),
                      I32(L.inv), ws + L.scratch, fp4_moe_route_scratch_bytes(T * topk, E), stream);
   if (st != FP4_OK) return st;
-  const uint32_t fmt = flags & FP4_MOE_MX;
+  const uint32_t fmt = flags & (FP4_MOE_MX | FP4_MOE_W4A8);
   const uint32_t tiling = flags & FP4_MOE_PAIR_TILES;
   st = fp4_moe_quantize_gather(tokens_bf16, T, topk, H, E, I32(L.offsets), I32(L.tile_offsets), I32(L.inv),
                                ws + L.a_codes, ws + L.a_sf, L.rows_cap, g_x, ws + L.header, 256, fmt, stream);

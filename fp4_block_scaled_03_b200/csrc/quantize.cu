@@ -244,14 +244,46 @@ __global__ void __launch_bounds__(128) mxfp4_quantize_gather_kernel(
   }
 }
 
-// Four fp32 -> 32 bits of E4M3 bytes (element 0 in the lowest byte), round to
-// nearest even, saturating at +-448, sign kept.  The cvt writes its first
-// source to the high byte of each 16-bit pair.
-__device__ __forceinline__ uint32_t pack4_e4m3(float a, float b, float c, float d) {
-  uint16_t lo, hi;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(b), "f"(a));
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(d), "f"(c));
-  return (uint32_t)lo | ((uint32_t)hi << 16);
+// MXFP8 (W4A8 activations): a lane's K step is 128 elements (four 32-element
+// blocks, one tiled scale word); codes are one E4M3 byte per element.
+__global__ void __launch_bounds__(128) mxfp8_quantize_gather_kernel(
+    const uint16_t *__restrict__ x, int64_t T, int64_t H, int32_t topk, int32_t E,
+    const int32_t *__restrict__ offsets, const int32_t *__restrict__ tile_offsets, const int32_t *__restrict__ inv,
+    uint8_t *__restrict__ a_codes, uint8_t *__restrict__ a_sf) {
+  const int lane = threadIdx.x & 31;
+  const int64_t n_ksteps = H / 128;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
+  for (int64_t t = blockIdx.x * (int64_t)(blockDim.x / 32) + (threadIdx.x >> 5); t < T; t += warps) {
+    int64_t dd[16];
+    gather_destinations(offsets, tile_offsets, inv, E, topk, t, lane, dd);
+    for (int64_t kw = lane; kw < n_ksteps; kw += 32) {
+      const uint4 *src = reinterpret_cast<const uint4 *>(x + t * H + kw * 128);
+      uint32_t code[32], sfw = 0;
+#pragma unroll
+      for (int blk = 0; blk < 4; ++blk) {
+        float f[32];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint4 v = __ldcs(src + 4 * blk + q);
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            f[8 * q + 2 * j] = bf16_bits_to_f32(w[j] & 0xFFFFu);
+            f[8 * q + 2 * j + 1] = bf16_bits_to_f32(w[j] >> 16);
+          }
+        }
+        sfw |= mxfp8_block32(f, code + 8 * blk) << (8 * blk);
+      }
+      for (int s = 0; s < topk; ++s) {
+        const int64_t d = dd[s];
+        if (d < 0) continue;
+        uint4 *out = reinterpret_cast<uint4 *>(a_codes + d * H + kw * 128);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) out[q] = make_uint4(code[4 * q], code[4 * q + 1], code[4 * q + 2], code[4 * q + 3]);
+        *reinterpret_cast<uint32_t *>(a_sf + sf_tiled_offset(d, kw * 4, n_ksteps)) = sfw;
+      }
+    }
+  }
 }
 
 // ---- MXFP8 quantize (W4A8 activations): one thread per 32-element block ----
@@ -554,7 +586,8 @@ fp4_status fp4_moe_quantize_gather(const void *x_bf16, int64_t T, int32_t topk, 
                                    const int32_t *offsets, const int32_t *tile_offsets, const int32_t *inv,
                                    uint8_t *a_codes, uint8_t *a_sf, int64_t rows_cap, float *global_scale,
                                    void *workspace, size_t ws_bytes, uint32_t flags, fp4_stream_t stream) {
-  const bool mx = flags & FP4_MOE_MX;
+  const bool w4a8 = flags & FP4_MOE_W4A8;
+  const bool mx = (flags & FP4_MOE_MX) || w4a8;
   if (!x_bf16 || !offsets || !tile_offsets || !inv || !a_codes || !a_sf) return FP4_ERR_INVALID_ARG;
   if (!mx && (!global_scale || !workspace)) return FP4_ERR_INVALID_ARG;
   if (T < 0 || topk < 1 || topk > 16 || E < 1 || E > 4096 || H <= 0 || H % 64 || (mx && H % 128))
@@ -571,8 +604,12 @@ fp4_status fp4_moe_quantize_gather(const void *x_bf16, int64_t T, int32_t topk, 
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t need = (T + 3) / 4;  // four rows (warps) per CTA
     const int64_t grid = need < (int64_t)sms * 16 ? need : (int64_t)sms * 16;
-    mxfp4_quantize_gather_kernel<<<(unsigned)grid, 128, 0, s>>>(x, T, H, topk, E, offsets, tile_offsets, inv,
-                                                                 a_codes, a_sf);
+    if (w4a8)
+      mxfp8_quantize_gather_kernel<<<(unsigned)grid, 128, 0, s>>>(x, T, H, topk, E, offsets, tile_offsets, inv,
+                                                                   a_codes, a_sf);
+    else
+      mxfp4_quantize_gather_kernel<<<(unsigned)grid, 128, 0, s>>>(x, T, H, topk, E, offsets, tile_offsets, inv,
+                                                                   a_codes, a_sf);
     FP4_HOST_CHECK(cudaGetLastError());
     return FP4_OK;
   }

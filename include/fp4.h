@@ -80,6 +80,7 @@ typedef enum { FP4_OUT_F32 = 0, FP4_OUT_BF16 = 1 } fp4_out_dtype;
 #define FP4_MOE_PAIR_TILES 0x20u     /* MoE NVFP4 w13 / w2: CTA-pair tiles instead of 1-CTA row tiles */
 #define FP4_GEMM_A_MXFP8 0x40u       /* fp4_gemm: W4A8 -- A is MXFP8 (E4M3, UE8M0 per 32), B MXFP4 */
 #define FP4_GEMM_B_MXFP8 0x80u       /* fp4_gemm with FP4_GEMM_A_MXFP8: B is MXFP8 too */
+#define FP4_MOE_W4A8 0x100u          /* MoE layer / stages: MXFP4 weights, MXFP8 activations and h */
 
 /* Human-readable name of a status code (static string). */
 const char *fp4_status_string(fp4_status s);
@@ -201,6 +202,13 @@ fp4_status fp4_gemm(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_
  * are unused (may be NULL).  x is MXFP4-quantized (per 32-block power-of-two
  * scale, no tensor scale), h is re-quantized to MXFP4 per 32-element block in
  * the w13 epilogue, and y = w[t,s] * h_q.W2_e^T.
+ *
+ * W4A8 variant (flags FP4_MOE_W4A8) [QAT §4.3]: MXFP4 weights as for
+ * FP4_MOE_MX (w13_codes / w2_codes 32-byte aligned), with x and h in MXFP8
+ * (one E4M3 byte per element, UE8M0 per 32; fp4_quantize(FP4_MXFP8) rule);
+ * the grouped GEMMs run FP8 x FP4 on tcgen05 kind::mxf8f6f4.  The stage
+ * buffers of gathered x and h hold one byte per element
+ * (fp4_moe_workspace_size_flags).
  * ------------------------------------------------------------------------- */
 typedef struct {
   const uint8_t *w13_codes;
@@ -215,6 +223,9 @@ typedef struct {
 /* Workspace bytes for fp4_moe_grouped_gemm at these sizes (256-byte aligned
  * sub-buffers: header, quantized x, routing tables, gathered rows, h, y). */
 size_t fp4_moe_workspace_size(int64_t T, int32_t topk, int64_t H, int64_t I, int32_t E);
+/* The same for the layer flags that change it: FP4_MOE_W4A8 stores the
+ * gathered activations and h one byte per element. */
+size_t fp4_moe_workspace_size_flags(int64_t T, int32_t topk, int64_t H, int64_t I, int32_t E, uint32_t flags);
 
 /*
  * fp4_moe_grouped_gemm -- the whole routed-expert layer in one call:
@@ -223,7 +234,7 @@ size_t fp4_moe_workspace_size(int64_t T, int32_t topk, int64_t H, int64_t I, int
  * the top-k weight -> fixed-order combine to bf16.
  *   tokens_bf16  [T][H];  expert_ids int32 [T][topk];
  *   topk_weights fp32 [T][topk] or NULL (weights 1.0);  out_bf16 [T][H].
- *   workspace >= fp4_moe_workspace_size(...), 256-byte aligned.
+ *   workspace >= fp4_moe_workspace_size_flags(..., flags), 256-byte aligned.
  *   flags: FP4_DEBUG_DUMP_H needs h_dump (fp32, rows = padded routed rows,
  *   I columns); otherwise h_dump may be NULL.
  * Expert ids outside [0,E) set FP4_ERR_BAD_EXPERT in the device status; such
@@ -288,7 +299,9 @@ fp4_status fp4_moe_gather(const uint8_t *x_codes, const uint8_t *x_sf, int64_t T
  * from the routing tables of fp4_moe_route.  global_scale: device fp32[1],
  * output.  workspace >= fp4_quantize_workspace_size() bytes.
  * With FP4_MOE_MX: MXFP4 instead (UE8M0 per 32, tiled with 32-element blocks,
- * H % 128 == 0); global_scale and workspace are unused (may be NULL). */
+ * H % 128 == 0); global_scale and workspace are unused (may be NULL).
+ * With FP4_MOE_W4A8: MXFP8 (a_codes one E4M3 byte per element, [rows_cap][H]),
+ * otherwise as FP4_MOE_MX. */
 fp4_status fp4_moe_quantize_gather(const void *x_bf16, int64_t T, int32_t topk, int64_t H, int32_t E,
                                    const int32_t *offsets, const int32_t *tile_offsets, const int32_t *inv,
                                    uint8_t *a_codes, uint8_t *a_sf, int64_t rows_cap, float *global_scale,

@@ -35,7 +35,7 @@ def build(T, H, I, E, k, seed=0, zipf=0.0, h_g=1e-3, w_sigma=0.02, w_frac=0.005,
     w2 = synth.weights_bf16((E * H, I), w_sigma, w_frac, w_factor, seed=seed + 3, device=dev)
     c.w13_codes = torch.empty((E * 2 * I, H // 2), dtype=torch.uint8, device=dev)
     c.w2_codes = torch.empty((E * H, I // 2), dtype=torch.uint8, device=dev)
-    div = 2 if fmt == "mx" else 1  # MX: one scale per 32 elements
+    div = 2 if fmt in ("mx", "w4a8") else 1  # MX: one scale per 32 elements
     c.fmt = fmt
     c.w13_sf = torch.empty(fp4.fp4_sf_tiled_bytes(E * 2 * I, H) // div, dtype=torch.uint8, device=dev)
     c.w2_sf = torch.empty(fp4.fp4_sf_tiled_bytes(E * H, I) // div, dtype=torch.uint8, device=dev)
@@ -52,7 +52,7 @@ def build(T, H, I, E, k, seed=0, zipf=0.0, h_g=1e-3, w_sigma=0.02, w_frac=0.005,
                 codes[sl] = cc
                 sf[e * sfb:(e + 1) * sfb] = ss
                 g[e] = gg[0]
-            elif fmt == "mx":
+            elif fmt in ("mx", "w4a8"):  # MXFP4 weights (w4a8: with MXFP8 activations)
                 cc, ss = fp4.quantize_mx(wb[sl], tiled=True)
                 codes[sl] = cc
                 sf[e * sfb:(e + 1) * sfb] = ss
@@ -77,7 +77,7 @@ def oracle_expert_weights(c, e):
     I, H = c.I, c.H
     w13 = f32(c.w13_bf[e * 2 * I:(e + 1) * 2 * I])
     w2 = f32(c.w2_bf[e * H:(e + 1) * H])
-    if getattr(c, "fmt", "nv") == "mx":
+    if getattr(c, "fmt", "nv") in ("mx", "w4a8"):
         q13, q2 = Q.mxfp4_quantize(w13), Q.mxfp4_quantize(w2)
         w1, w3 = MO.deinterleave_w13(Q.mxfp4_dequantize(*q13))
         return w1, w3, Q.mxfp4_dequantize(*q2), q13, q2
@@ -89,6 +89,9 @@ def oracle_expert_weights(c, e):
 
 
 def oracle_x(c):
+    if getattr(c, "fmt", "nv") == "w4a8":
+        xq = Q.mxfp8_quantize(c.x_f32)
+        return xq, Q.mxfp8_dequantize(*xq)
     if getattr(c, "fmt", "nv") == "mx":
         xq = Q.mxfp4_quantize(c.x_f32)
         return xq, Q.mxfp4_dequantize(*xq)

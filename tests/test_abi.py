@@ -45,6 +45,10 @@ def test_status_strings_and_sizes():
     a = fp4.fp4_moe_workspace_size(64, 6, 7168, 2048, 384)
     assert a > 0 and fp4.fp4_moe_workspace_size(128, 6, 7168, 2048, 384) > a
     assert fp4.fp4_moe_route_scratch_bytes(98304, 384) == 96 * 384 * 4
+    # W4A8 keeps the gathered x and h one byte per element: a larger workspace; other flags change nothing
+    assert fp4.fp4_moe_workspace_size_flags(64, 6, 7168, 2048, 384, 0) == a
+    assert fp4.fp4_moe_workspace_size_flags(64, 6, 7168, 2048, 384, fp4.FP4_MOE_MX) == a
+    assert fp4.fp4_moe_workspace_size_flags(64, 6, 7168, 2048, 384, fp4.FP4_MOE_W4A8) > a
 
 
 def _fake(addr):

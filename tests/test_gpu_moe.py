@@ -531,3 +531,146 @@ def test_layer_end_to_end_mx(T, H, I, E, k, zipf):
     ok = (ulps <= 1) | (np.abs(got - ref) <= G.bf16_ulp(np.abs(ref)) + sl + k * 2.0**-24 * sum_abs)
     assert ok.all(), int((~ok).sum())
     print(f"MX layer T={T}: {float((ulps <= 1).mean()):.6f} of outputs within 1 bf16 ulp of the oracle")
+
+
+# ---- W4A8: MXFP4 weights, MXFP8 activations and h ("DeepSeek-V4 FP4 QAT" §4.3) ----
+
+def _mx8_scale_exp(amax):
+    """X = clamp(floor(log2 amax) - 8, -127, 127), 0 for amax == 0 (MXFP8)."""
+    a = np.asarray(amax, dtype=np.float32)
+    X = np.zeros(a.shape, dtype=np.int64)
+    nz = a > 0
+    X[nz] = np.clip(F.floor_log2_f32(a[nz]) - 8, -127, 127)
+    return X
+
+
+def _band_quantize_check_mx8(h_ref, tol, codes_gpu, sc_gpu):
+    """MXFP8 analogue of _band_quantize_check_mx (E4M3 elements)."""
+    n, cols = h_ref.shape
+    nb = cols // 32
+    lo = (h_ref - tol).astype(np.float32)
+    hi = (h_ref + tol).astype(np.float32)
+    c_mid, s_mid = Q.mxfp8_quantize(h_ref.astype(np.float32))
+    amax_lo = np.where(np.sign(lo) == np.sign(hi), np.minimum(np.abs(lo), np.abs(hi)), 0).reshape(n, nb, 32).max(2)
+    amax_hi = np.maximum(np.abs(lo), np.abs(hi)).reshape(n, nb, 32).max(2)
+    X_lo, X_hi = _mx8_scale_exp(amax_lo), _mx8_scale_exp(amax_hi)
+    X_gpu = sc_gpu.astype(np.int64) - 127
+    sc_ok = ((X_gpu >= X_lo) & (X_gpu <= X_hi)) | ((sc_gpu == 0) & (amax_lo == 0))
+    p = np.repeat(np.ldexp(1.0, -X_gpu), 32, axis=1)
+    v_lo = F.e4m3_decode(F.e4m3_encode((lo * p).astype(np.float32)))
+    v_hi = F.e4m3_decode(F.e4m3_encode((hi * p).astype(np.float32)))
+    v_gpu = F.e4m3_decode(codes_gpu)
+    el_ok = (v_gpu >= np.minimum(v_lo, v_hi)) & (v_gpu <= np.maximum(v_lo, v_hi))
+    stable = (X_lo == X_hi) & (v_lo == v_hi).reshape(n, nb, 32).all(2)
+    exact = (sc_gpu == s_mid) & (v_gpu == F.e4m3_decode(c_mid)).reshape(n, nb, 32).all(2)
+    ok = np.where(stable, exact, sc_ok & el_ok.reshape(n, nb, 32).all(2))
+    return int((~exact).sum()), int((~stable).sum()), ok
+
+
+@pytest.mark.parametrize("T,H,k,E", [(300, 1024, 4, 9), (1000, 7168, 6, 64)])
+def test_quantize_gather_w4a8_bit_exact(T, H, k, E):
+    fp4 = _lib()
+    x = synth.activations_bf16((T, H), seed=T + 7, device="cuda")
+    ids, _, _ = synth.router(T, E, k, seed=T + 8, zipf_s=1.1, device="cuda")
+    r = _route_gpu(ids, T, k, E)
+    cap = fp4.moe_rows_cap(T, k, E)
+    a_c = torch.zeros((cap, H), dtype=torch.uint8, device="cuda")
+    a_s = torch.zeros(fp4.fp4_sf_tiled_bytes(cap, H) // 2, dtype=torch.uint8, device="cuda")
+    fp4.fp4_moe_quantize_gather(x, T, k, H, E, r["offsets"], r["tile_offsets"], r["inv"], a_c, a_s, cap, None, None,
+                                fp4.FP4_MOE_W4A8)
+    counts, offsets, perm, inv = MO.route(ids.cpu().numpy(), E)
+    toff = _tile_offsets_ref(counts)
+    rc, rs = Q.mxfp8_quantize(x.float().cpu().numpy())
+    pad_rows = np.concatenate([toff[e] * 128 + np.arange(counts[e]) for e in range(E)]).astype(np.int64)
+    tokens = perm // k
+    assert np.array_equal(np_u8(a_c)[pad_rows], rc[tokens])
+    assert np.array_equal(LY.sf_from_mma(np_u8(a_s), cap, H, block=32)[pad_rows], rs[tokens])
+
+
+@pytest.mark.parametrize("T,H,I,E,k,zipf", [(200, 512, 256, 8, 2, 0.0), (700, 1024, 512, 6, 6, 1.1)])
+def test_w13_swiglu_requant_w4a8(T, H, I, E, k, zipf):
+    fp4 = _lib()
+    c = moe_case.build(T, H, I, E, k, seed=T + 17, zipf=zipf, fmt="w4a8")
+    r = _route_gpu(c.ids, T, k, E)
+    cap = fp4.moe_rows_cap(T, k, E)
+    a_c = torch.empty((cap, H), dtype=torch.uint8, device="cuda")
+    a_s = torch.empty(fp4.fp4_sf_tiled_bytes(cap, H) // 2, dtype=torch.uint8, device="cuda")
+    fp4.fp4_moe_quantize_gather(c.x, T, k, H, E, r["offsets"], r["tile_offsets"], r["inv"], a_c, a_s, cap, None, None,
+                                fp4.FP4_MOE_W4A8)
+    h_c = torch.zeros((cap, I), dtype=torch.uint8, device="cuda")
+    h_s = torch.zeros(fp4.fp4_sf_tiled_bytes(cap, I) // 2, dtype=torch.uint8, device="cuda")
+    h_d = torch.zeros((cap, I), dtype=torch.float32, device="cuda")
+    fp4.fp4_moe_w13(a_c, a_s, None, c.weights, H, I, E, r["counts"], r["tile_offsets"], cap, h_c, h_s,
+                    fp4.FP4_DEBUG_DUMP_H | fp4.FP4_MOE_W4A8, h_d)
+    assert fp4.fp4_get_device_status() == 0
+    counts, offsets, perm, inv = MO.route(c.ids_np, E)
+    toff = _tile_offsets_ref(counts)
+    (xq, x_dq) = moe_case.oracle_x(c)
+    h_dump = h_d.cpu().numpy()
+    h_codes = np_u8(h_c)
+    h_sc = LY.sf_from_mma(np_u8(h_s), cap, I, block=32)
+    total_diff = 0
+    for e in range(E):
+        if counts[e] == 0:
+            continue
+        w1, w3, _, _, _ = moe_case.oracle_expert_weights(c, e)
+        xr = x_dq[perm[offsets[e]:offsets[e + 1]] // k]
+        gate, up = xr @ w1.T, xr @ w3.T
+        h = MO.swiglu(gate, up)
+        tol = _h_tol(xr, w1, w3, gate, up, h)
+        prow = toff[e] * 128 + np.arange(counts[e])
+        err = np.abs(h_dump[prow] - h)
+        assert np.all(err <= tol), (e, float((err / tol).max()))
+        n_diff, n_band, ok = _band_quantize_check_mx8(h, tol, h_codes[prow], h_sc[prow])
+        assert ok.all(), (e, int((~ok).sum()))
+        total_diff += n_diff
+    # E4M3 has 8x finer steps than E2M1, so more blocks sit near a rounding boundary
+    assert total_diff <= 0.05 * (T * k * I // 32) + 8, total_diff
+
+
+@pytest.mark.parametrize("T,H,I,E,k,zipf", [(256, 512, 256, 8, 2, 0.0), (1000, 1024, 512, 16, 6, 1.1)])
+def test_layer_end_to_end_w4a8(T, H, I, E, k, zipf):
+    """fp4_moe_grouped_gemm with FP4_MOE_W4A8 against the oracle's W4A8 layer
+    (MXFP8 x, MXFP4 weights, MXFP8 h).  An h block that is unstable within
+    the w13 error band may move each of its elements by up to twice the
+    largest MXFP8 error at the band's top scale (64 * 2^(X_hi + 1) each side)."""
+    fp4 = _lib()
+    c = moe_case.build(T, H, I, E, k, seed=T + 19, zipf=zipf, fmt="w4a8")
+    out = fp4.moe_layer(c.x, c.ids, c.w, c.weights, H, I, E, w4a8=True)
+    assert fp4.fp4_get_device_status() == 0
+    counts, offsets, perm, inv = MO.route(c.ids_np, E)
+    (xq, x_dq) = moe_case.oracle_x(c)
+    y = np.zeros((T * k, H))
+    slack = np.zeros((T * k, H))
+    for e in range(E):
+        if counts[e] == 0:
+            continue
+        w1, w3, w2, _, _ = moe_case.oracle_expert_weights(c, e)
+        rr = slice(offsets[e], offsets[e + 1])
+        xr = x_dq[perm[rr] // k]
+        gate, up = xr @ w1.T, xr @ w3.T
+        h = MO.swiglu(gate, up)
+        tol = _h_tol(xr, w1, w3, gate, up, h)
+        hc, hs = Q.mxfp8_quantize(h.astype(np.float32))
+        h_dq = Q.mxfp8_dequantize(hc, hs)
+        wt = c.w_np.reshape(-1)[perm[rr]].astype(np.float64)[:, None]
+        y[rr] = wt * (h_dq @ w2.T)
+        n = len(h)
+        amax_hi = (np.abs(h) + tol).reshape(n, -1, 32).max(2).astype(np.float32)
+        s_top = np.ldexp(1.0, _mx8_scale_exp(amax_hi) + 1)
+        lo, hi = (h - tol).astype(np.float32), (h + tol).astype(np.float32)
+        c_lo, s_lo = Q.mxfp8_quantize(lo)
+        c_hi, s_hi = Q.mxfp8_quantize(hi)
+        unstable = ~((s_lo == hs) & (s_hi == hs) & (c_lo == hc).reshape(n, -1, 32).all(2) &
+                     (c_hi == hc).reshape(n, -1, 32).all(2))
+        dh = np.repeat(np.where(unstable, 2 * 64.0 * s_top, 0.0), 32, axis=1) + (np.repeat(unstable, 32, axis=1) * tol)
+        slack[rr] = wt * (dh @ np.abs(w2).T) + G.FP32_REL_TOL * wt * (np.abs(h_dq) @ np.abs(w2).T)
+    ref, ref_bits = MO.combine_ref(y, inv)
+    sl = sum(slack[inv[:, s]] for s in range(k))
+    sum_abs = sum(np.abs(y[inv[:, s]]) for s in range(k))
+    got_bits = bf16_bits(out)
+    got = F.bf16_bits_to_f32(got_bits).astype(np.float64)
+    ulps = bf16_ulps_apart(got_bits, ref_bits)
+    ok = (ulps <= 1) | (np.abs(got - ref) <= G.bf16_ulp(np.abs(ref)) + sl + k * 2.0**-24 * sum_abs)
+    assert ok.all(), int((~ok).sum())
+    print(f"W4A8 layer T={T}: {float((ulps <= 1).mean()):.6f} of outputs within 1 bf16 ulp of the oracle")
