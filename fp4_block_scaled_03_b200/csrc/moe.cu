@@ -65,9 +65,11 @@ fp4_status fp4_moe_grouped_gemm(const void *tokens_bf16, const int32_t *expert_i
                                 int64_t T, int32_t topk, const fp4_moe_weights *w, int64_t H, int64_t I, int32_t E,
                                 void *out_bf16, void *workspace, size_t ws_bytes, uint32_t flags, float *h_dump,
                                 fp4_stream_t stream) {
-  if (!tokens_bf16 || !expert_ids || !w || !out_bf16 || !workspace) return FP4_ERR_INVALID_ARG;
+  if (!w || !workspace) return FP4_ERR_INVALID_ARG;
   if (T < 0 || topk < 1 || topk > 16 || E < 1 || E > 4096) return FP4_ERR_UNSUPPORTED_SHAPE;
   if (H < 256 || H % 256 || I < 256 || I % 256) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return FP4_OK;  // empty batch: no work, token / id / output pointers may be NULL
+  if (!tokens_bf16 || !expert_ids || !out_bf16) return FP4_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(workspace) & 255u) return FP4_ERR_ALIGNMENT;
   const MoeLayout L = moe_layout(T, topk, H, I, E, (flags & FP4_MOE_W4A8) ? 1 : 2);
   if (ws_bytes < L.total) return FP4_ERR_WORKSPACE;

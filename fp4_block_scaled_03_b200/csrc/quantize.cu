@@ -489,8 +489,10 @@ extern "C" {
 fp4_status fp4_quantize(fp4_format fmt, const void *x_bf16, int64_t rows, int64_t cols, int64_t ld, uint8_t *codes,
                         uint8_t *scales, float *global_scale, uint32_t flags, void *workspace, size_t ws_bytes,
                         fp4_stream_t stream) {
-  if (!x_bf16 || !codes || !scales || rows < 0 || cols <= 0 || ld < cols) return FP4_ERR_INVALID_ARG;
+  if (rows < 0 || cols <= 0 || ld < cols) return FP4_ERR_INVALID_ARG;
   if (fmt != FP4_NV && fmt != FP4_MX && fmt != FP4_MXFP8) return FP4_ERR_INVALID_ARG;
+  if (rows == 0) return FP4_OK;  // empty input: no work, row pointers may be NULL
+  if (!x_bf16 || !codes || !scales) return FP4_ERR_INVALID_ARG;
   if (!aligned16(x_bf16) || !aligned16(codes) || (ld * 2) % 16) return FP4_ERR_ALIGNMENT;
   const DeviceCtx *ctx = device_ctx();
   if (!ctx) return FP4_ERR_CUDA;
@@ -588,6 +590,7 @@ fp4_status fp4_moe_quantize_gather(const void *x_bf16, int64_t T, int32_t topk, 
                                    void *workspace, size_t ws_bytes, uint32_t flags, fp4_stream_t stream) {
   const bool w4a8 = flags & FP4_MOE_W4A8;
   const bool mx = (flags & FP4_MOE_MX) || w4a8;
+  if (T == 0 && topk >= 1 && topk <= 16 && E >= 1 && E <= 4096 && H > 0) return FP4_OK;  // empty batch
   if (!x_bf16 || !offsets || !tile_offsets || !inv || !a_codes || !a_sf) return FP4_ERR_INVALID_ARG;
   if (!mx && (!global_scale || !workspace)) return FP4_ERR_INVALID_ARG;
   if (T < 0 || topk < 1 || topk > 16 || E < 1 || E > 4096 || H <= 0 || H % 64 || (mx && H % 128))

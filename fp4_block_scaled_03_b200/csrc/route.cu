@@ -309,9 +309,11 @@ size_t fp4_moe_route_scratch_bytes(int64_t R, int32_t E) {
 fp4_status fp4_moe_route(const int32_t *expert_ids, int64_t T, int32_t topk, int32_t E, int32_t *counts,
                          int32_t *offsets, int32_t *tile_offsets, int32_t *perm, int32_t *inv, void *scratch,
                          size_t scratch_bytes, fp4_stream_t stream) {
-  if (!expert_ids || !counts || !offsets || !tile_offsets || !perm || !inv || !scratch) return FP4_ERR_INVALID_ARG;
+  if (!counts || !offsets || !tile_offsets || !scratch) return FP4_ERR_INVALID_ARG;
   if (T < 0 || topk < 1 || topk > 16 || E < 1 || E > 4096) return FP4_ERR_UNSUPPORTED_SHAPE;
   const int64_t R = T * topk;
+  // an empty batch still writes zero counts and offsets; its row arrays may be NULL
+  if (R > 0 && (!expert_ids || !perm || !inv)) return FP4_ERR_INVALID_ARG;
   if (R > 2147483647LL / 2) return FP4_ERR_UNSUPPORTED_SHAPE;
   if (scratch_bytes < fp4_moe_route_scratch_bytes(R, E)) return FP4_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(scratch) & 3u)) return FP4_ERR_ALIGNMENT;
@@ -336,9 +338,9 @@ fp4_status fp4_moe_route(const int32_t *expert_ids, int64_t T, int32_t topk, int
 
 fp4_status fp4_moe_topk(const float *logits, int64_t T, int32_t E, int32_t topk, int32_t *expert_ids,
                         float *topk_weights, fp4_stream_t stream) {
-  if (!logits || !expert_ids || !topk_weights) return FP4_ERR_INVALID_ARG;
   if (T < 0 || E < 1 || E > 65536 || topk < 1 || topk > 16 || topk > E) return FP4_ERR_UNSUPPORTED_SHAPE;
-  if (T == 0) return FP4_OK;
+  if (T == 0) return FP4_OK;  // empty batch: pointers may be NULL
+  if (!logits || !expert_ids || !topk_weights) return FP4_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   int64_t grid = (T + 7) / 8;
   const int64_t cap = (int64_t)sm_count() * 16;
@@ -351,8 +353,9 @@ fp4_status fp4_moe_topk(const float *logits, int64_t T, int32_t E, int32_t topk,
 fp4_status fp4_moe_gather(const uint8_t *x_codes, const uint8_t *x_sf, int64_t T, int32_t topk, int64_t H,
                           int32_t E, const int32_t *offsets, const int32_t *tile_offsets, const int32_t *perm,
                           uint8_t *a_codes, uint8_t *a_sf, int64_t rows_cap, fp4_stream_t stream) {
-  if (!x_codes || !x_sf || !offsets || !tile_offsets || !perm || !a_codes || !a_sf) return FP4_ERR_INVALID_ARG;
   if (T < 0 || topk < 1 || topk > 16 || E < 1 || E > 4096 || H <= 0 || H % 64) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return FP4_OK;  // empty batch: pointers may be NULL
+  if (!x_codes || !x_sf || !offsets || !tile_offsets || !perm || !a_codes || !a_sf) return FP4_ERR_INVALID_ARG;
   if (rows_cap < T * topk + 127LL * E) return FP4_ERR_WORKSPACE;
   if (!al16(x_codes) || !al16(a_codes) || (reinterpret_cast<uintptr_t>(x_sf) & 3u) ||
       (reinterpret_cast<uintptr_t>(a_sf) & 3u))
@@ -372,8 +375,9 @@ fp4_status fp4_moe_gather(const uint8_t *x_codes, const uint8_t *x_sf, int64_t T
 
 fp4_status fp4_moe_combine(const float *y, const int32_t *inv, int64_t T, int32_t topk, int64_t H, void *out_bf16,
                            fp4_stream_t stream) {
-  if (!y || !inv || !out_bf16) return FP4_ERR_INVALID_ARG;
   if (T < 0 || topk < 1 || topk > 16 || H <= 0 || H % 16) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return FP4_OK;  // empty batch: pointers may be NULL
+  if (!y || !inv || !out_bf16) return FP4_ERR_INVALID_ARG;
   if (!al16(y) || !al16(out_bf16)) return FP4_ERR_ALIGNMENT;
   if (T == 0) return FP4_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

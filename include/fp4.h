@@ -67,6 +67,10 @@ typedef enum {
   FP4_ERR_CUDA = 8               /* a CUDA runtime/driver call failed */
 } fp4_status;
 
+/* Empty inputs: a call whose row or token count (rows, T) is 0 does no work
+ * and returns FP4_OK (fp4_moe_route still writes zero counts and offsets);
+ * the pointers to its row arrays may then be NULL.  Other arguments are
+ * still checked. */
 typedef enum { FP4_NV = 0, FP4_MX = 1, FP4_MXFP8 = 2 } fp4_format;
 
 typedef enum { FP4_OUT_F32 = 0, FP4_OUT_BF16 = 1 } fp4_out_dtype;

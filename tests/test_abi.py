@@ -95,6 +95,26 @@ def test_host_validation_without_gpu():
     assert L.fp4_gemm(A, A, None, A + 16, A, None, A, 0, 128, 256, 512, 0x40, None) == 2
 
 
+def test_empty_inputs_do_no_work_with_null_row_pointers():
+    """rows / T == 0: FP4_OK without touching the row arrays (NULL here) and
+    without a CUDA call, so it holds on a host with no GPU too."""
+    import fp4_block_scaled_03_b200 as fp4
+
+    L = fp4.lib
+    A = 0x10000
+    assert L.fp4_quantize(0, None, 0, 64, 64, None, None, None, 0, None, 0, None) == 0
+    assert L.fp4_moe_combine(None, None, 0, 6, 512, None, None) == 0
+    assert L.fp4_moe_topk(None, 0, 64, 6, None, None, None) == 0
+    assert L.fp4_moe_gather(None, None, 0, 2, 256, 4, None, None, None, None, None, 0, None) == 0
+    assert L.fp4_moe_quantize_gather(None, 0, 2, 256, 4, None, None, None, None, None, 0, None, None, 0, 0, None) == 0
+    w = fp4.MoeWeights(A, A, A, A, A, A, A)
+    assert L.fp4_moe_grouped_gemm(None, None, None, 0, 2, ctypes.byref(w), 256, 256, 4, None, A, 1 << 20, 0, None,
+                                  None) == 0
+    # the shape and the layer's own arguments are still checked
+    assert L.fp4_moe_grouped_gemm(None, None, None, 0, 2, None, 256, 256, 4, None, A, 1 << 20, 0, None, None) == 1
+    assert L.fp4_moe_combine(None, None, 0, 6, 500, None, None) == 3
+
+
 def test_package_fails_loudly_without_library(tmp_path, monkeypatch):
     """Importing the binding from a copy without libfp4.so raises (no fallback)."""
     import importlib.util

@@ -1,0 +1,55 @@
+"""Degenerate and extreme MoE inputs against the oracle: an empty batch, one
+expert with top-1, the largest expert count the ABI takes (4096), and every
+token routed to one expert (many 128-row tiles / 256-row chunks of one
+expert).  The value checks are the layer and stage checks of
+test_gpu_moe."""
+import numpy as np
+import pytest
+import torch
+
+from tests import moe_case
+from tests import test_gpu_moe as TM
+
+pytestmark = pytest.mark.gpu
+
+
+def test_route_empty_batch_writes_zero_tables():
+    import fp4_block_scaled_03_b200 as fp4
+
+    E = 7
+    counts = torch.full((E,), -1, dtype=torch.int32, device="cuda")
+    offsets = torch.full((E + 1,), -1, dtype=torch.int32, device="cuda")
+    toffs = torch.full((E + 1,), -1, dtype=torch.int32, device="cuda")
+    scratch = torch.empty(256, dtype=torch.uint8, device="cuda")
+    empty = torch.empty(0, dtype=torch.int32, device="cuda")
+    fp4.fp4_moe_route(empty, 0, 2, E, counts, offsets, toffs, empty, empty, scratch)
+    assert fp4.fp4_get_device_status() == 0
+    assert counts.abs().sum().item() == 0 and offsets.abs().sum().item() == 0 and toffs.abs().sum().item() == 0
+
+
+def test_layer_empty_batch():
+    import fp4_block_scaled_03_b200 as fp4
+
+    c = moe_case.build(8, 512, 256, 4, 2, seed=1)
+    x = c.x[:0]
+    out = fp4.moe_layer(x, c.ids[:0], c.w[:0], c.weights, 512, 256, 4)
+    assert out.shape == (0, 512)
+    assert fp4.fp4_get_device_status() == 0
+
+
+@pytest.mark.parametrize("tiling", TM.TILINGS)
+def test_layer_single_expert_top1(tiling):
+    TM.test_layer_end_to_end(300, 512, 256, 1, 1, 0.0, tiling)
+
+
+def test_layer_max_experts():
+    """E = 4096 (the ABI's limit): 64 tokens x top-6 touch a few hundred
+    experts; every other expert has no rows and no tiles."""
+    TM.test_layer_end_to_end(64, 512, 256, 4096, 6, 1.1, "rows")
+
+
+@pytest.mark.parametrize("tiling", TM.TILINGS)
+def test_all_tokens_on_one_expert(tiling):
+    c = moe_case.build(1000, 512, 256, 8, 1, seed=3, counts=[0, 0, 1000, 0, 0, 0, 0, 0])
+    TM._check_w13(c, tiling)
+    TM._check_w2(c, tiling)
