@@ -1,7 +1,8 @@
 """Benchmark of the NVFP4 W4A4 routed-expert hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W]
-                    [--workload pro|flash|flashmx|decode|pro64|dense4096|dense4096mx|dense4096w4a8|quant]
+                    [--workload pro|flash|flashmx|flashw4a8|decode|pro64|dense4096|dense4096mx|dense4096w4a8|
+                                router|quant]
                     [--impl fp4|reference]
 
 A step is one pass of the whole hot path over one synthetic batch: dynamic
@@ -643,6 +644,71 @@ def run_dense(args, world, rank, peaks, mx=False, w4a8=False):
     }
 
 
+def run_router(args, world, rank, peaks):
+    """Router at the Pro shape: bf16 gate GEMM (16384 x 7168 -> 384 logits, tcgen05
+    kind::f16) + top-6 softmax, one fp4_moe_router call per step."""
+    import torch
+
+    import fp4_block_scaled_03_b200 as fp4
+    import synth
+
+    T, H, E, k = 16384, 7168, 384, 6
+    x = synth.activations_bf16((T, H), seed=rank, device="cuda")
+    wg = synth.weights_bf16((E, H), 0.02, 0.0, 1.0, seed=rank + 1, device="cuda")
+    logits = torch.empty((T, E), dtype=torch.float32, device="cuda")
+    ids = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+
+    def step(ev=None):
+        if ev:
+            ev[0].record()
+        fp4.fp4_gemm_bf16(x, wg, logits, T, E, H)
+        if ev:
+            ev[1].record()
+        fp4.fp4_moe_topk(logits, T, E, k, ids, w)
+        if ev:
+            ev[2].record()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    barrier(world)
+    g = tk = tot = 0.0
+    for i in range(args.steps):
+        flush.zero_()
+        torch.cuda.synchronize()
+        step(evs[i])
+        torch.cuda.synchronize()
+        g += evs[i][0].elapsed_time(evs[i][1])
+        tk += evs[i][1].elapsed_time(evs[i][2])
+        tot += evs[i][0].elapsed_time(evs[i][2])
+    clocks = sampler.stop() if sampler else None
+    ms = max_over_ranks(tot / args.steps, world)
+    gms = g / args.steps
+    flops = 2.0 * T * E * H
+    peak = peaks["bf16"]
+    return {
+        "metric": METRIC, "value": round(world * flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16 (gate GEMM, fp32 accumulate) + fp32 top-k softmax",
+        "data": "synthetic (seeded)",
+        "config": {"workload": "Router at the Pro shape: 16384 tokens x hidden 7168 -> 384 expert logits, top-6",
+                   "l2": "flushed (256 MB write) before each timed step"},
+        "roofline": {"bound": "tensor", "kernel": "fp4_gemm_kernel<256, f32, bf16>",
+                     "achieved": round(flops / (gms * 1e-3) / 1e12, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
+                     "frac": round(flops / (gms * 1e-3) / 1e12 / peak, 4), "traffic": None,
+                     "peak_note": "measured burst bf16 cuBLAS, of " + peaks["src"]},
+        "stages_ms": {"gate_gemm": round(gms, 4), "topk": round(tk / args.steps, 4)},
+        "gpu_launches": 2 * args.steps, "clocks": clocks,
+    }
+
+
 def run_quant(args, world, rank, peaks):
     import torch
 
@@ -739,7 +805,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="pro", choices=list(WORKLOADS) + ["dense4096", "dense4096mx", "dense4096w4a8", "quant"])
+    ap.add_argument("--workload", default="pro", choices=list(WORKLOADS) + ["dense4096", "dense4096mx", "dense4096w4a8", "router", "quant"])
     ap.add_argument("--impl", default="fp4", choices=["fp4", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--pair-tiles", action="store_true",
@@ -765,6 +831,8 @@ def main():
     elif args.workload in ("dense4096", "dense4096mx", "dense4096w4a8"):
         line = run_dense(args, world, rank, peaks, mx=args.workload.endswith("mx"),
                          w4a8=args.workload.endswith("w4a8"))
+    elif args.workload == "router":
+        line = run_router(args, world, rank, peaks)
     else:
         line = run_quant(args, world, rank, peaks)
     if rank == 0 and line is not None:

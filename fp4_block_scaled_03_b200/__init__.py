@@ -80,6 +80,8 @@ _SIGS = {
     "fp4_quantize": (ctypes.c_int, [ctypes.c_int, _P, _I64, _I64, _I64, _P, _P, _P, _U32, _P, _SZ, _P]),
     "fp4_mx_to_nv": (ctypes.c_int, [_P, _P, _I64, _I64, _I64, _P, _P, _U32, _P]),
     "fp4_e2m1_to_e4m3": (ctypes.c_int, [_P, _I64, _I64, _P, _P]),
+    "fp4_gemm_bf16": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _I64, _P]),
+    "fp4_moe_router": (ctypes.c_int, [_P, _I64, _I64, _P, _I32, _I32, _P, _P, _P, _P]),
     "fp4_gemm": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, ctypes.c_int, _I64, _I64, _I64, _U32, _P]),
     "fp4_moe_workspace_size": (_SZ, [_I64, _I32, _I64, _I64, _I32]),
     "fp4_moe_workspace_size_flags": (_SZ, [_I64, _I32, _I64, _I64, _I32, _U32]),
@@ -146,6 +148,15 @@ def fp4_mx_to_nv(codes, mx_scales, rows, cols, num_tensors, nv_scales, nv_global
 
 def fp4_e2m1_to_e4m3(codes_e2m1, rows, cols, codes_e4m3):
     _check(lib.fp4_e2m1_to_e4m3(_ptr(codes_e2m1), rows, cols, _ptr(codes_e4m3), _stream()), "fp4_e2m1_to_e4m3")
+
+
+def fp4_gemm_bf16(a, b, c, M, N, K):
+    _check(lib.fp4_gemm_bf16(_ptr(a), _ptr(b), _ptr(c), M, N, K, _stream()), "fp4_gemm_bf16")
+
+
+def fp4_moe_router(x, T, H, gate_w, E, topk, logits, expert_ids, topk_weights):
+    _check(lib.fp4_moe_router(_ptr(x), T, H, _ptr(gate_w), E, topk, _ptr(logits), _ptr(expert_ids),
+                              _ptr(topk_weights), _stream()), "fp4_moe_router")
 
 
 def fp4_gemm(a_codes, a_sf, a_g, b_codes, b_sf, b_g, c, c_dtype, M, N, K, flags=0):
@@ -313,6 +324,26 @@ def gemm(a_codes, a_sf, a_g, b_codes, b_sf, b_g, M, N, K, out_dtype=torch.float3
     fp4_gemm(a_codes, a_sf, a_g, b_codes, b_sf, b_g, c, FP4_OUT_F32 if out_dtype == torch.float32 else FP4_OUT_BF16,
              M, N, K, flags)
     return c
+
+
+def gemm_bf16(a, b):
+    """fp32 a [M,K] . b [N,K]^T for bf16 a, b."""
+    M, K = a.shape
+    N = b.shape[0]
+    c = torch.empty((M, N), dtype=torch.float32, device=a.device)
+    fp4_gemm_bf16(a, b, c, M, N, K)
+    return c
+
+
+def router(x, gate_w, topk):
+    """Gate projection + top-k: (logits fp32 [T,E], expert_ids int32 [T,k], weights fp32 [T,k])."""
+    T, H = x.shape
+    E = gate_w.shape[0]
+    logits = torch.empty((T, E), dtype=torch.float32, device=x.device)
+    ids = torch.empty((T, topk), dtype=torch.int32, device=x.device)
+    w = torch.empty((T, topk), dtype=torch.float32, device=x.device)
+    fp4_moe_router(x, T, H, gate_w, E, topk, logits, ids, w)
+    return logits, ids, w
 
 
 class MoeWeightSet:

@@ -153,7 +153,8 @@ __device__ __forceinline__ TileInfo tile_info(const Params &p, int t) {
 
 // KIND: 0 NVFP4 x NVFP4 (kind::mxf4nvf4, E4M3 scale per 16); 1 MXFP4 x MXFP4
 // (kind::mxf4, UE8M0 per 32); 2 W4A8, MXFP8 A x MXFP4 or MXFP8 B
-// (kind::mxf8f6f4, UE8M0 per 32, 128 K-elements per stage).
+// (kind::mxf8f6f4, UE8M0 per 32, 128 K-elements per stage); 3 bf16 x bf16
+// (kind::f16, no block scales, 64 K-elements per stage; the router's gate GEMM).
 template <int BN, int EPI, int KIND>
 __global__ void __launch_bounds__(kThreads, 1)
     fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -164,6 +165,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // scale words (512-byte tiles) per 128-row slab per stage: one per K step of
   // 64 (NVFP4), per two K steps (MXFP4), or one for the stage's 4 x 32 (W4A8)
   constexpr int WPS = KIND == 0 ? 4 : KIND == 1 ? 2 : 1;
+  constexpr bool kScaled = KIND != 3;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *smA = smem;
@@ -227,17 +229,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kt = 0; kt < p.k_stages; ++kt) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, &s_abort, p.status, lim)) { ok = false; break; }
           const int nk = min(4, p.kw - kt * 4);
-          const int nw = KIND == 0 ? nk : KIND == 1 ? (nk + 1) / 2 : 1;  // scale words this stage
+          const int nw = !kScaled ? 0 : KIND == 0 ? nk : KIND == 1 ? (nk + 1) / 2 : 1;  // scale words this stage
           const uint32_t sf_bytes = (uint32_t)nw * 512u;
           int halves = 0;
-          for (int h = 0; h < C::HALVES; ++h)
+          for (int h = 0; h < C::HALVES && kScaled; ++h)
             if ((int64_t)(b_slab0 + h) * 128 < p.b_sf_rows) ++halves;
           const uint32_t bytes = C::A_BYTES + (KIND == 2 ? p.b_tx : (uint32_t)C::B_BYTES) + sf_bytes * (1 + halves);
           mbar_arrive_expect_tx(&full[stage], bytes);
           tma_load_2d(smA + stage * C::A_BYTES, &tmA, &full[stage], kt * BK_BYTES, ti.a_row0);
           tma_load_2d(smB + stage * C::B_BYTES, &tmB, &full[stage], kt * BK_BYTES, ti.b_row0);
-          bulk_load(smSFA + stage * C::SFA_BYTES, p.a_sf + ((int64_t)ti.a_slab * p.kw_sf + kt * WPS) * 512, sf_bytes,
-                    &full[stage]);
+          if (kScaled)
+            bulk_load(smSFA + stage * C::SFA_BYTES, p.a_sf + ((int64_t)ti.a_slab * p.kw_sf + kt * WPS) * 512,
+                      sf_bytes, &full[stage]);
           for (int h = 0; h < halves; ++h)
             bulk_load(smSFB + stage * C::SFB_BYTES + h * WPS * 512,
                       p.b_sf + ((int64_t)(b_slab0 + h) * p.kw_sf + kt * WPS) * 512, sf_bytes, &full[stage]);
@@ -253,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 2) {
     // ------------------------------------------------------------ scale copier
-    if (lane == 0) {
+    if (lane == 0 && kScaled) {
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true, any = false;
@@ -290,9 +293,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = KIND == 0 ? idesc_mxf4nvf4(BM, BN)
+      const uint32_t idesc = KIND == 0   ? idesc_mxf4nvf4(BM, BN)
                              : KIND == 1 ? idesc_mxf4(BM, BN)
-                                         : idesc_mxf8f6f4(BM, BN, 0u /*E4M3*/, (uint32_t)p.b_fmt);
+                             : KIND == 2 ? idesc_mxf8f6f4(BM, BN, 0u /*E4M3*/, (uint32_t)p.b_fmt)
+                                         : idesc_bf16(BM, BN);
       int stage = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true, any_mma = false;
@@ -302,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         for (int kt = 0; kt < p.k_stages; ++kt) {
           if (!mbar_wait(&full[stage], phase, &s_abort, p.status, lim)) { ok = false; break; }
-          if (!mbar_wait(&sf_full[stage], phase, &s_abort, p.status, lim)) { ok = false; break; }
+          if (kScaled && !mbar_wait(&sf_full[stage], phase, &s_abort, p.status, lim)) { ok = false; break; }
           tc_fence_after();
           const int nk = min(4, p.kw - kt * 4);
           const uint32_t ta = tmem + C::SF_COL0 + stage * C::SF_SLOT_COLS;
@@ -313,7 +317,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             if (j < nk) {
-              if (KIND == 2) {  // K step j (32 elements): byte j of the stage's scale word
+              if (KIND == 3) {  // K step j: 16 bf16 elements, +32 bytes
+                mma_bf16(t_acc, ad + (uint64_t)(j * 2), bd + (uint64_t)(j * 2), idesc, (kt > 0 || j > 0) ? 1u : 0u);
+              } else if (KIND == 2) {  // K step j (32 elements): byte j of the stage's scale word
                 const uint32_t byte = (uint32_t)j;
                 mma_mxf8f6f4(t_acc, ad + (uint64_t)(j * 2), bd + (uint64_t)(j * 2), idesc | (byte << 29) | (byte << 4),
                              ta | (byte << 30), tb | (byte << 30), (kt > 0 || j > 0) ? 1u : 0u);
@@ -580,6 +586,32 @@ fp4_status fp4_gemm(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_
   }
   if (c_dtype == FP4_OUT_F32) return launch<kBN, EPI_F32>(ta, tb, tb, p, grid, s);
   return launch<kBN, EPI_BF16>(ta, tb, tb, p, grid, s);
+}
+
+fp4_status fp4_gemm_bf16(const void *a_bf16, const void *b_bf16, float *c, int64_t M, int64_t N, int64_t K,
+                         fp4_stream_t stream) {
+  if (!a_bf16 || !b_bf16 || !c) return FP4_ERR_INVALID_ARG;
+  if (M < 1 || N < 1 || K < 64 || K % 64 || N % 8) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (M > (1LL << 30) || N > (1LL << 30) || K > (1LL << 30)) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (!al16(a_bf16) || !al16(b_bf16) || !al16(c)) return FP4_ERR_ALIGNMENT;
+  const DeviceCtx *ctx = device_ctx();
+  if (!ctx) return FP4_ERR_CUDA;
+  CUtensorMap ta, tb;  // bf16 rows viewed as bytes: 128-byte swizzle rows of 64 elements
+  if (!make_code_map(&ta, a_bf16, (uint64_t)M, (uint64_t)K * 2, BM)) return FP4_ERR_CUDA;
+  if (!make_code_map(&tb, b_bf16, (uint64_t)N, (uint64_t)K * 2, kBN)) return FP4_ERR_CUDA;
+  Params p = {};
+  p.M = (int)M; p.N = (int)N; p.K = (int)K;
+  p.n_tiles = (int)((N + kBN - 1) / kBN);
+  p.m_tiles = (int)((M + BM - 1) / BM);
+  p.k_stages = (int)(K / 64);
+  p.kw = (int)(K / 16);  // MMA K steps of 16 elements
+  p.c = c;
+  p.status = ctx->status;
+  p.wait_limit = ctx->wait_limit_ns;
+  const int64_t tiles = (int64_t)p.m_tiles * p.n_tiles;
+  if (tiles > 2147483647LL) return FP4_ERR_UNSUPPORTED_SHAPE;
+  const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
+  return launch<kBN, EPI_F32, 3>(ta, tb, tb, p, grid, reinterpret_cast<cudaStream_t>(stream));
 }
 
 fp4_status fp4_moe_w13(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_g, const fp4_moe_weights *w,

@@ -350,6 +350,17 @@ fp4_status fp4_moe_topk(const float *logits, int64_t T, int32_t E, int32_t topk,
   return FP4_OK;
 }
 
+fp4_status fp4_moe_router(const void *x_bf16, int64_t T, int64_t H, const void *gate_w_bf16, int32_t E,
+                          int32_t topk, float *logits, int32_t *expert_ids, float *topk_weights, fp4_stream_t stream) {
+  if (T < 0 || H < 64 || H % 64 || E < 8 || E % 8 || E > 65536 || topk < 1 || topk > 16 || topk > E)
+    return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return FP4_OK;  // empty batch: pointers may be NULL
+  if (!x_bf16 || !gate_w_bf16 || !logits || !expert_ids || !topk_weights) return FP4_ERR_INVALID_ARG;
+  const fp4_status st = fp4_gemm_bf16(x_bf16, gate_w_bf16, logits, T, E, H, stream);
+  if (st != FP4_OK) return st;
+  return fp4_moe_topk(logits, T, E, topk, expert_ids, topk_weights, stream);
+}
+
 fp4_status fp4_moe_gather(const uint8_t *x_codes, const uint8_t *x_sf, int64_t T, int32_t topk, int64_t H,
                           int32_t E, const int32_t *offsets, const int32_t *tile_offsets, const int32_t *perm,
                           uint8_t *a_codes, uint8_t *a_sf, int64_t rows_cap, fp4_stream_t stream) {

@@ -252,6 +252,19 @@ fp4_status fp4_moe_grouped_gemm(const void *tokens_bf16, const int32_t *expert_i
 
 /* ---- the layer's stages, each callable on its own ------------------------ */
 
+/* bf16 x bf16 -> fp32 GEMM on tcgen05 kind::f16 (the router's gate
+ * projection): c[M][N] = a[M][K] . b[N][K]^T, both K-major, fp32
+ * accumulation.  K % 64 == 0, N % 8 == 0; pointers 16-byte aligned. */
+fp4_status fp4_gemm_bf16(const void *a_bf16, const void *b_bf16, float *c, int64_t M, int64_t N, int64_t K,
+                         fp4_stream_t stream);
+
+/* Router [QAT §3.1; ARCH §2.1]: logits = x . W_gate^T (fp4_gemm_bf16; x bf16
+ * [T][H], gate_w bf16 [E][H], logits fp32 [T][E], an output), then
+ * fp4_moe_topk on those logits.  H % 64 == 0, E % 8 == 0. */
+fp4_status fp4_moe_router(const void *x_bf16, int64_t T, int64_t H, const void *gate_w_bf16, int32_t E,
+                          int32_t topk, float *logits, int32_t *expert_ids, float *topk_weights,
+                          fp4_stream_t stream);
+
 /* Router top-k [QAT §3.1: each token is sent to its top-k experts; ARCH §2.1:
  * top-6 of 384]: logits fp32 [T][E] -> expert_ids int32 [T][topk] (the topk
  * largest logits in descending order, ties to the lower expert id) and
