@@ -183,7 +183,7 @@ def barrier(world):
 
 # ---------------------------------------------------------------------------
 class MoeBench:
-    def __init__(self, name, seed, pair_tiles=False):
+    def __init__(self, name, seed, pair_tiles=False, dynamic_h=False):
         import torch
 
         import fp4_block_scaled_03_b200 as fp4
@@ -197,6 +197,10 @@ class MoeBench:
         self.pair = pair_tiles and not self.mx
         if self.pair:
             self.flags |= fp4.FP4_MOE_PAIR_TILES
+        # NVFP4 row tiles: the h scale from each batch (two-phase w13) instead of a calibrated one
+        self.dynamic_h = dynamic_h and not self.mx and not self.pair
+        if self.dynamic_h:
+            self.flags |= fp4.FP4_MOE_DYNAMIC_H
         T, H, I, E, k, zipf, sigma, desc = WORKLOADS[name]
         self.T, self.H, self.I, self.E, self.k, self.desc, self.name = T, H, I, E, k, desc, name
         dev = "cuda"
@@ -261,6 +265,12 @@ class MoeBench:
         self.out = torch.empty((T, H), dtype=torch.bfloat16, device=d)
         self.wset = fp4.MoeWeightSet(self.w13_codes, self.w13_sf, self.w13_g, self.w2_codes, self.w2_sf, self.w2_g,
                                      self.h_g)
+        if self.dynamic_h:
+            self.h_f32 = torch.empty((cap, I), dtype=torch.float32, device=d)
+            self.h_amax = i32(E)
+            self.g_dyn = torch.empty(E, dtype=torch.float32, device=d)
+            self.wset_dyn = fp4.MoeWeightSet(self.w13_codes, self.w13_sf, self.w13_g, self.w2_codes, self.w2_sf,
+                                             self.w2_g, self.g_dyn)
 
     def calibrate(self):
         """h_g[e] = max|h| over expert e's rows of this batch / 2688 (once;
@@ -268,7 +278,7 @@ class MoeBench:
         import torch
 
         fp4 = self.fp4
-        if self.mx:
+        if self.mx or self.dynamic_h:
             return
         dump = torch.zeros((self.cap, self.I), dtype=torch.float32, device="cuda")
         self.step(events=None, dump=dump)
@@ -297,10 +307,17 @@ class MoeBench:
         fp4.fp4_moe_quantize_gather(self.x, T, k, H, E, self.offs, self.toffs, self.inv, self.a_c, self.a_s, cap,
                                     self.xg, self.qws, self.flags)
         ev(2)
-        fp4.fp4_moe_w13(self.a_c, self.a_s, self.xg, self.wset, H, I, E, self.counts_d, self.toffs, cap, self.h_c,
-                        self.h_s, (fp4.FP4_DEBUG_DUMP_H if dump is not None else 0) | self.flags, dump)
+        if self.dynamic_h:  # phase 1 (fp32 h + amax) and phase 2 (NVFP4 h with g = amax/2688), timed as w13
+            fp4.fp4_moe_w13_h(self.a_c, self.a_s, self.xg, self.wset, H, I, E, self.counts_d, self.toffs, cap,
+                              self.h_f32, self.h_amax)
+            fp4.fp4_moe_h_requant(self.h_f32, self.counts_d, self.toffs, I, E, cap, self.h_amax, self.g_dyn,
+                                  self.h_c, self.h_s)
+        else:
+            fp4.fp4_moe_w13(self.a_c, self.a_s, self.xg, self.wset, H, I, E, self.counts_d, self.toffs, cap,
+                            self.h_c, self.h_s, (fp4.FP4_DEBUG_DUMP_H if dump is not None else 0) | self.flags,
+                            dump)
         ev(3)
-        fp4.fp4_moe_w2(self.h_c, self.h_s, self.wset, H, I, E, self.counts_d, self.offs, self.toffs, self.perm, self.w,
+        fp4.fp4_moe_w2(self.h_c, self.h_s, self.wset_dyn if self.dynamic_h else self.wset, H, I, E, self.counts_d, self.offs, self.toffs, self.perm, self.w,
                        cap, self.y, self.flags)
         ev(4)
         fp4.fp4_moe_combine(self.y, self.inv, T, k, H, self.out)
@@ -338,7 +355,7 @@ def run_moe(args, world, rank, peaks):
     import torch
 
     fp4 = __import__("fp4_block_scaled_03_b200")
-    b = MoeBench(args.workload, seed=rank * 7919, pair_tiles=args.pair_tiles)
+    b = MoeBench(args.workload, seed=rank * 7919, pair_tiles=args.pair_tiles, dynamic_h=args.dynamic_h)
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
     for _ in range(args.warmup):
@@ -467,6 +484,9 @@ def run_moe(args, world, rank, peaks):
                    "l2": "inputs larger than L2 (weights %.2f GB)" % (b.E * 3 * b.H * b.I * 0.5625 / 1e9),
                    "experts_touched": int((b.counts > 0).sum().item()),
                    "tiling": b.tiling_desc(), "mma_rows": b.mma_rows(),
+                   "h_scale": ("power of two per 32 (MX)" if b.mx else
+                               "per expert from this batch (two-phase w13)" if b.dynamic_h else
+                               "static per expert, calibrated once on the batch"),
                    "padding_frac": round(1.0 - b.R / max(1, b.mma_rows()), 4)},
         "roofline": {"bound": "tensor", "kernel": b.kernel_name("w13") + " (grouped w13 + SwiGLU + requant)",
                      "achieved": round(w13_tf, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
@@ -489,7 +509,7 @@ def run_moe(args, world, rank, peaks):
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "how": "fp4_moe_grouped_gemm per step; pinned host->device inputs and device->host output on their own"
                        " streams, overlapping neighbouring steps (2 buffer sets)"},
-        "gpu_launches": MoeBench.LAUNCHES_PER_STEP * args.steps,
+        "gpu_launches": (MoeBench.LAUNCHES_PER_STEP + (1 if b.dynamic_h else 0)) * args.steps,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -808,6 +828,8 @@ def main():
     ap.add_argument("--workload", default="pro", choices=list(WORKLOADS) + ["dense4096", "dense4096mx", "dense4096w4a8", "router", "quant"])
     ap.add_argument("--impl", default="fp4", choices=["fp4", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--dynamic-h", action="store_true",
+                    help="NVFP4 MoE workloads: per-expert h scale from each batch (two-phase w13)")
     ap.add_argument("--pair-tiles", action="store_true",
                     help="MoE workloads: CTA-pair tiles (cta_group::2, tokens on N) for the NVFP4 grouped GEMMs")
     args = ap.parse_args()

@@ -27,6 +27,7 @@ FP4_GEMM_MX = 0x8
 FP4_GEMM_A_MXFP8 = 0x40
 FP4_GEMM_B_MXFP8 = 0x80
 FP4_MOE_W4A8 = 0x100
+FP4_MOE_DYNAMIC_H = 0x200
 FP4_MOE_MX = 0x10
 FP4_MOE_PAIR_TILES = 0x20
 
@@ -81,6 +82,9 @@ _SIGS = {
     "fp4_mx_to_nv": (ctypes.c_int, [_P, _P, _I64, _I64, _I64, _P, _P, _U32, _P]),
     "fp4_e2m1_to_e4m3": (ctypes.c_int, [_P, _I64, _I64, _P, _P]),
     "fp4_gemm_bf16": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _I64, _P]),
+    "fp4_moe_w13_h": (ctypes.c_int, [_P, _P, _P, ctypes.POINTER(MoeWeights), _I64, _I64, _I32, _P, _P, _I64, _P, _P,
+                                     _P]),
+    "fp4_moe_h_requant": (ctypes.c_int, [_P, _P, _P, _I64, _I32, _I64, _P, _P, _P, _P, _P]),
     "fp4_moe_router": (ctypes.c_int, [_P, _I64, _I64, _P, _I32, _I32, _P, _P, _P, _P]),
     "fp4_gemm": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, ctypes.c_int, _I64, _I64, _I64, _U32, _P]),
     "fp4_moe_workspace_size": (_SZ, [_I64, _I32, _I64, _I64, _I32]),
@@ -199,6 +203,17 @@ def fp4_moe_w13(a_codes, a_sf, a_g, w, H, I, E, counts, tile_offsets, rows_cap, 
     _check(lib.fp4_moe_w13(_ptr(a_codes), _ptr(a_sf), _ptr(a_g), ctypes.byref(w.c_struct()), H, I, E, _ptr(counts),
                            _ptr(tile_offsets), rows_cap, _ptr(h_codes), _ptr(h_sf), flags, _ptr(h_dump), _stream()),
            "fp4_moe_w13")
+
+
+def fp4_moe_w13_h(a_codes, a_sf, a_g, w, H, I, E, counts, tile_offsets, rows_cap, h_f32, h_amax):
+    _check(lib.fp4_moe_w13_h(_ptr(a_codes), _ptr(a_sf), _ptr(a_g), ctypes.byref(w.c_struct()), H, I, E,
+                             _ptr(counts), _ptr(tile_offsets), rows_cap, _ptr(h_f32), _ptr(h_amax), _stream()),
+           "fp4_moe_w13_h")
+
+
+def fp4_moe_h_requant(h_f32, counts, tile_offsets, I, E, rows_cap, h_amax, h_g_out, h_codes, h_sf):
+    _check(lib.fp4_moe_h_requant(_ptr(h_f32), _ptr(counts), _ptr(tile_offsets), I, E, rows_cap, _ptr(h_amax),
+                                 _ptr(h_g_out), _ptr(h_codes), _ptr(h_sf), _stream()), "fp4_moe_h_requant")
 
 
 def fp4_moe_w2(h_codes, h_sf, w, H, I, E, counts, offsets, tile_offsets, perm, topk_weights, rows_cap, y, flags=0):
@@ -364,13 +379,14 @@ def moe_rows_cap(T, topk, E):
 
 
 def moe_layer(x, expert_ids, topk_weights, w, H, I, E, workspace=None, out=None, h_dump=None, mx=False,
-              pair_tiles=False, w4a8=False):
+              pair_tiles=False, w4a8=False, dynamic_h=False):
     """mx: MXFP4 weights, activations and h.  w4a8: MXFP4 weights with MXFP8
     activations and h (FP8 x FP4 grouped GEMMs)."""
     T, topk = expert_ids.shape
     dev = x.device
     flags = (FP4_DEBUG_DUMP_H if h_dump is not None else 0) | (FP4_MOE_MX if mx else 0)
     flags |= (FP4_MOE_PAIR_TILES if pair_tiles else 0) | (FP4_MOE_W4A8 if w4a8 else 0)
+    flags |= FP4_MOE_DYNAMIC_H if dynamic_h else 0
     if workspace is None:
         workspace = _u8(fp4_moe_workspace_size_flags(T, topk, H, I, E, flags), dev)
     if out is None:

@@ -100,6 +100,8 @@ struct Params {
   uint8_t *h_codes;
   uint8_t *h_sf;
   float *h_dump;
+  float *h_f32;            // dynamic h scale, phase 1: fp32 h out instead of NVFP4 codes
+  unsigned int *h_amax;    // ... and per-expert max |h| (fp32 bits, atomicMax)
   int I;
   const int32_t *perm;
   const float *topk_w;
@@ -384,6 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (EPI == EPI_W2 && p.topk_w) scale = MX ? p.topk_w[p.perm[ti.out_row0 + row]]
                                                 : __fmul_rn(alpha, p.topk_w[p.perm[ti.out_row0 + row]]);
       const int colh = ti.n0 + half * HC;
+      float hmax = 0.0f;  // dynamic h scale: this thread's max |h| over the tile
       if constexpr (EPI == EPI_W13 && KIND >= 1) {
         // MXFP4 h (KIND 1) or MXFP8 h (KIND 2, W4A8): one 32-element block per
         // pair of 32-column chunks (16 gate + 16 up columns each), quantized
@@ -458,6 +461,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const int hc = col0 / 2;
           const int64_t prow = (int64_t)ti.a_row0 + row;  // padded row
+          if (p.h_f32) {  // phase 1 of the dynamic h scale: keep h in fp32, track the expert's amax
+            float4 *d = reinterpret_cast<float4 *>(p.h_f32 + prow * p.I + hc);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) d[i] = make_float4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) hmax = fmaxf(hmax, fabsf(h[i]));
+            continue;
+          }
           uint32_t lo, hi;
           const uint32_t sf = nvfp4_block16(h, p.h_g[ti.e], &lo, &hi);
           *reinterpret_cast<uint2 *>(p.h_codes + prow * (p.I / 2) + hc / 2) = make_uint2(lo, hi);
@@ -496,6 +507,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       }  // generic epilogue
+      if constexpr (EPI == EPI_W13 && KIND == 0) {
+        if (p.h_amax) {  // one atomic per warp: the lanes holding valid rows reduce first
+          const unsigned mask = __activemask();
+          const unsigned m = __reduce_max_sync(mask, __float_as_uint(hmax));
+          if (lane == __ffs(mask) - 1) atomicMax(p.h_amax + ti.e, m);
+        }
+      }
     }
     if (EPI == EPI_W2 && lane == 0) bulk_wait_all();  // stores complete before the CTA exits
   }
@@ -614,20 +632,27 @@ fp4_status fp4_gemm_bf16(const void *a_bf16, const void *b_bf16, float *c, int64
   return launch<kBN, EPI_F32, 3>(ta, tb, tb, p, grid, reinterpret_cast<cudaStream_t>(stream));
 }
 
-fp4_status fp4_moe_w13(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_g, const fp4_moe_weights *w,
-                       int64_t H, int64_t I, int32_t E, const int32_t *counts, const int32_t *tile_offsets,
-                       int64_t rows_cap, uint8_t *h_codes, uint8_t *h_sf, uint32_t flags, float *h_dump,
-                       fp4_stream_t stream) {
-  if (!a_codes || !a_sf || !w || !w->w13_codes || !w->w13_sf || !counts || !tile_offsets || !h_codes || !h_sf)
+// fp4_moe_w13, or with h_f32 / h_amax set (NVFP4 only) phase 1 of the
+// dynamic h scale: fp32 h and per-expert amax instead of NVFP4 h.
+static fp4_status moe_w13_impl(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_g,
+                               const fp4_moe_weights *w, int64_t H, int64_t I, int32_t E, const int32_t *counts,
+                               const int32_t *tile_offsets, int64_t rows_cap, uint8_t *h_codes, uint8_t *h_sf,
+                               uint32_t flags, float *h_dump, float *h_f32, unsigned int *h_amax,
+                               fp4_stream_t stream) {
+  const bool dyn = h_f32 != nullptr;
+  if (!a_codes || !a_sf || !w || !w->w13_codes || !w->w13_sf || !counts || !tile_offsets ||
+      (!dyn && (!h_codes || !h_sf)) || (dyn && !h_amax))
     return FP4_ERR_INVALID_ARG;
   const bool w4a8 = flags & FP4_MOE_W4A8;  // MXFP8 activations and h, MXFP4 weights
   const bool mx = (flags & FP4_MOE_MX) || w4a8;
-  if (!mx && (!a_g || !w->w13_g || !w->h_g)) return FP4_ERR_INVALID_ARG;
+  if (!mx && (!a_g || !w->w13_g || (!dyn && !w->h_g))) return FP4_ERR_INVALID_ARG;
   if ((flags & FP4_DEBUG_DUMP_H) && !h_dump) return FP4_ERR_INVALID_ARG;
+  if (dyn && (mx || (flags & FP4_MOE_PAIR_TILES))) return FP4_ERR_INVALID_ARG;
   if (H < 256 || H % 256 || I < 256 || I % 256 || E < 1 || E > 4096 || rows_cap < 1) return FP4_ERR_UNSUPPORTED_SHAPE;
   if ((int64_t)E * 2 * I > (1LL << 31) - 1 || rows_cap > (1LL << 31) - 1) return FP4_ERR_UNSUPPORTED_SHAPE;
-  if (!al16(a_codes) || !al16(a_sf) || !al16(w->w13_codes) || !al16(w->w13_sf) || !al16(h_codes) || !al16(h_sf) ||
-      (h_dump && !al16(h_dump)) || (w4a8 && (reinterpret_cast<uintptr_t>(w->w13_codes) & 31u)))
+  if (!al16(a_codes) || !al16(a_sf) || !al16(w->w13_codes) || !al16(w->w13_sf) || (h_codes && !al16(h_codes)) ||
+      (h_sf && !al16(h_sf)) || (h_dump && !al16(h_dump)) || (h_f32 && !al16(h_f32)) ||
+      (w4a8 && (reinterpret_cast<uintptr_t>(w->w13_codes) & 31u)))
     return FP4_ERR_ALIGNMENT;
   if (!mx && (flags & FP4_MOE_PAIR_TILES)) {
     if (((rows_cap + 255) / 256 + E) * (2 * I / 256) > (1LL << 31) - 1) return FP4_ERR_UNSUPPORTED_SHAPE;
@@ -659,11 +684,31 @@ fp4_status fp4_moe_w13(const uint8_t *a_codes, const uint8_t *a_sf, const float 
   p.w_g = w->w13_g; p.h_g = w->h_g;
   p.h_codes = h_codes; p.h_sf = h_sf; p.I = (int)I;
   p.h_dump = (flags & FP4_DEBUG_DUMP_H) ? h_dump : nullptr;
+  p.h_f32 = h_f32;
+  p.h_amax = h_amax;
   p.status = ctx->status;
   p.wait_limit = ctx->wait_limit_ns;
+  if (dyn) FP4_HOST_CHECK(cudaMemsetAsync(h_amax, 0, (size_t)E * sizeof(unsigned int),
+                                          reinterpret_cast<cudaStream_t>(stream)));
   if (w4a8) return launch<kBN, EPI_W13, 2>(ta, tb, tb, p, sm_count(), reinterpret_cast<cudaStream_t>(stream));
   if (mx) return launch<kBN, EPI_W13, 1>(ta, tb, tb, p, sm_count(), reinterpret_cast<cudaStream_t>(stream));
   return launch<kBN, EPI_W13>(ta, tb, tb, p, sm_count(), reinterpret_cast<cudaStream_t>(stream));
+}
+
+fp4_status fp4_moe_w13(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_g, const fp4_moe_weights *w,
+                       int64_t H, int64_t I, int32_t E, const int32_t *counts, const int32_t *tile_offsets,
+                       int64_t rows_cap, uint8_t *h_codes, uint8_t *h_sf, uint32_t flags, float *h_dump,
+                       fp4_stream_t stream) {
+  return moe_w13_impl(a_codes, a_sf, a_g, w, H, I, E, counts, tile_offsets, rows_cap, h_codes, h_sf, flags, h_dump,
+                      nullptr, nullptr, stream);
+}
+
+fp4_status fp4_moe_w13_h(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_g, const fp4_moe_weights *w,
+                         int64_t H, int64_t I, int32_t E, const int32_t *counts, const int32_t *tile_offsets,
+                         int64_t rows_cap, float *h_f32, uint32_t *h_amax, fp4_stream_t stream) {
+  if (!h_f32 || !h_amax) return FP4_ERR_INVALID_ARG;
+  return moe_w13_impl(a_codes, a_sf, a_g, w, H, I, E, counts, tile_offsets, rows_cap, nullptr, nullptr, 0, nullptr,
+                      h_f32, h_amax, stream);
 }
 
 fp4_status fp4_moe_w2(const uint8_t *h_codes, const uint8_t *h_sf, const fp4_moe_weights *w, int64_t H, int64_t I,

@@ -14,14 +14,17 @@ namespace {
 
 struct MoeLayout {
   size_t header, counts, offsets, tile_offsets, perm, inv, scratch, a_codes, a_sf, h_codes, h_sf, y;
+  size_t h_f32, h_amax, h_g;  // dynamic h scale only (0 bytes otherwise)
   size_t total;
   int64_t rows_cap;
 };
 
 size_t up256(size_t v) { return (v + 255) & ~size_t(255); }
 
-// codes_per_byte: 2 for FP4 activations and h, 1 for FP8 (W4A8).
-MoeLayout moe_layout(int64_t T, int32_t topk, int64_t H, int64_t I, int32_t E, int codes_per_byte) {
+// codes_per_byte: 2 for FP4 activations and h, 1 for FP8 (W4A8); dyn_h: room
+// for the dynamic h scale's fp32 h and per-expert amax / scale.
+MoeLayout moe_layout(int64_t T, int32_t topk, int64_t H, int64_t I, int32_t E, int codes_per_byte,
+                     bool dyn_h = false) {
   MoeLayout L;
   const int64_t R = T * topk;
   L.rows_cap = ((R + 127LL * E + 127) / 128) * 128;
@@ -43,6 +46,9 @@ MoeLayout moe_layout(int64_t T, int32_t topk, int64_t H, int64_t I, int32_t E, i
   L.h_codes = take((size_t)(L.rows_cap * I / codes_per_byte));
   L.h_sf = take(fp4_sf_tiled_bytes(L.rows_cap, I));
   L.y = take((size_t)R * (size_t)H * 4);
+  L.h_f32 = take(dyn_h ? (size_t)L.rows_cap * (size_t)I * 4 : 0);
+  L.h_amax = take(dyn_h ? (size_t)E * 4 : 0);
+  L.h_g = take(dyn_h ? (size_t)E * 4 : 0);
   L.total = off;
   return L;
 }
@@ -58,7 +64,7 @@ size_t fp4_moe_workspace_size(int64_t T, int32_t topk, int64_t H, int64_t I, int
 
 size_t fp4_moe_workspace_size_flags(int64_t T, int32_t topk, int64_t H, int64_t I, int32_t E, uint32_t flags) {
   if (T < 0 || topk < 1 || H <= 0 || I <= 0 || E < 1) return 0;
-  return moe_layout(T, topk, H, I, E, (flags & FP4_MOE_W4A8) ? 1 : 2).total;
+  return moe_layout(T, topk, H, I, E, (flags & FP4_MOE_W4A8) ? 1 : 2, (flags & FP4_MOE_DYNAMIC_H) != 0).total;
 }
 
 fp4_status fp4_moe_grouped_gemm(const void *tokens_bf16, const int32_t *expert_ids, const float *topk_weights,
@@ -71,7 +77,9 @@ fp4_status fp4_moe_grouped_gemm(const void *tokens_bf16, const int32_t *expert_i
   if (T == 0) return FP4_OK;  // empty batch: no work, token / id / output pointers may be NULL
   if (!tokens_bf16 || !expert_ids || !out_bf16) return FP4_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(workspace) & 255u) return FP4_ERR_ALIGNMENT;
-  const MoeLayout L = moe_layout(T, topk, H, I, E, (flags & FP4_MOE_W4A8) ? 1 : 2);
+  const bool dyn_h = flags & FP4_MOE_DYNAMIC_H;
+  if (dyn_h && (flags & (FP4_MOE_MX | FP4_MOE_W4A8 | FP4_MOE_PAIR_TILES))) return FP4_ERR_INVALID_ARG;
+  const MoeLayout L = moe_layout(T, topk, H, I, E, (flags & FP4_MOE_W4A8) ? 1 : 2, dyn_h);
   if (ws_bytes < L.total) return FP4_ERR_WORKSPACE;
   if ((flags & FP4_DEBUG_DUMP_H) && !h_dump) return FP4_ERR_INVALID_ARG;
   if (T == 0) return FP4_OK;
@@ -87,10 +95,24 @@ fp4_status fp4_moe_grouped_gemm(const void *tokens_bf16, const int32_t *expert_i
   st = fp4_moe_quantize_gather(tokens_bf16, T, topk, H, E, I32(L.offsets), I32(L.tile_offsets), I32(L.inv),
                                ws + L.a_codes, ws + L.a_sf, L.rows_cap, g_x, ws + L.header, 256, fmt, stream);
   if (st != FP4_OK) return st;
-  st = fp4_moe_w13(ws + L.a_codes, ws + L.a_sf, g_x, w, H, I, E, I32(L.counts), I32(L.tile_offsets), L.rows_cap,
-                   ws + L.h_codes, ws + L.h_sf, (flags & FP4_DEBUG_DUMP_H) | fmt | tiling, h_dump, stream);
+  fp4_moe_weights wd = *w;  // the dynamic h scale replaces the static one for w2
+  if (dyn_h) {
+    // phase 1: fp32 h (into h_dump when the caller asked for it) and per-expert amax; phase 2: NVFP4 h
+    float *hf = (flags & FP4_DEBUG_DUMP_H) ? h_dump : reinterpret_cast<float *>(ws + L.h_f32);
+    uint32_t *amax = reinterpret_cast<uint32_t *>(ws + L.h_amax);
+    float *g_h = reinterpret_cast<float *>(ws + L.h_g);
+    st = fp4_moe_w13_h(ws + L.a_codes, ws + L.a_sf, g_x, w, H, I, E, I32(L.counts), I32(L.tile_offsets), L.rows_cap,
+                       hf, amax, stream);
+    if (st != FP4_OK) return st;
+    st = fp4_moe_h_requant(hf, I32(L.counts), I32(L.tile_offsets), I, E, L.rows_cap, amax, g_h, ws + L.h_codes,
+                           ws + L.h_sf, stream);
+    wd.h_g = g_h;
+  } else {
+    st = fp4_moe_w13(ws + L.a_codes, ws + L.a_sf, g_x, w, H, I, E, I32(L.counts), I32(L.tile_offsets), L.rows_cap,
+                     ws + L.h_codes, ws + L.h_sf, (flags & FP4_DEBUG_DUMP_H) | fmt | tiling, h_dump, stream);
+  }
   if (st != FP4_OK) return st;
-  st = fp4_moe_w2(ws + L.h_codes, ws + L.h_sf, w, H, I, E, I32(L.counts), I32(L.offsets), I32(L.tile_offsets),
+  st = fp4_moe_w2(ws + L.h_codes, ws + L.h_sf, &wd, H, I, E, I32(L.counts), I32(L.offsets), I32(L.tile_offsets),
                   I32(L.perm), topk_weights, L.rows_cap, reinterpret_cast<float *>(ws + L.y), fmt | tiling, stream);
   if (st != FP4_OK) return st;
   return fp4_moe_combine(reinterpret_cast<const float *>(ws + L.y), I32(L.inv), T, topk, H, out_bf16, stream);

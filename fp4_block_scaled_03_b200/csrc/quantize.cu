@@ -286,6 +286,53 @@ __global__ void __launch_bounds__(128) mxfp8_quantize_gather_kernel(
   }
 }
 
+// ---- dynamic h scale, phase 2: NVFP4-quantize each routed row of h -----------
+// g_e = amax_e / 2688 from the per-expert max |h| of phase 1 (fp32 bits); one
+// warp per padded row, a lane per K step of 64 (four 16-element blocks, one
+// tiled scale word).  Padding rows are skipped.
+__global__ void __launch_bounds__(128) h_requant_kernel(const float *__restrict__ h, int64_t rows_cap, int64_t I,
+                                                        int32_t E, const int32_t *__restrict__ counts,
+                                                        const int32_t *__restrict__ tile_offsets,
+                                                        const unsigned int *__restrict__ amax_bits,
+                                                        float *__restrict__ g_out, uint8_t *__restrict__ h_codes,
+                                                        uint8_t *__restrict__ h_sf) {
+  const int lane = threadIdx.x & 31;
+  const int64_t gtid = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  for (int64_t e = gtid; e < E; e += (int64_t)gridDim.x * blockDim.x)
+    g_out[e] = __fdiv_rn(__uint_as_float(amax_bits[e]), 2688.0f);
+  const int64_t n_ksteps = I / 64;
+  const int64_t rows = (int64_t)tile_offsets[E] * 128;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
+  for (int64_t r = gtid >> 5; r < rows && r < rows_cap; r += warps) {
+    const int32_t tile = (int32_t)(r >> 7);
+    int lo = 0, hi = E;  // largest e with tile_offsets[e] <= tile
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (tile_offsets[mid] <= tile) lo = mid; else hi = mid;
+    }
+    if (r - (int64_t)tile_offsets[lo] * 128 >= counts[lo]) continue;  // padding row
+    const float g = __fdiv_rn(__uint_as_float(amax_bits[lo]), 2688.0f);
+    for (int64_t kw = lane; kw < n_ksteps; kw += 32) {
+      const float4 *src = reinterpret_cast<const float4 *>(h + r * I + kw * 64);
+      uint32_t code[8], sfw = 0;
+#pragma unroll
+      for (int blk = 0; blk < 4; ++blk) {
+        float f[16];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float4 v = __ldcs(src + 4 * blk + q);
+          f[4 * q] = v.x; f[4 * q + 1] = v.y; f[4 * q + 2] = v.z; f[4 * q + 3] = v.w;
+        }
+        sfw |= nvfp4_block16(f, g, code + 2 * blk, code + 2 * blk + 1) << (8 * blk);
+      }
+      uint4 *out = reinterpret_cast<uint4 *>(h_codes + r * (I / 2) + kw * 32);
+      out[0] = make_uint4(code[0], code[1], code[2], code[3]);
+      out[1] = make_uint4(code[4], code[5], code[6], code[7]);
+      *reinterpret_cast<uint32_t *>(h_sf + sf_tiled_offset(r, kw * 4, n_ksteps)) = sfw;
+    }
+  }
+}
+
 // ---- MXFP8 quantize (W4A8 activations): one thread per 32-element block ----
 // Same block rule as MXFP4 with E4M3 elements: X = clamp(floor(log2 amax) - 8),
 // element = E4M3_RNE_satfinite(x * 2^-X).
@@ -537,6 +584,24 @@ fp4_status fp4_quantize(fp4_format fmt, const void *x_bf16, int64_t rows, int64_
     nvfp4_quantize_kernel<true><<<grid, kThreads, 0, s>>>(x, rows, cols, ld, codes, scales, amax, global_scale, g_in);
   else
     nvfp4_quantize_kernel<false><<<grid, kThreads, 0, s>>>(x, rows, cols, ld, codes, scales, amax, global_scale, g_in);
+  FP4_HOST_CHECK(cudaGetLastError());
+  return FP4_OK;
+}
+
+fp4_status fp4_moe_h_requant(const float *h_f32, const int32_t *counts, const int32_t *tile_offsets, int64_t I,
+                             int32_t E, int64_t rows_cap, const uint32_t *h_amax, float *h_g_out, uint8_t *h_codes,
+                             uint8_t *h_sf, fp4_stream_t stream) {
+  if (!h_f32 || !counts || !tile_offsets || !h_amax || !h_g_out || !h_codes || !h_sf) return FP4_ERR_INVALID_ARG;
+  if (I < 64 || I % 64 || E < 1 || E > 4096 || rows_cap < 1) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(h_f32) || !aligned16(h_codes) || (reinterpret_cast<uintptr_t>(h_sf) & 3u))
+    return FP4_ERR_ALIGNMENT;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t need = (rows_cap + 3) / 4;  // four rows (warps) per CTA
+  const int64_t grid = need < (int64_t)sms * 16 ? need : (int64_t)sms * 16;
+  h_requant_kernel<<<(unsigned)grid, 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      h_f32, rows_cap, I, E, counts, tile_offsets, h_amax, h_g_out, h_codes, h_sf);
   FP4_HOST_CHECK(cudaGetLastError());
   return FP4_OK;
 }

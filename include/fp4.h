@@ -85,6 +85,7 @@ typedef enum { FP4_OUT_F32 = 0, FP4_OUT_BF16 = 1 } fp4_out_dtype;
 #define FP4_GEMM_A_MXFP8 0x40u       /* fp4_gemm: W4A8 -- A is MXFP8 (E4M3, UE8M0 per 32), B MXFP4 */
 #define FP4_GEMM_B_MXFP8 0x80u       /* fp4_gemm with FP4_GEMM_A_MXFP8: B is MXFP8 too */
 #define FP4_MOE_W4A8 0x100u          /* MoE layer / stages: MXFP4 weights, MXFP8 activations and h */
+#define FP4_MOE_DYNAMIC_H 0x200u     /* MoE layer (NVFP4, row tiles): h scale per expert from this batch */
 
 /* Human-readable name of a status code (static string). */
 const char *fp4_status_string(fp4_status s);
@@ -240,7 +241,10 @@ size_t fp4_moe_workspace_size_flags(int64_t T, int32_t topk, int64_t H, int64_t 
  *   topk_weights fp32 [T][topk] or NULL (weights 1.0);  out_bf16 [T][H].
  *   workspace >= fp4_moe_workspace_size_flags(..., flags), 256-byte aligned.
  *   flags: FP4_DEBUG_DUMP_H needs h_dump (fp32, rows = padded routed rows,
- *   I columns); otherwise h_dump may be NULL.
+ *   I columns); otherwise h_dump may be NULL.  FP4_MOE_DYNAMIC_H (NVFP4 row
+ *   tiles only): h is re-quantized with g_h[e] = max |h| over expert e's rows
+ *   of this batch / 2688 (fp4_moe_w13_h + fp4_moe_h_requant); w->h_g is not
+ *   read; the workspace grows by rows_cap * I * 4 bytes.
  * Expert ids outside [0,E) set FP4_ERR_BAD_EXPERT in the device status; such
  * slots contribute nothing.
  */
@@ -340,6 +344,26 @@ fp4_status fp4_moe_w13(const uint8_t *a_codes, const uint8_t *a_sf, const float 
                        const int32_t *counts, const int32_t *tile_offsets, int64_t rows_cap,
                        uint8_t *h_codes, uint8_t *h_sf, uint32_t flags, float *h_dump,
                        fp4_stream_t stream);
+
+/* Dynamic per-expert h scale (FP4_MOE_DYNAMIC_H in the layer) in two
+ * phases [QAT §四 reads the h scale as calibrated; this derives it from the
+ * batch instead]:
+ * fp4_moe_w13_h -- phase 1: the grouped w13 GEMM + SwiGLU of fp4_moe_w13
+ *   (NVFP4, row tiles) writing fp32 h [rows_cap][I] (rows that hold a routed
+ *   row) and h_amax uint32 [E] = the fp32 bits of max |h| over each expert's
+ *   rows (zeroed by the call first).  w->h_g is not read. */
+fp4_status fp4_moe_w13_h(const uint8_t *a_codes, const uint8_t *a_sf, const float *a_g,
+                         const fp4_moe_weights *w, int64_t H, int64_t I, int32_t E,
+                         const int32_t *counts, const int32_t *tile_offsets, int64_t rows_cap,
+                         float *h_f32, uint32_t *h_amax, fp4_stream_t stream);
+
+/* fp4_moe_h_requant -- phase 2: h_g_out[e] = amax_e / 2688 (fp32), and each
+ * routed row of h_f32 NVFP4-quantized with its expert's g (the fp4_quantize
+ * NV rule) into h_codes [rows_cap][I/2] and tiled h_sf; padding rows are not
+ * written.  I % 64 == 0. */
+fp4_status fp4_moe_h_requant(const float *h_f32, const int32_t *counts, const int32_t *tile_offsets,
+                             int64_t I, int32_t E, int64_t rows_cap, const uint32_t *h_amax,
+                             float *h_g_out, uint8_t *h_codes, uint8_t *h_sf, fp4_stream_t stream);
 
 /* Grouped w2 GEMM: y[offsets[e]+i] = w[perm[row]] * h_g[e]*w2_g[e] * (h . W2_e^T)
  * y: fp32 [T*topk][H] in routed order; topk_weights may be NULL.

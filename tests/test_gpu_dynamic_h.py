@@ -1,0 +1,122 @@
+"""Dynamic per-expert h scale (FP4_MOE_DYNAMIC_H): phase 1 (fp4_moe_w13_h,
+fp32 h and per-expert amax) and phase 2 (fp4_moe_h_requant) against the
+oracle.  The scale is the NVFP4 tensor-scale rule ("DeepSeek-V4.1-Flash-NVFP4"
+§二) applied to each expert's rows of h: g_e = max |h_e| / 2688.
+
+Every integer decision is checked on the device's own fp32 h: the amax bits,
+g (one fp32 division), and the codes and scales (the oracle's quantizer with
+that g) are bit-exact; h itself is checked against the oracle's fp64 h within
+the w13 error band, and g against the oracle's g within that band's reach."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import formats as F
+from oracle import gemm as G
+from oracle import layouts as LY
+from oracle import moe as MO
+from oracle import quant as Q
+from tests import moe_case
+from tests import test_gpu_moe as TM
+from tests._util import bf16_bits, bf16_ulps_apart, np_u8
+
+pytestmark = pytest.mark.gpu
+
+
+def _lib():
+    import fp4_block_scaled_03_b200 as fp4
+
+    return fp4
+
+
+@pytest.mark.parametrize("T,H,I,E,k,zipf", [(200, 512, 256, 8, 2, 0.0), (700, 1024, 512, 6, 6, 1.1)])
+def test_two_phase_h_requant(T, H, I, E, k, zipf):
+    fp4 = _lib()
+    c = moe_case.build(T, H, I, E, k, seed=T + 23, zipf=zipf)
+    xc, xs, xg = fp4.quantize_nv(c.x)
+    r = TM._route_gpu(c.ids, T, k, E)
+    cap = fp4.moe_rows_cap(T, k, E)
+    a_c = torch.empty((cap, H // 2), dtype=torch.uint8, device="cuda")
+    a_s = torch.empty(fp4.fp4_sf_tiled_bytes(cap, H), dtype=torch.uint8, device="cuda")
+    fp4.fp4_moe_gather(xc, xs, T, k, H, E, r["offsets"], r["tile_offsets"], r["perm"], a_c, a_s, cap)
+    h_f = torch.zeros((cap, I), dtype=torch.float32, device="cuda")
+    amax = torch.full((E,), 0xFFFFFFF, dtype=torch.int32, device="cuda")  # overwritten (zeroed) by the call
+    fp4.fp4_moe_w13_h(a_c, a_s, xg, c.weights, H, I, E, r["counts"], r["tile_offsets"], cap, h_f, amax)
+    g_out = torch.empty(E, dtype=torch.float32, device="cuda")
+    h_c = torch.zeros((cap, I // 2), dtype=torch.uint8, device="cuda")
+    h_s = torch.zeros(fp4.fp4_sf_tiled_bytes(cap, I), dtype=torch.uint8, device="cuda")
+    fp4.fp4_moe_h_requant(h_f, r["counts"], r["tile_offsets"], I, E, cap, amax, g_out, h_c, h_s)
+    assert fp4.fp4_get_device_status() == 0
+
+    counts, offsets, perm, inv = MO.route(c.ids_np, E)
+    toff = TM._tile_offsets_ref(counts)
+    (xq, x_dq) = moe_case.oracle_x(c)
+    hg = h_f.cpu().numpy()
+    am = amax.cpu().numpy().astype(np.uint32).view(np.float32)
+    g = g_out.cpu().numpy()
+    codes = np_u8(h_c)
+    sf = LY.sf_from_mma(np_u8(h_s), cap, I)
+    for e in range(E):
+        if counts[e] == 0:
+            continue
+        prow = toff[e] * 128 + np.arange(counts[e])
+        h_dev = hg[prow]
+        # decisions on the device's own h: amax, g, codes and scales bit-exact
+        assert am[e] == np.abs(h_dev).max()
+        assert g[e] == Q.nv_global_scale(h_dev)
+        rc, rs, _ = Q.nvfp4_quantize(h_dev, g=np.float32(g[e]))
+        assert np.array_equal(codes[prow], rc) and np.array_equal(sf[prow], rs)
+        # h against the oracle's fp64 h, and g against the oracle's g
+        w1, w3, _, _, _ = moe_case.oracle_expert_weights(c, e)
+        xr = x_dq[perm[offsets[e]:offsets[e + 1]] // k]
+        gate, up = xr @ w1.T, xr @ w3.T
+        h = MO.swiglu(gate, up)
+        tol = TM._h_tol(xr, w1, w3, gate, up, h)
+        assert np.all(np.abs(h_dev - h) <= tol)
+        g_ref = np.abs(h).max() / 2688.0
+        assert abs(float(g[e]) - g_ref) <= tol.max() / 2688.0 + 2 ** -23 * g_ref
+
+
+@pytest.mark.parametrize("T,H,I,E,k,zipf", [(256, 512, 256, 8, 2, 0.0), (1000, 1024, 512, 16, 6, 1.1)])
+def test_layer_dynamic_h_end_to_end(T, H, I, E, k, zipf):
+    """The layer with FP4_MOE_DYNAMIC_H: its h (dumped) against the oracle's
+    within the band, and the output against the oracle's rest of the layer
+    run on the device's h -- g, codes and scales decided on that h, then w2
+    and the fixed-order combine: within 1 bf16 ulp, the w2 bound and the
+    combine's fp32-sum bound."""
+    fp4 = _lib()
+    c = moe_case.build(T, H, I, E, k, seed=T + 29, zipf=zipf)
+    cap = fp4.moe_rows_cap(T, k, E)
+    dump = torch.zeros((cap, I), dtype=torch.float32, device="cuda")
+    out = fp4.moe_layer(c.x, c.ids, c.w, c.weights, H, I, E, h_dump=dump, dynamic_h=True)
+    assert fp4.fp4_get_device_status() == 0
+    counts, offsets, perm, inv = MO.route(c.ids_np, E)
+    toff = TM._tile_offsets_ref(counts)
+    (xq, x_dq) = moe_case.oracle_x(c)
+    hd = dump.cpu().numpy()
+    y = np.zeros((T * k, H))
+    slack = np.zeros((T * k, H))
+    for e in range(E):
+        if counts[e] == 0:
+            continue
+        w1, w3, w2, _, _ = moe_case.oracle_expert_weights(c, e)
+        rr = slice(offsets[e], offsets[e + 1])
+        xr = x_dq[perm[rr] // k]
+        gate, up = xr @ w1.T, xr @ w3.T
+        h = MO.swiglu(gate, up)
+        prow = toff[e] * 128 + np.arange(counts[e])
+        h_dev = hd[prow]
+        assert np.all(np.abs(h_dev - h) <= TM._h_tol(xr, w1, w3, gate, up, h))
+        g = Q.nv_global_scale(h_dev)
+        h_dq = Q.nvfp4_dequantize(*Q.nvfp4_quantize(h_dev, g=g))
+        wt = c.w_np.reshape(-1)[perm[rr]].astype(np.float64)[:, None]
+        y[rr] = wt * (h_dq @ w2.T)
+        slack[rr] = G.FP32_REL_TOL * wt * (np.abs(h_dq) @ np.abs(w2).T)
+    ref, ref_bits = MO.combine_ref(y, inv)
+    sl = sum(slack[inv[:, s]] for s in range(k))
+    sum_abs = sum(np.abs(y[inv[:, s]]) for s in range(k))
+    got_bits = bf16_bits(out)
+    got = F.bf16_bits_to_f32(got_bits).astype(np.float64)
+    ulps = bf16_ulps_apart(got_bits, ref_bits)
+    ok = (ulps <= 1) | (np.abs(got - ref) <= G.bf16_ulp(np.abs(ref)) + sl + k * 2.0**-24 * sum_abs)
+    assert ok.all(), int((~ok).sum())
