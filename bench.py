@@ -252,7 +252,7 @@ class MoeBench:
         self.xc = torch.empty((T, H // 2), dtype=torch.uint8, device=d)
         self.xs = torch.empty((T, H // 16), dtype=torch.uint8, device=d)
         self.xg = torch.empty(1, dtype=torch.float32, device=d)
-        self.qws = u8(256)
+        self.qws = u8(max(256, fp4.fp4_moe_quantize_gather_workspace_size(cap, H, 0)))
         self.counts_d, self.offs, self.toffs = i32(E), i32(E + 1), i32(E + 1)
         self.perm, self.inv = i32(R), i32(R)
         self.scratch = u8(fp4.fp4_moe_route_scratch_bytes(R, E))

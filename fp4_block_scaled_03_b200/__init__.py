@@ -98,6 +98,7 @@ _SIGS = {
     "fp4_moe_route": (ctypes.c_int, [_P, _I64, _I32, _I32, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "fp4_moe_route_noalloc": (ctypes.c_int, [_P, _I64, _I32, _I32, _P, _P, _P, _P, _P, _P]),
     "fp4_moe_gather": (ctypes.c_int, [_P, _P, _I64, _I32, _I64, _I32, _P, _P, _P, _P, _P, _I64, _P]),
+    "fp4_moe_quantize_gather_workspace_size": (_SZ, [_I64, _I64, _U32]),
     "fp4_moe_quantize_gather": (ctypes.c_int,
                                 [_P, _I64, _I32, _I64, _I32, _P, _P, _P, _P, _P, _I64, _P, _P, _SZ, _U32, _P]),
     "fp4_moe_w13": (
@@ -189,6 +190,10 @@ def fp4_moe_route_noalloc(expert_ids, T, topk, E, counts, offsets, tile_offsets,
 def fp4_moe_gather(x_codes, x_sf, T, topk, H, E, offsets, tile_offsets, perm, a_codes, a_sf, rows_cap):
     _check(lib.fp4_moe_gather(_ptr(x_codes), _ptr(x_sf), T, topk, H, E, _ptr(offsets), _ptr(tile_offsets),
                               _ptr(perm), _ptr(a_codes), _ptr(a_sf), rows_cap, _stream()), "fp4_moe_gather")
+
+
+def fp4_moe_quantize_gather_workspace_size(rows_cap, H, flags=0):
+    return lib.fp4_moe_quantize_gather_workspace_size(rows_cap, H, flags)
 
 
 def fp4_moe_quantize_gather(x, T, topk, H, E, offsets, tile_offsets, inv, a_codes, a_sf, rows_cap, global_scale,

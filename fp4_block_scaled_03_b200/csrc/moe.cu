@@ -15,6 +15,7 @@ namespace {
 struct MoeLayout {
   size_t header, counts, offsets, tile_offsets, perm, inv, scratch, a_codes, a_sf, h_codes, h_sf, y;
   size_t h_f32, h_amax, h_g;  // dynamic h scale only (0 bytes otherwise)
+  size_t qws, qws_bytes;      // quantize+gather workspace (NVFP4: global amax + row-order scale words)
   size_t total;
   int64_t rows_cap;
 };
@@ -46,6 +47,8 @@ MoeLayout moe_layout(int64_t T, int32_t topk, int64_t H, int64_t I, int32_t E, i
   L.h_codes = take((size_t)(L.rows_cap * I / codes_per_byte));
   L.h_sf = take(fp4_sf_tiled_bytes(L.rows_cap, I));
   L.y = take((size_t)R * (size_t)H * 4);
+  L.qws_bytes = codes_per_byte == 2 ? fp4_moe_quantize_gather_workspace_size(L.rows_cap, H, 0) : 0;
+  L.qws = take(L.qws_bytes);
   L.h_f32 = take(dyn_h ? (size_t)L.rows_cap * (size_t)I * 4 : 0);
   L.h_amax = take(dyn_h ? (size_t)E * 4 : 0);
   L.h_g = take(dyn_h ? (size_t)E * 4 : 0);
@@ -93,7 +96,7 @@ fp4_status fp4_moe_grouped_gemm(const void *tokens_bf16, const int32_t *expert_i
   const uint32_t fmt = flags & (FP4_MOE_MX | FP4_MOE_W4A8);
   const uint32_t tiling = flags & FP4_MOE_PAIR_TILES;
   st = fp4_moe_quantize_gather(tokens_bf16, T, topk, H, E, I32(L.offsets), I32(L.tile_offsets), I32(L.inv),
-                               ws + L.a_codes, ws + L.a_sf, L.rows_cap, g_x, ws + L.header, 256, fmt, stream);
+                               ws + L.a_codes, ws + L.a_sf, L.rows_cap, g_x, ws + L.qws, L.qws_bytes, fmt, stream);
   if (st != FP4_OK) return st;
   fp4_moe_weights wd = *w;  // the dynamic h scale replaces the static one for w2
   if (dyn_h) {

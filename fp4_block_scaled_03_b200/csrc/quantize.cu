@@ -161,8 +161,10 @@ __device__ __forceinline__ void gather_destinations(const int32_t *__restrict__ 
 __global__ void __launch_bounds__(128) nvfp4_quantize_gather_kernel(
     const uint16_t *__restrict__ x, int64_t T, int64_t H, int32_t topk, int32_t E,
     const int32_t *__restrict__ offsets, const int32_t *__restrict__ tile_offsets, const int32_t *__restrict__ inv,
-    uint8_t *__restrict__ a_codes, uint8_t *__restrict__ a_sf, const unsigned int *__restrict__ amax_bits,
+    uint8_t *__restrict__ a_codes, uint32_t *__restrict__ sf_rows, const unsigned int *__restrict__ amax_bits,
     float *__restrict__ g_out) {
+  // scale words go row-major to sf_rows [rows][H/64] (coalesced); sf_rows_to_tiled_kernel
+  // then writes the tiled layout one whole 512-byte tile at a time
   const float g = __fdiv_rn(__uint_as_float(*amax_bits), 2688.0f);
   if (blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
   const int lane = threadIdx.x & 31;
@@ -171,11 +173,19 @@ __global__ void __launch_bounds__(128) nvfp4_quantize_gather_kernel(
   for (int64_t t = blockIdx.x * (int64_t)(blockDim.x / 32) + (threadIdx.x >> 5); t < T; t += warps) {
     int64_t dd[16];
     gather_destinations(offsets, tile_offsets, inv, E, topk, t, lane, dd);
-    for (int64_t kw = lane; kw < n_ksteps; kw += 32) {
-      const uint4 *src = reinterpret_cast<const uint4 *>(x + t * H + kw * 64);
-      uint4 v[8];
+    uint4 v[8];
+    if (lane < n_ksteps) {
+      const uint4 *src = reinterpret_cast<const uint4 *>(x + t * H + lane * 64);
 #pragma unroll
       for (int q = 0; q < 8; ++q) v[q] = __ldcs(src + q);
+    }
+    for (int64_t kw = lane; kw < n_ksteps; kw += 32) {
+      uint4 vn[8];  // the lane's next K step, in flight while this one is quantized
+      if (kw + 32 < n_ksteps) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + t * H + (kw + 32) * 64);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) vn[q] = __ldcs(src + q);
+      }
       uint32_t code[8], sfw = 0;
 #pragma unroll
       for (int blk = 0; blk < 4; ++blk) {
@@ -196,8 +206,38 @@ __global__ void __launch_bounds__(128) nvfp4_quantize_gather_kernel(
         uint4 *out = reinterpret_cast<uint4 *>(a_codes + d * (H / 2) + kw * 32);
         out[0] = make_uint4(code[0], code[1], code[2], code[3]);
         out[1] = make_uint4(code[4], code[5], code[6], code[7]);
-        *reinterpret_cast<uint32_t *>(a_sf + sf_tiled_offset(d, kw * 4, n_ksteps)) = sfw;
+        sf_rows[d * n_ksteps + kw] = sfw;
       }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v[q] = vn[q];
+    }
+  }
+}
+
+// Row-major scale words [rows][n_ksteps] -> the tiled layout: one CTA per
+// 128-row slab and 32 K steps, staged through shared memory so that every
+// 512-byte tile (32 lines x 16 bytes; line l = rows l, l+32, l+64, l+96) is
+// written whole.  Slabs past the routed rows (tile_offsets[E]) are skipped.
+__global__ void __launch_bounds__(256) sf_rows_to_tiled_kernel(const uint32_t *__restrict__ sf_rows,
+                                                               int64_t n_ksteps, const int32_t *__restrict__ tile_offsets,
+                                                               int32_t E, uint8_t *__restrict__ a_sf) {
+  __shared__ uint32_t tile[128][33];
+  const int64_t slabs = tile_offsets[E];
+  const int64_t kgroups = (n_ksteps + 31) / 32;
+  for (int64_t job = blockIdx.x; job < slabs * kgroups; job += gridDim.x) {
+    const int64_t slab = job / kgroups, k0 = (job - slab * kgroups) * 32;
+    const int kn = (int)min((int64_t)32, n_ksteps - k0);
+    __syncthreads();
+    for (int i = threadIdx.x; i < 128 * 32; i += 256) {
+      const int r = i >> 5, c = i & 31;
+      if (c < kn) tile[r][c] = sf_rows[(slab * 128 + r) * n_ksteps + k0 + c];
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < 32 * 32; i += 256) {  // line l of the tile of K step k0 + c
+      const int c = i >> 5, l = i & 31;
+      if (c < kn)
+        *reinterpret_cast<uint4 *>(a_sf + ((slab * n_ksteps + k0 + c) * 512 + l * 16)) =
+            make_uint4(tile[l][c], tile[l + 32][c], tile[l + 64][c], tile[l + 96][c]);
     }
   }
 }
@@ -661,7 +701,7 @@ fp4_status fp4_moe_quantize_gather(const void *x_bf16, int64_t T, int32_t topk, 
   if (T < 0 || topk < 1 || topk > 16 || E < 1 || E > 4096 || H <= 0 || H % 64 || (mx && H % 128))
     return FP4_ERR_UNSUPPORTED_SHAPE;
   if (rows_cap < T * topk + 127LL * E) return FP4_ERR_WORKSPACE;
-  if (!mx && ws_bytes < fp4_quantize_workspace_size()) return FP4_ERR_WORKSPACE;
+  if (ws_bytes < fp4_moe_quantize_gather_workspace_size(rows_cap, H, flags)) return FP4_ERR_WORKSPACE;
   if (!aligned16(x_bf16) || !aligned16(a_codes) || (!mx && !aligned16(workspace))) return FP4_ERR_ALIGNMENT;
   if (T == 0) return FP4_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -690,10 +730,21 @@ fp4_status fp4_moe_quantize_gather(const void *x_bf16, int64_t T, int32_t topk, 
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t need = (T + 3) / 4;  // four rows (warps) per CTA
   const int64_t grid = need < (int64_t)sms * 16 ? need : (int64_t)sms * 16;
+  uint32_t *sf_rows = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(workspace) + 256);
   nvfp4_quantize_gather_kernel<<<(unsigned)grid, 128, 0, s>>>(x, T, H, topk, E, offsets, tile_offsets, inv, a_codes,
-                                                               a_sf, amax, global_scale);
+                                                               sf_rows, amax, global_scale);
+  FP4_HOST_CHECK(cudaGetLastError());
+  const int64_t jobs = (rows_cap / 128) * ((H / 64 + 31) / 32);  // an upper bound; the kernel stops at the routed rows
+  const int64_t tgrid = jobs < (int64_t)sms * 8 ? (jobs > 0 ? jobs : 1) : (int64_t)sms * 8;
+  sf_rows_to_tiled_kernel<<<(unsigned)tgrid, 256, 0, s>>>(sf_rows, H / 64, tile_offsets, E, a_sf);
   FP4_HOST_CHECK(cudaGetLastError());
   return FP4_OK;
+}
+
+size_t fp4_moe_quantize_gather_workspace_size(int64_t rows_cap, int64_t H, uint32_t flags) {
+  if (rows_cap < 0 || H <= 0) return 0;
+  if (flags & (FP4_MOE_MX | FP4_MOE_W4A8)) return 0;  // the MX paths need none
+  return 256 + (size_t)rows_cap * (size_t)(H / 64) * 4;  // global amax, then the row-major scale words
 }
 
 }  // extern "C"

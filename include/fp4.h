@@ -318,11 +318,14 @@ fp4_status fp4_moe_gather(const uint8_t *x_codes, const uint8_t *x_sf, int64_t T
  * global scale as fp4_quantize(FP4_NV, dynamic) followed by fp4_moe_gather,
  * written straight into the expert rows (a_codes [rows_cap][H/2], tiled a_sf)
  * from the routing tables of fp4_moe_route.  global_scale: device fp32[1],
- * output.  workspace >= fp4_quantize_workspace_size() bytes.
+ * output.  workspace >= fp4_moe_quantize_gather_workspace_size(rows_cap, H,
+ * flags) bytes, 16-byte aligned (the global amax and the scale words in row
+ * order, which a second pass writes out in the tiled layout).
  * With FP4_MOE_MX: MXFP4 instead (UE8M0 per 32, tiled with 32-element blocks,
  * H % 128 == 0); global_scale and workspace are unused (may be NULL).
  * With FP4_MOE_W4A8: MXFP8 (a_codes one E4M3 byte per element, [rows_cap][H]),
  * otherwise as FP4_MOE_MX. */
+size_t fp4_moe_quantize_gather_workspace_size(int64_t rows_cap, int64_t H, uint32_t flags);
 fp4_status fp4_moe_quantize_gather(const void *x_bf16, int64_t T, int32_t topk, int64_t H, int32_t E,
                                    const int32_t *offsets, const int32_t *tile_offsets, const int32_t *inv,
                                    uint8_t *a_codes, uint8_t *a_sf, int64_t rows_cap, float *global_scale,

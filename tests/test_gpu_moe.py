@@ -378,7 +378,7 @@ def test_quantize_gather_fused_bit_exact(T, H, k, E, zipf):
     a_c = torch.zeros((cap, H // 2), dtype=torch.uint8, device="cuda")
     a_s = torch.zeros(fp4.fp4_sf_tiled_bytes(cap, H), dtype=torch.uint8, device="cuda")
     g = torch.empty(1, dtype=torch.float32, device="cuda")
-    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    ws = torch.empty(fp4.fp4_moe_quantize_gather_workspace_size(cap, H, 0), dtype=torch.uint8, device="cuda")
     fp4.fp4_moe_quantize_gather(x, T, k, H, E, r["offsets"], r["tile_offsets"], r["inv"], a_c, a_s, cap, g, ws)
     counts, offsets, perm, inv = MO.route(ids.cpu().numpy(), E)
     toff = _tile_offsets_ref(counts)
