@@ -35,6 +35,16 @@ blocks whose codes are all (signed) zeros get scale 0; codes are unchanged.
 A tensor whose exponent span would need an E4M3 power below 2^-9 cannot be
 remapped losslessly and is reported as a range error.
 
+Lossy-span fallback ("DeepSeek-V4 architecture" §6.3 says the conversion is
+lossless only while the ratio of the scale factors stays under a threshold;
+it gives no rule beyond it).  Reading: a live block whose exact E4M3 power
+2^k would fall below 2^-9 (k < -9) is re-expressed at the smallest power,
+2^-9: each element value val(c) * 2^k (in units of g) becomes the E2M1 code
+nearest to val(c) * 2^(k+9), ties to even, the sign bit kept -- the same
+rounding the NVFP4 quantizer applies -- and the block's scale is 2^-9 if any
+re-encoded magnitude is nonzero, else 0.  Every other block is remapped
+exactly as in the lossless case.
+
 MXFP8 (the W4A8 activation format: "DeepSeek-V4 FP4 QAT" §4.3 recommends FP8
 activations against FP4 weights, and §4.2 keeps the power-of-two block scale
 of the MX format).  Reading: the MXFP4 rule above with the E4M3 element
@@ -220,3 +230,50 @@ def mx_to_nv(packed, mx_scales, num_tensors=1):
         nv_sf[sl, 1::2] = sf_blk
         gs[t] = pow2_f32(e_max - 8)
     return nv_sf, gs
+
+
+def mx_to_nv_lossy(packed, mx_scales, num_tensors=1):
+    """MXFP4 -> NVFP4 remap that re-encodes the blocks below E4M3's range
+    (the lossy-span fallback above) instead of refusing the tensor.
+
+    Returns (codes uint8 [.., cols/2], nv_sf uint8 [.., cols/16],
+    g fp32 [num_tensors], lossy int64 [num_tensors] = re-encoded 32-blocks).
+    A UE8M0 NaN byte is still an error."""
+    packed = np.asarray(packed, dtype=np.uint8)
+    mx_scales = np.asarray(mx_scales, dtype=np.uint8)
+    total_rows, half_cols = packed.shape
+    cols = half_cols * 2
+    assert total_rows % num_tensors == 0
+    if np.any(mx_scales == 255):
+        raise ValueError("UE8M0 NaN scale in input")
+    rows = total_rows // num_tensors
+    codes = unpack_nibbles(packed).reshape(total_rows, cols // MX_BLOCK, MX_BLOCK).copy()
+    live = np.any((codes & 7) != 0, axis=2)
+    e = mx_scales.astype(np.int64) - 127
+    nv_sf = np.zeros((total_rows, cols // NV_BLOCK), dtype=np.uint8)
+    gs = np.zeros(num_tensors, dtype=np.float32)
+    lossy = np.zeros(num_tensors, dtype=np.int64)
+    for t in range(num_tensors):
+        r0 = t * rows
+        lt = live[r0:r0 + rows]
+        if not np.any(lt):
+            continue
+        e_max = int(np.max(e[r0:r0 + rows][lt]))
+        gs[t] = pow2_f32(e_max - 8)
+        for r in range(r0, r0 + rows):
+            for j in range(cols // MX_BLOCK):
+                if not live[r, j]:
+                    continue
+                k = int(e[r, j]) - e_max + 8
+                if k >= -9:
+                    sf = e4m3_power_of_two(k)
+                else:
+                    lossy[t] += 1
+                    # exact value in units of g * 2^-9; a power of two this small may
+                    # underflow fp32 to a signed zero, which still rounds to code 0
+                    x = (e2m1_decode(codes[r, j]) * np.ldexp(1.0, k + 9)).astype(np.float32)
+                    codes[r, j] = e2m1_encode(x)
+                    sf = e4m3_power_of_two(-9) if np.any(codes[r, j] & 7) else np.uint8(0)
+                nv_sf[r, 2 * j] = sf
+                nv_sf[r, 2 * j + 1] = sf
+    return pack_nibbles(codes.reshape(total_rows, cols)), nv_sf, gs, lossy
