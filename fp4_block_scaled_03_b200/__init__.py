@@ -28,6 +28,7 @@ FP4_GEMM_A_MXFP8 = 0x40
 FP4_GEMM_B_MXFP8 = 0x80
 FP4_MOE_W4A8 = 0x100
 FP4_MOE_DYNAMIC_H = 0x200
+FP4_MX2NV_ALLOW_LOSSY = 0x400
 FP4_MOE_MX = 0x10
 FP4_MOE_PAIR_TILES = 0x20
 
@@ -80,6 +81,7 @@ _SIGS = {
     "fp4_quantize_workspace_size": (_SZ, []),
     "fp4_quantize": (ctypes.c_int, [ctypes.c_int, _P, _I64, _I64, _I64, _P, _P, _P, _U32, _P, _SZ, _P]),
     "fp4_mx_to_nv": (ctypes.c_int, [_P, _P, _I64, _I64, _I64, _P, _P, _U32, _P]),
+    "fp4_mx_to_nv_codes": (ctypes.c_int, [_P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _U32, _P]),
     "fp4_e2m1_to_e4m3": (ctypes.c_int, [_P, _I64, _I64, _P, _P]),
     "fp4_gemm_bf16": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _I64, _P]),
     "fp4_moe_w13_h": (ctypes.c_int, [_P, _P, _P, ctypes.POINTER(MoeWeights), _I64, _I64, _I32, _P, _P, _I64, _P, _P,
@@ -322,6 +324,30 @@ def e2m1_to_e4m3(codes):
     out = torch.empty((rows, half * 2), dtype=torch.uint8, device=codes.device)
     fp4_e2m1_to_e4m3(codes, rows, half * 2, out)
     return out
+
+
+def fp4_mx_to_nv_codes(codes, mx_scales, rows, cols, num_tensors, nv_codes, nv_scales, nv_global, lossy_blocks,
+                       flags=0):
+    _check(lib.fp4_mx_to_nv_codes(_ptr(codes), _ptr(mx_scales), rows, cols, num_tensors, _ptr(nv_codes),
+                                  _ptr(nv_scales), _ptr(nv_global), _ptr(lossy_blocks), flags, _stream()),
+           "fp4_mx_to_nv_codes")
+
+
+def mx_to_nv_codes(codes, mx_scales, num_tensors, tiled=False, allow_lossy=True, out_codes=None):
+    """MX -> NV remap that writes the codes too; with allow_lossy, blocks below
+    E4M3's range are re-encoded at 2^-9.  Returns (codes, scales, g, lossy)."""
+    total_rows, half = codes.shape
+    rows, cols = total_rows // num_tensors, half * 2
+    if tiled:
+        nv = _u8(num_tensors * fp4_sf_tiled_bytes(rows, cols), codes.device)
+    else:
+        nv = torch.empty((total_rows, cols // 16), dtype=torch.uint8, device=codes.device)
+    oc = torch.empty_like(codes) if out_codes is None else out_codes
+    g = torch.empty(num_tensors, dtype=torch.float32, device=codes.device)
+    lossy = torch.empty(num_tensors, dtype=torch.int64, device=codes.device)
+    flags = (FP4_SCALE_LAYOUT_TILED if tiled else 0) | (FP4_MX2NV_ALLOW_LOSSY if allow_lossy else 0)
+    fp4_mx_to_nv_codes(codes, mx_scales, rows, cols, num_tensors, oc, nv, g, lossy, flags)
+    return oc, nv, g, lossy
 
 
 def mx_to_nv(codes, mx_scales, num_tensors, tiled=False):

@@ -508,11 +508,33 @@ __device__ __forceinline__ float pow2_f32(int e) {  // exact 2^e, e in [-149, 12
   return __uint_as_float(1u << (e + 149));
 }
 
-template <bool kTiled>
-__global__ void __launch_bounds__(kThreads) mx_to_nv_kernel(const uint8_t *__restrict__ codes,
-                                                            const uint8_t *__restrict__ mx, int64_t rows,
-                                                            int64_t cols, uint8_t *__restrict__ nv,
-                                                            float *__restrict__ nv_global, int64_t tiled_bytes) {
+// E2M1 magnitude code nearest to val(m) * 2^-d (d >= 1), ties to the even
+// code: the re-encoding of a block below E4M3's smallest power of two.
+// Magnitudes in units of 0.5 are integers (0 1 2 3 4 6 8 12), so the search
+// compares exact integer distances.
+__device__ __forceinline__ uint32_t e2m1_shift_down(uint32_t m, int d) {
+  if (d > 5) return 0;  // val(m) * 2^-6 <= 0.09375: nearest is 0
+  const int half_units[8] = {0, 1, 2, 3, 4, 6, 8, 12};
+  const int v = half_units[m];
+  uint32_t best = 0;
+  int best_dist = v;  // distance to code 0
+  for (uint32_t c = 1; c < 8; ++c) {
+    const int dist = abs(v - (half_units[c] << d));
+    if (dist < best_dist || (dist == best_dist && (c & 1u) == 0)) {
+      best = c;
+      best_dist = dist;
+    }
+  }
+  return best;
+}
+
+// kCodes: also write the codes to out_codes (which may alias `codes`) and,
+// with kLossy, re-encode the blocks below E4M3's range instead of refusing.
+template <bool kTiled, bool kCodes, bool kLossy>
+__global__ void __launch_bounds__(kThreads) mx_to_nv_kernel(const uint8_t *codes, const uint8_t *__restrict__ mx,
+                                                            int64_t rows, int64_t cols, uint8_t *__restrict__ nv,
+                                                            float *__restrict__ nv_global, int64_t tiled_bytes,
+                                                            uint8_t *out_codes, int64_t *lossy_blocks) {
   const int64_t t = blockIdx.x;
   const int64_t nb = rows * (cols / 32);
   const uint8_t *cb = codes + t * rows * (cols / 2);
@@ -545,18 +567,41 @@ __global__ void __launch_bounds__(kThreads) mx_to_nv_kernel(const uint8_t *__res
   emin = s_min[0];
   bad = s_bad[0];
   const bool any_live = emax > -1000;
-  if (bad || (any_live && emax - emin > 17)) {
+  if (bad || (!kLossy && any_live && emax - emin > 17)) {
     if (threadIdx.x == 0) nv_global[t] = __uint_as_float(0x7FC00000u);  // NaN marks a refused tensor
+    if (kCodes && lossy_blocks && threadIdx.x == 0) lossy_blocks[t] = 0;
     return;
   }
   if (threadIdx.x == 0) nv_global[t] = any_live ? pow2_f32(emax - 8) : 0.0f;
+  uint8_t *ocb = kCodes ? out_codes + t * rows * (cols / 2) : nullptr;
+  int n_lossy = 0;
   for (int64_t i = threadIdx.x; i < nb; i += blockDim.x) {
-    const uint4 c = *reinterpret_cast<const uint4 *>(cb + i * 16);
+    uint4 c = *reinterpret_cast<const uint4 *>(cb + i * 16);
     uint32_t code = 0;
     if (block_live(c)) {
-      const int k = ((int)sb[i] - 127) - emax + 8;  // in [-9, 8]
-      code = k >= -6 ? (uint32_t)((k + 7) << 3) : (1u << (k + 9));
+      const int k = ((int)sb[i] - 127) - emax + 8;  // exact while k >= -9
+      if (kLossy && k < -9) {  // re-express at 2^-9: every magnitude shrinks by 2^(k+9)
+        uint32_t w[4] = {c.x, c.y, c.z, c.w}, any = 0;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t o = 0;
+#pragma unroll
+          for (int n = 0; n < 8; ++n) {
+            const uint32_t nib = (w[q] >> (4 * n)) & 0xFu;
+            const uint32_t m = e2m1_shift_down(nib & 7u, -9 - k);
+            any |= m;
+            o |= ((nib & 8u) | m) << (4 * n);
+          }
+          w[q] = o;
+        }
+        c = make_uint4(w[0], w[1], w[2], w[3]);
+        code = any ? 0x01u : 0u;  // 2^-9, E4M3's smallest power of two
+        ++n_lossy;
+      } else {
+        code = k >= -6 ? (uint32_t)((k + 7) << 3) : (1u << (k + 9));
+      }
     }
+    if (kCodes) *reinterpret_cast<uint4 *>(ocb + i * 16) = c;
     if (kTiled) {  // block i = (row, 32-block j): 16-blocks 2j and 2j+1 are adjacent bytes
       const int64_t r = i / (cols / 32), j = i - r * (cols / 32);
       *reinterpret_cast<uint16_t *>(ob + sf_tiled_offset(r, 2 * j, cols / 64)) = (uint16_t)(code | (code << 8));
@@ -564,12 +609,35 @@ __global__ void __launch_bounds__(kThreads) mx_to_nv_kernel(const uint8_t *__res
       *reinterpret_cast<uint16_t *>(ob + 2 * i) = (uint16_t)(code | (code << 8));
     }
   }
+  if (kCodes && lossy_blocks) {
+    __shared__ int s_lossy;
+    if (threadIdx.x == 0) s_lossy = 0;
+    __syncthreads();
+    if (n_lossy) atomicAdd(&s_lossy, n_lossy);
+    __syncthreads();
+    if (threadIdx.x == 0) lossy_blocks[t] = s_lossy;
+  }
 }
 
 }  // namespace
 }  // namespace fp4
 
 using namespace fp4;
+
+// Offline remap steps are synchronous: wait for the stream and report any
+// refused tensor (a NaN global).
+static fp4_status remap_refused(const float *nv_global, int64_t num_tensors, cudaStream_t s) {
+  FP4_HOST_CHECK(cudaStreamSynchronize(s));
+  fp4_status st = FP4_OK;
+  float host[256];
+  for (int64_t i0 = 0; i0 < num_tensors; i0 += 256) {
+    const int64_t n = num_tensors - i0 < 256 ? num_tensors - i0 : 256;
+    FP4_HOST_CHECK(cudaMemcpy(host, nv_global + i0, sizeof(float) * (size_t)n, cudaMemcpyDeviceToHost));
+    for (int64_t i = 0; i < n; ++i)
+      if (host[i] != host[i]) st = FP4_ERR_RANGE;
+  }
+  return st;
+}
 
 extern "C" {
 
@@ -669,24 +737,46 @@ fp4_status fp4_mx_to_nv(const uint8_t *codes, const uint8_t *mx_scales, int64_t 
   if (!aligned16(codes) || (reinterpret_cast<uintptr_t>(nv_scales) & 1u)) return FP4_ERR_ALIGNMENT;
   if (num_tensors > 2147483647) return FP4_ERR_UNSUPPORTED_SHAPE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t tb = tiled ? (int64_t)fp4_sf_tiled_bytes(rows, cols) : 0;
   if (tiled)
-    mx_to_nv_kernel<true><<<(unsigned)num_tensors, kThreads, 0, s>>>(codes, mx_scales, rows, cols, nv_scales, nv_global,
-                                                                    (int64_t)fp4_sf_tiled_bytes(rows, cols));
+    mx_to_nv_kernel<true, false, false><<<(unsigned)num_tensors, kThreads, 0, s>>>(
+        codes, mx_scales, rows, cols, nv_scales, nv_global, tb, nullptr, nullptr);
   else
-    mx_to_nv_kernel<false><<<(unsigned)num_tensors, kThreads, 0, s>>>(codes, mx_scales, rows, cols, nv_scales,
-                                                                     nv_global, 0);
+    mx_to_nv_kernel<false, false, false><<<(unsigned)num_tensors, kThreads, 0, s>>>(
+        codes, mx_scales, rows, cols, nv_scales, nv_global, tb, nullptr, nullptr);
   FP4_HOST_CHECK(cudaGetLastError());
-  // offline step: report refused tensors (NaN globals) synchronously
-  FP4_HOST_CHECK(cudaStreamSynchronize(s));
-  fp4_status st = FP4_OK;
-  float host[256];
-  for (int64_t i0 = 0; i0 < num_tensors; i0 += 256) {
-    const int64_t n = num_tensors - i0 < 256 ? num_tensors - i0 : 256;
-    FP4_HOST_CHECK(cudaMemcpy(host, nv_global + i0, sizeof(float) * (size_t)n, cudaMemcpyDeviceToHost));
-    for (int64_t i = 0; i < n; ++i)
-      if (host[i] != host[i]) st = FP4_ERR_RANGE;
-  }
-  return st;
+  return remap_refused(nv_global, num_tensors, s);
+}
+
+fp4_status fp4_mx_to_nv_codes(const uint8_t *codes, const uint8_t *mx_scales, int64_t rows, int64_t cols,
+                              int64_t num_tensors, uint8_t *nv_codes, uint8_t *nv_scales, float *nv_global,
+                              int64_t *lossy_blocks, uint32_t flags, fp4_stream_t stream) {
+  if (!codes || !mx_scales || !nv_codes || !nv_scales || !nv_global || rows <= 0 || cols <= 0 || num_tensors <= 0)
+    return FP4_ERR_INVALID_ARG;
+  const bool tiled = flags & FP4_SCALE_LAYOUT_TILED;
+  const bool lossy = flags & FP4_MX2NV_ALLOW_LOSSY;
+  if (cols % 32 || (tiled && cols % 64)) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(codes) || !aligned16(nv_codes) || (reinterpret_cast<uintptr_t>(nv_scales) & 1u) ||
+      (reinterpret_cast<uintptr_t>(lossy_blocks) & 7u))
+    return FP4_ERR_ALIGNMENT;
+  if (num_tensors > 2147483647) return FP4_ERR_UNSUPPORTED_SHAPE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t tb = tiled ? (int64_t)fp4_sf_tiled_bytes(rows, cols) : 0;
+  const unsigned g = (unsigned)num_tensors;
+  if (tiled && lossy)
+    mx_to_nv_kernel<true, true, true><<<g, kThreads, 0, s>>>(codes, mx_scales, rows, cols, nv_scales, nv_global, tb,
+                                                            nv_codes, lossy_blocks);
+  else if (tiled)
+    mx_to_nv_kernel<true, true, false><<<g, kThreads, 0, s>>>(codes, mx_scales, rows, cols, nv_scales, nv_global, tb,
+                                                             nv_codes, lossy_blocks);
+  else if (lossy)
+    mx_to_nv_kernel<false, true, true><<<g, kThreads, 0, s>>>(codes, mx_scales, rows, cols, nv_scales, nv_global, tb,
+                                                             nv_codes, lossy_blocks);
+  else
+    mx_to_nv_kernel<false, true, false><<<g, kThreads, 0, s>>>(codes, mx_scales, rows, cols, nv_scales, nv_global,
+                                                              tb, nv_codes, lossy_blocks);
+  FP4_HOST_CHECK(cudaGetLastError());
+  return remap_refused(nv_global, num_tensors, s);
 }
 
 fp4_status fp4_moe_quantize_gather(const void *x_bf16, int64_t T, int32_t topk, int64_t H, int32_t E,

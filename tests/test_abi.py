@@ -85,6 +85,11 @@ def test_host_validation_without_gpu():
     assert L.fp4_moe_gather(A, A, 8, 2, 256, 4, A, A, A, A, A, 16, None) == 6
     # MX->NV: cols not a multiple of 32
     assert L.fp4_mx_to_nv(A, A, 4, 48, 1, A, A, 0, None) == 3
+    # MX->NV with codes: null output codes, cols % 32, misaligned codes / count buffer
+    assert L.fp4_mx_to_nv_codes(A, A, 4, 64, 1, None, A, A, None, 0x400, None) == 1
+    assert L.fp4_mx_to_nv_codes(A, A, 4, 48, 1, A, A, A, None, 0x400, None) == 3
+    assert L.fp4_mx_to_nv_codes(A, A, 4, 64, 1, A + 8, A, A, None, 0x400, None) == 2
+    assert L.fp4_mx_to_nv_codes(A, A, 4, 64, 1, A, A, A, A + 4, 0x400, None) == 2
     # FP4 -> FP8 widening: cols % 32, misaligned output, null input
     assert L.fp4_e2m1_to_e4m3(A, 4, 48, A, None) == 3
     assert L.fp4_e2m1_to_e4m3(A, 4, 64, A + 8, None) == 2

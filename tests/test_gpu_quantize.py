@@ -152,3 +152,89 @@ def test_remap_tiled_layout():
         got = LY.sf_from_mma(np_u8(nv_t[t * tb:(t + 1) * tb]), rows, cols)
         assert np.array_equal(got, rnv[t * rows:(t + 1) * rows])
     assert f32_bits_equal(g.cpu().numpy(), rg)
+
+
+def _wide_span_mx(nt, rows, cols, seed):
+    """MX codes and UE8M0 scales whose tensors span far more than 17 octaves
+    (tensor 1 stays inside the lossless span), with some dead blocks."""
+    rng = np.random.default_rng(seed)
+    codes = rng.integers(0, 256, (nt * rows, cols // 2), dtype=np.uint8)
+    e = rng.integers(-90, 40, (nt * rows, cols // 32))
+    e[rows:2 * rows] = rng.integers(-6, 8, (rows, cols // 32))
+    dead = rng.random((nt * rows, cols // 32)) < 0.05
+    for r, j in zip(*np.nonzero(dead)):
+        codes[r, 16 * j:16 * j + 16] = 0x88 if (r + j) % 2 else 0x00  # signed zeros only
+    return codes, (e + 127).astype(np.uint8)
+
+
+@pytest.mark.parametrize("tiled", [False, True])
+@pytest.mark.parametrize("inplace", [False, True])
+def test_remap_lossy_bit_exact(tiled, inplace):
+    """fp4_mx_to_nv_codes with FP4_MX2NV_ALLOW_LOSSY: codes, scales, globals
+    and re-encoded block counts equal the oracle's lossy remap bit for bit
+    (several tensors, rows not a multiple of 128, spans up to 129 octaves)."""
+    fp4 = _lib()
+    nt, rows, cols = 3, 96, 192
+    codes, sc = _wide_span_mx(nt, rows, cols, seed=11 + 2 * tiled + inplace)
+    c_d = torch.from_numpy(codes.copy()).cuda()
+    s_d = torch.from_numpy(sc).cuda()
+    oc, nv, g, lossy = fp4.mx_to_nv_codes(c_d, s_d, nt, tiled=tiled, allow_lossy=True,
+                                          out_codes=c_d if inplace else None)
+    rc, rsf, rg, rl = Q.mx_to_nv_lossy(codes, sc, nt)
+    assert np.array_equal(np_u8(oc), rc)
+    if inplace:
+        assert oc.data_ptr() == c_d.data_ptr()
+    if tiled:
+        tb = fp4.fp4_sf_tiled_bytes(rows, cols)
+        for t in range(nt):
+            got = LY.sf_from_mma(np_u8(nv[t * tb:(t + 1) * tb]), rows, cols)
+            assert np.array_equal(got, rsf[t * rows:(t + 1) * rows])
+    else:
+        assert np.array_equal(np_u8(nv), rsf)
+    assert f32_bits_equal(g.cpu().numpy(), rg)
+    assert np.array_equal(lossy.cpu().numpy(), rl)
+    assert rl[0] > 0 and rl[1] == 0 and rl[2] > 0
+    assert fp4.fp4_get_device_status() == 0
+
+
+def test_remap_codes_without_lossy_flag_matches_lossless_remap():
+    """Without the flag, fp4_mx_to_nv_codes is fp4_mx_to_nv plus a code copy:
+    the wide tensors are refused (FP4_ERR_RANGE, NaN global, codes and scales
+    untouched) and the tensor inside the span is remapped exactly."""
+    fp4 = _lib()
+    nt, rows, cols = 3, 64, 128
+    codes, sc = _wide_span_mx(nt, rows, cols, seed=5)
+    c_d = torch.from_numpy(codes).cuda()
+    s_d = torch.from_numpy(sc).cuda()
+    oc = torch.full_like(c_d, 0x5A)
+    nv = torch.full((nt * rows, cols // 16), 0xAB, dtype=torch.uint8, device="cuda")
+    g = torch.empty(nt, dtype=torch.float32, device="cuda")
+    lossy = torch.full((nt,), -1, dtype=torch.int64, device="cuda")
+    with pytest.raises(fp4.Fp4Error) as ei:
+        fp4.fp4_mx_to_nv_codes(c_d, s_d, rows, cols, nt, oc, nv, g, lossy, 0)
+    assert ei.value.code == 4
+    gh = g.cpu().numpy()
+    assert np.isnan(gh[0]) and np.isnan(gh[2])
+    sl = slice(rows, 2 * rows)
+    rnv, rg = Q.mx_to_nv(codes[sl], sc[sl], 1)
+    assert np.array_equal(np_u8(nv[sl]), rnv) and f32_bits_equal(gh[1:2], rg)
+    assert np.array_equal(np_u8(oc[sl]), codes[sl])
+    assert torch.all(oc[:rows] == 0x5A) and torch.all(nv[:rows] == 0xAB)
+    assert lossy.cpu().tolist() == [0, 0, 0]
+    assert fp4.fp4_get_device_status() == 0
+
+
+def test_remap_lossy_still_refuses_nan_scale():
+    fp4 = _lib()
+    rows, cols = 4, 64
+    c_d = torch.full((2 * rows, cols // 2), 0x11, dtype=torch.uint8, device="cuda")
+    s_d = torch.full((2 * rows, cols // 32), 127, dtype=torch.uint8, device="cuda")
+    s_d[rows, 1] = 255
+    oc = torch.empty_like(c_d)
+    nv = torch.empty((2 * rows, cols // 16), dtype=torch.uint8, device="cuda")
+    g = torch.empty(2, dtype=torch.float32, device="cuda")
+    with pytest.raises(fp4.Fp4Error) as ei:
+        fp4.fp4_mx_to_nv_codes(c_d, s_d, rows, cols, 2, oc, nv, g, None, fp4.FP4_MX2NV_ALLOW_LOSSY)
+    assert ei.value.code == 4
+    gh = g.cpu().numpy()
+    assert gh[0] == np.float32(2.0**-8) and np.isnan(gh[1])
