@@ -323,7 +323,11 @@ class MoeBench:
         fp4.fp4_moe_combine(self.y, self.inv, T, k, H, self.out)
         ev(5)
 
-    LAUNCHES_PER_STEP = 8  # 3 routing, amax, quantize+gather, w13, w2, combine
+    def launches_per_step(self):
+        """Kernels one step launches: 3 routing; quantize + gather (NVFP4:
+        tensor amax, fused quantize-gather, scale transpose; MX / W4A8: one);
+        w13 (+ the h requant with a dynamic h scale); w2; combine."""
+        return 3 + (1 if self.mx else 3) + 1 + (1 if self.dynamic_h else 0) + 1 + 1
 
     def mma_rows(self):
         """Routed rows the grouped GEMMs run through the tensor cores: each
@@ -509,7 +513,7 @@ def run_moe(args, world, rank, peaks):
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "how": "fp4_moe_grouped_gemm per step; pinned host->device inputs and device->host output on their own"
                        " streams, overlapping neighbouring steps (2 buffer sets)"},
-        "gpu_launches": (MoeBench.LAUNCHES_PER_STEP + (1 if b.dynamic_h else 0)) * args.steps,
+        "gpu_launches": b.launches_per_step() * args.steps,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -737,6 +741,7 @@ def run_quant(args, world, rank, peaks):
 
     H = 7168
     res = []
+    total_launches = 0
     for T in [1024 * 2**i for i in range(8)]:
         x = synth.activations_bf16((T, H), seed=T, device="cuda")
         c = torch.empty((T, H // 2), dtype=torch.uint8, device="cuda")
@@ -746,6 +751,7 @@ def run_quant(args, world, rank, peaks):
         ws = torch.empty(256, dtype=torch.uint8, device="cuda")
         flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
         out = {}
+        n_launch = 0
         for mode, flags, gg in (("static", fp4.FP4_STATIC_GLOBAL_SCALE, g), ("dynamic", 0, gd)):
             for _ in range(args.warmup):
                 fp4.fp4_quantize(fp4.FP4_NV, x, T, H, H, c, s, gg, flags, ws, 256)
@@ -760,7 +766,14 @@ def run_quant(args, world, rank, peaks):
                 times.append(e0.elapsed_time(e1))
             ms = sorted(times)[len(times) // 2]
             out[mode] = round(T * H * 2.5625 / (ms * 1e-3) / 1e9, 1)
-        res.append({"T": T, "static_gbs": out["static"], "dynamic_gbs": out["dynamic"]})
+            # the dynamic call is two kernels (tensor amax, then quantize): its
+            # algorithmic bytes add the amax pass's read of x (2 B / element)
+            if mode == "dynamic":
+                out["dynamic_2pass"] = round(T * H * 4.5625 / (ms * 1e-3) / 1e9, 1)
+            n_launch += args.steps * (1 if mode == "static" else 2)
+        total_launches += n_launch
+        res.append({"T": T, "static_gbs": out["static"], "dynamic_gbs": out["dynamic"],
+                    "dynamic_gbs_incl_amax_pass": out["dynamic_2pass"]})
         del x, c, s, flush
     top = res[-1]
     return {"metric": METRIC, "value": top["static_gbs"], "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -769,7 +782,8 @@ def run_quant(args, world, rank, peaks):
             "config": {"workload": "NVFP4 activation quantize bf16 [T,7168], T=1k..128k", "l2": "flushed"},
             "roofline": {"bound": "hbm", "achieved": top["static_gbs"], "peak": peaks["hbm"], "unit": "GB/s",
                          "frac": round(top["static_gbs"] / peaks["hbm"], 4), "traffic": None},
-            "sweep": res, "gpu_launches": None}
+            "sweep": res, "gpu_launches": total_launches,
+            "note": "timed region per call: one fp4_quantize; static = 1 kernel, dynamic = tensor amax + quantize"}
 
 
 # ---------------------------------------------------------------------------
