@@ -112,6 +112,12 @@ _SIGS = {
         [_P, _P, ctypes.POINTER(MoeWeights), _I64, _I64, _I32, _P, _P, _P, _P, _P, _I64, _P, _U32, _P],
     ),
     "fp4_moe_combine": (ctypes.c_int, [_P, _P, _I64, _I32, _I64, _P, _P]),
+    "fp4_amax_bf16": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P]),
+    "fp4_nv_global_scale": (ctypes.c_int, [_P, _I64, _P, _P]),
+    "fp4_moe_ep_record_bytes": (_SZ, [_I64]),
+    "fp4_moe_ep_pack": (ctypes.c_int, [_P, _P, _I64, _I32, _I64, _P, _P, _P, _I64, _I32, _P, _P]),
+    "fp4_moe_ep_unpack": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P, _P, _P]),
+    "fp4_gather_rows": (ctypes.c_int, [_P, _I64, _P, _I64, _P, _P]),
     "fp4_get_device_status": (ctypes.c_int, [_P]),
     "fp4_set_wait_limit_ns": (None, [ctypes.c_uint64]),
 }
@@ -231,6 +237,32 @@ def fp4_moe_w2(h_codes, h_sf, w, H, I, E, counts, offsets, tile_offsets, perm, t
 
 def fp4_moe_combine(y, inv, T, topk, H, out):
     _check(lib.fp4_moe_combine(_ptr(y), _ptr(inv), T, topk, H, _ptr(out), _stream()), "fp4_moe_combine")
+
+
+def fp4_amax_bf16(x, rows, cols, ld, amax_bits):
+    _check(lib.fp4_amax_bf16(_ptr(x), rows, cols, ld, _ptr(amax_bits), _stream()), "fp4_amax_bf16")
+
+
+def fp4_nv_global_scale(amax_bits, n, g):
+    _check(lib.fp4_nv_global_scale(_ptr(amax_bits), n, _ptr(g), _stream()), "fp4_nv_global_scale")
+
+
+def fp4_moe_ep_record_bytes(H):
+    return lib.fp4_moe_ep_record_bytes(H)
+
+
+def fp4_moe_ep_pack(x_codes, x_sf, T, topk, H, expert_ids, topk_weights, perm, R, experts_per_rank, records):
+    _check(lib.fp4_moe_ep_pack(_ptr(x_codes), _ptr(x_sf), T, topk, H, _ptr(expert_ids), _ptr(topk_weights),
+                               _ptr(perm), R, experts_per_rank, _ptr(records), _stream()), "fp4_moe_ep_pack")
+
+
+def fp4_moe_ep_unpack(records, R, H, codes, sf, weights, expert_ids):
+    _check(lib.fp4_moe_ep_unpack(_ptr(records), R, H, _ptr(codes), _ptr(sf), _ptr(weights), _ptr(expert_ids),
+                                 _stream()), "fp4_moe_ep_unpack")
+
+
+def fp4_gather_rows(src, row_bytes, idx, n, dst):
+    _check(lib.fp4_gather_rows(_ptr(src), row_bytes, _ptr(idx), n, _ptr(dst), _stream()), "fp4_gather_rows")
 
 
 def fp4_moe_grouped_gemm(tokens, expert_ids, topk_weights, T, topk, w, H, I, E, out, workspace, flags=0,

@@ -1,0 +1,143 @@
+// Expert-parallel dispatch and return of routed rows.
+//
+// "DeepSeek-V4 architecture", §6.1: with the experts split across GPUs, each
+// routed token row travels to the GPU that holds its expert and the expert's
+// output row travels back, by all-to-all exchanges.  Here the experts are
+// split into equal contiguous ranges, one per rank; a row goes out as one
+// fixed-size record -- its NVFP4 codes and block scales (0.5625 B per
+// element, the format the GEMMs read) plus its routing weight and local
+// expert id -- so that one all-to-all moves everything the owner needs.
+//
+//   record = codes [H/2] | scales [H/16] (E4M3, canonical) | weight fp32 |
+//            local expert int32 | 8 zero bytes          (a multiple of 16 B)
+//
+// The kernels only move bytes: a warp per record (or row), 16-byte vectors.
+#include "common.cuh"
+
+namespace fp4 {
+namespace {
+
+constexpr int kWarps = 8;  // warps per CTA
+
+int64_t record_bytes(int64_t H) { return H / 2 + H / 16 + 16; }
+
+int grid_rows(int64_t n) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t need = (n + kWarps - 1) / kWarps;
+  const int64_t cap = (int64_t)sms * 8;
+  return (int)(need < cap ? (need < 1 ? 1 : need) : cap);
+}
+
+bool al16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Record i <- token perm[i] / topk of the quantized x, with that slot's
+// weight and its expert's index inside the owner's range.
+__global__ void __launch_bounds__(32 * kWarps)
+    ep_pack_kernel(const uint4 *__restrict__ codes, const uint4 *__restrict__ sf, int32_t topk, int64_t H,
+                   const int32_t *__restrict__ ids, const float *__restrict__ w, const int32_t *__restrict__ perm,
+                   int64_t R, int32_t e_local, uint4 *__restrict__ rec) {
+  const int lane = threadIdx.x & 31;
+  const int64_t nc = H / 32, ns = H / 256, nr = nc + ns + 1;  // 16-byte chunks
+  for (int64_t i = blockIdx.x * (int64_t)kWarps + (threadIdx.x >> 5); i < R; i += (int64_t)gridDim.x * kWarps) {
+    const int32_t j = perm[i];
+    const int64_t t = j / topk;
+    uint4 *out = rec + i * nr;
+    for (int64_t c = lane; c < nc; c += 32) out[c] = codes[t * nc + c];
+    for (int64_t c = lane; c < ns; c += 32) out[nc + c] = sf[t * ns + c];
+    if (lane == 0) {
+      const float wt = w ? w[j] : 1.0f;
+      out[nc + ns] = make_uint4(__float_as_uint(wt), (uint32_t)(ids[j] % e_local), 0u, 0u);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(32 * kWarps)
+    ep_unpack_kernel(const uint4 *__restrict__ rec, int64_t R, int64_t H, uint4 *__restrict__ codes,
+                     uint4 *__restrict__ sf, float *__restrict__ w, int32_t *__restrict__ ids) {
+  const int lane = threadIdx.x & 31;
+  const int64_t nc = H / 32, ns = H / 256, nr = nc + ns + 1;
+  for (int64_t i = blockIdx.x * (int64_t)kWarps + (threadIdx.x >> 5); i < R; i += (int64_t)gridDim.x * kWarps) {
+    const uint4 *in = rec + i * nr;
+    for (int64_t c = lane; c < nc; c += 32) codes[i * nc + c] = in[c];
+    for (int64_t c = lane; c < ns; c += 32) sf[i * ns + c] = in[nc + c];
+    if (lane == 0) {
+      const uint4 tail = in[nc + ns];
+      w[i] = __uint_as_float(tail.x);
+      ids[i] = (int32_t)tail.y;
+    }
+  }
+}
+
+// dst row i <- src row idx[i] (rows of n16 16-byte chunks).
+__global__ void __launch_bounds__(32 * kWarps)
+    gather_rows_kernel(const uint4 *__restrict__ src, int64_t n16, const int32_t *__restrict__ idx, int64_t n,
+                       uint4 *__restrict__ dst) {
+  const int lane = threadIdx.x & 31;
+  for (int64_t i = blockIdx.x * (int64_t)kWarps + (threadIdx.x >> 5); i < n; i += (int64_t)gridDim.x * kWarps) {
+    const uint4 *in = src + (int64_t)idx[i] * n16;
+    uint4 *out = dst + i * n16;
+    for (int64_t c = lane; c < n16; c += 32) out[c] = __ldcs(in + c);
+  }
+}
+
+}  // namespace
+}  // namespace fp4
+
+using namespace fp4;
+
+extern "C" {
+
+size_t fp4_moe_ep_record_bytes(int64_t H) { return H > 0 ? (size_t)record_bytes(H) : 0; }
+
+fp4_status fp4_moe_ep_pack(const uint8_t *x_codes, const uint8_t *x_sf, int64_t T, int32_t topk, int64_t H,
+                           const int32_t *expert_ids, const float *topk_weights, const int32_t *perm, int64_t R,
+                           int32_t experts_per_rank, uint8_t *records, fp4_stream_t stream) {
+  if (T < 0 || R < 0 || topk < 1 || topk > 16 || experts_per_rank < 1 || H <= 0) return FP4_ERR_INVALID_ARG;
+  if (H % 256) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (R > T * topk) return FP4_ERR_INVALID_ARG;
+  if (R == 0) return FP4_OK;
+  if (!x_codes || !x_sf || !expert_ids || !perm || !records) return FP4_ERR_INVALID_ARG;
+  if (!al16(x_codes) || !al16(x_sf) || !al16(records)) return FP4_ERR_ALIGNMENT;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  ep_pack_kernel<<<grid_rows(R), 32 * kWarps, 0, s>>>(reinterpret_cast<const uint4 *>(x_codes),
+                                                     reinterpret_cast<const uint4 *>(x_sf), topk, H, expert_ids,
+                                                     topk_weights, perm, R, experts_per_rank,
+                                                     reinterpret_cast<uint4 *>(records));
+  FP4_HOST_CHECK(cudaGetLastError());
+  return FP4_OK;
+}
+
+fp4_status fp4_moe_ep_unpack(const uint8_t *records, int64_t R, int64_t H, uint8_t *codes, uint8_t *sf,
+                             float *weights, int32_t *expert_ids, fp4_stream_t stream) {
+  if (R < 0 || H <= 0) return FP4_ERR_INVALID_ARG;
+  if (H % 256) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (R == 0) return FP4_OK;
+  if (!records || !codes || !sf || !weights || !expert_ids) return FP4_ERR_INVALID_ARG;
+  if (!al16(records) || !al16(codes) || !al16(sf) || (reinterpret_cast<uintptr_t>(weights) & 3u) ||
+      (reinterpret_cast<uintptr_t>(expert_ids) & 3u))
+    return FP4_ERR_ALIGNMENT;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  ep_unpack_kernel<<<grid_rows(R), 32 * kWarps, 0, s>>>(reinterpret_cast<const uint4 *>(records), R, H,
+                                                       reinterpret_cast<uint4 *>(codes), reinterpret_cast<uint4 *>(sf),
+                                                       weights, expert_ids);
+  FP4_HOST_CHECK(cudaGetLastError());
+  return FP4_OK;
+}
+
+fp4_status fp4_gather_rows(const void *src, int64_t row_bytes, const int32_t *idx, int64_t n, void *dst,
+                           fp4_stream_t stream) {
+  if (n < 0 || row_bytes <= 0) return FP4_ERR_INVALID_ARG;
+  if (row_bytes % 16) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (n == 0) return FP4_OK;
+  if (!src || !idx || !dst) return FP4_ERR_INVALID_ARG;
+  if (!al16(src) || !al16(dst)) return FP4_ERR_ALIGNMENT;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  gather_rows_kernel<<<grid_rows(n), 32 * kWarps, 0, s>>>(reinterpret_cast<const uint4 *>(src), row_bytes / 16, idx, n,
+                                                         reinterpret_cast<uint4 *>(dst));
+  FP4_HOST_CHECK(cudaGetLastError());
+  return FP4_OK;
+}
+
+}  // extern "C"

@@ -72,6 +72,13 @@ __global__ void __launch_bounds__(kThreads) amax_bf16_kernel(const uint16_t *__r
   }
 }
 
+// g = amax / (448 * 6), one fp32 division, as the dynamic quantizer takes it.
+__global__ void __launch_bounds__(kThreads) global_scale_kernel(const uint32_t *__restrict__ amax_bits, int64_t n,
+                                                                float *__restrict__ g) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    g[i] = __fdiv_rn(__uint_as_float(amax_bits[i]), 2688.0f);
+}
+
 // ---- NVFP4 quantize: one thread per 16-element block -----------------------
 template <bool kTiled>
 __global__ void __launch_bounds__(kThreads) nvfp4_quantize_kernel(
@@ -692,6 +699,31 @@ fp4_status fp4_quantize(fp4_format fmt, const void *x_bf16, int64_t rows, int64_
     nvfp4_quantize_kernel<true><<<grid, kThreads, 0, s>>>(x, rows, cols, ld, codes, scales, amax, global_scale, g_in);
   else
     nvfp4_quantize_kernel<false><<<grid, kThreads, 0, s>>>(x, rows, cols, ld, codes, scales, amax, global_scale, g_in);
+  FP4_HOST_CHECK(cudaGetLastError());
+  return FP4_OK;
+}
+
+fp4_status fp4_amax_bf16(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld, uint32_t *amax_bits,
+                         fp4_stream_t stream) {
+  if (!amax_bits || rows < 0 || cols <= 0 || ld < cols) return FP4_ERR_INVALID_ARG;
+  if (cols % 8) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (rows > 0 && !x_bf16) return FP4_ERR_INVALID_ARG;
+  if ((rows > 0 && !aligned16(x_bf16)) || (ld * 2) % 16 || (reinterpret_cast<uintptr_t>(amax_bits) & 3u))
+    return FP4_ERR_ALIGNMENT;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  FP4_HOST_CHECK(cudaMemsetAsync(amax_bits, 0, sizeof(uint32_t), s));
+  if (rows == 0) return FP4_OK;
+  amax_bf16_kernel<<<grid_for(rows * (cols / 8)), kThreads, 0, s>>>(static_cast<const uint16_t *>(x_bf16), rows, cols,
+                                                                    ld, amax_bits);
+  FP4_HOST_CHECK(cudaGetLastError());
+  return FP4_OK;
+}
+
+fp4_status fp4_nv_global_scale(const uint32_t *amax_bits, int64_t n, float *g, fp4_stream_t stream) {
+  if (!amax_bits || !g || n < 0) return FP4_ERR_INVALID_ARG;
+  if (n == 0) return FP4_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  global_scale_kernel<<<grid_for(n), kThreads, 0, s>>>(amax_bits, n, g);
   FP4_HOST_CHECK(cudaGetLastError());
   return FP4_OK;
 }

@@ -1,0 +1,191 @@
+"""Expert-parallel MoE layer: one process per GPU, the experts split into
+equal contiguous ranges, routed rows exchanged by all-to-all.
+
+"DeepSeek-V4 architecture", §6.1 splits the experts across GPUs and moves
+each routed token to its expert's GPU and the expert output back.  Here one
+layer step on every rank is:
+
+  1. tensor amax of this rank's tokens; max over the ranks (all-reduce);
+     g = amax / (448*6).  Every rank quantizes with the same g, the scale the
+     1-GPU layer would take over the concatenation of all ranks' tokens.
+  2. NVFP4-quantize x with g; route over all E experts.  The rows bound for
+     rank d are a contiguous range of the routed (expert, token, slot) order;
+     pack them as fixed-size records (codes, scales, routing weight, local
+     expert id: fp4_moe_ep_pack).
+  3. all-to-all of the per-rank row counts, then of the records.
+  4. unpack; route the received rows over the local experts (one slot each);
+     gather them into expert tiles; grouped w13 (SwiGLU + h requant) and w2
+     (routing weight) on tcgen05; put the outputs back in received order.
+  5. all-to-all of the fp32 output rows back to their senders: they arrive in
+     the sender's routed order, so the fixed-order combine finishes the layer.
+
+Received rows of one expert stay in (source rank, token, slot) order, which
+is the 1-GPU layer's (expert, token, slot) order over the concatenated
+tokens; every row meets the same kernels with the same inputs, so the
+result equals the 1-GPU layer's bit for bit.
+
+The collectives are torch.distributed's (NCCL over NVLink on GPUs).  Remote
+rows always land in local memory before a kernel reads them.  The compute
+steps are the library's kernels (``CudaOps``); the orchestration takes any
+object with the same four methods, so its exchange logic can also run on CPU
+ranks."""
+import torch
+import torch.distributed as dist
+
+from . import (FP4_NV, FP4_STATIC_GLOBAL_SCALE, MoeWeightSet, _u8, fp4_amax_bf16, fp4_gather_rows,
+               fp4_moe_combine, fp4_moe_ep_pack, fp4_moe_ep_record_bytes, fp4_moe_ep_unpack, fp4_moe_gather,
+               fp4_moe_route, fp4_moe_route_scratch_bytes, fp4_moe_w13, fp4_moe_w2, fp4_nv_global_scale,
+               fp4_quantize, fp4_sf_tiled_bytes, moe_rows_cap)
+
+
+def expert_range(E, world, rank):
+    """The experts rank `rank` owns: [rank*E/world, (rank+1)*E/world)."""
+    if E % world:
+        raise ValueError(f"{E} experts do not split evenly over {world} ranks")
+    epr = E // world
+    return rank * epr, (rank + 1) * epr
+
+
+def local_weights(w, E, I, H, world, rank):
+    """Views of a whole layer's MoeWeightSet restricted to this rank's
+    experts (each expert's rows and tiled scales are contiguous)."""
+    e0, e1 = expert_range(E, world, rank)
+    s13 = fp4_sf_tiled_bytes(2 * I, H)
+    s2 = fp4_sf_tiled_bytes(H, I)
+    return MoeWeightSet(w.w13_codes[e0 * 2 * I:e1 * 2 * I], w.w13_sf[e0 * s13:e1 * s13], w.w13_g[e0:e1],
+                        w.w2_codes[e0 * H:e1 * H], w.w2_sf[e0 * s2:e1 * s2], w.w2_g[e0:e1], w.h_g[e0:e1])
+
+
+class TorchComm:
+    """The exchange steps over a torch.distributed process group.  NCCL moves
+    device tensors directly; another backend (gloo) gets host copies."""
+
+    def __init__(self, group=None):
+        self.group = group
+        self.rank = dist.get_rank(group)
+        self.world = dist.get_world_size(group)
+        self.host_staging = dist.get_backend(group) != "nccl"
+
+    def _stage(self, t):
+        return t.cpu() if self.host_staging and t.is_cuda else t
+
+    def all_reduce_max_(self, t):
+        s = self._stage(t)
+        dist.all_reduce(s, op=dist.ReduceOp.MAX, group=self.group)
+        if s is not t:
+            t.copy_(s)
+        return t
+
+    def all_to_all(self, send, send_rows, recv_rows):
+        """Rows send[sum(send_rows[:d]) : +send_rows[d]] go to rank d; the
+        result holds recv_rows[s] rows from each rank s, in rank order."""
+        s = self._stage(send.contiguous())
+        recv = s.new_empty((sum(recv_rows),) + tuple(send.shape[1:]))
+        dist.all_to_all_single(recv, s, output_split_sizes=list(recv_rows), input_split_sizes=list(send_rows),
+                               group=self.group)
+        return recv.to(send.device) if recv.device != send.device else recv
+
+    def exchange_counts(self, send_rows):
+        """Each rank's row counts for every destination -> the counts every
+        source will send here."""
+        dev = "cuda" if not self.host_staging else "cpu"
+        s = torch.tensor(list(send_rows), dtype=torch.int64, device=dev)
+        r = torch.empty_like(s)
+        dist.all_to_all_single(r, s, group=self.group)
+        return [int(v) for v in r.tolist()]
+
+
+class CudaOps:
+    """The compute steps of the EP layer on this rank's GPU, all in libfp4."""
+
+    def __init__(self, w_local, H, I, E, world, rank):
+        self.w, self.H, self.I, self.E = w_local, H, I, E
+        self.world, self.rank = world, rank
+        self.epr = E // world
+        self.rec_bytes = fp4_moe_ep_record_bytes(H)
+
+    def amax(self, x):
+        T, H = x.shape
+        a = torch.empty(1, dtype=torch.int32, device=x.device)
+        fp4_amax_bf16(x, T, H, x.stride(0), a)
+        return a
+
+    def dispatch(self, x, amax, expert_ids, topk_weights):
+        """Quantize with the shared scale, route over all experts and pack
+        the routed rows as records: (records, rows per destination, state)."""
+        T, H = x.shape
+        k = expert_ids.shape[1]
+        dev = x.device
+        g = torch.empty(1, dtype=torch.float32, device=dev)
+        fp4_nv_global_scale(amax, 1, g)
+        codes = torch.empty((T, H // 2), dtype=torch.uint8, device=dev)
+        sf = torch.empty((T, H // 16), dtype=torch.uint8, device=dev)
+        if T:
+            fp4_quantize(FP4_NV, x, T, H, x.stride(0), codes, sf, g, FP4_STATIC_GLOBAL_SCALE, None, 0)
+        R = T * k
+        counts = torch.empty(self.E, dtype=torch.int32, device=dev)
+        offsets = torch.empty(self.E + 1, dtype=torch.int32, device=dev)
+        toffs = torch.empty(self.E + 1, dtype=torch.int32, device=dev)
+        perm = torch.empty(max(R, 1), dtype=torch.int32, device=dev)
+        inv = torch.empty(max(R, 1), dtype=torch.int32, device=dev)
+        scratch = _u8(fp4_moe_route_scratch_bytes(R, self.E), dev)
+        fp4_moe_route(expert_ids, T, k, self.E, counts, offsets, toffs, perm, inv, scratch)
+        bounds = offsets[::self.epr].tolist()  # one host read: the all-to-all needs the split sizes
+        send_rows = [bounds[d + 1] - bounds[d] for d in range(self.world)]
+        records = _u8(max(R, 1) * self.rec_bytes, dev).view(max(R, 1), self.rec_bytes)[:R]
+        fp4_moe_ep_pack(codes, sf, T, k, H, expert_ids, topk_weights, perm, R, self.epr, records)
+        return records, send_rows, {"g": g, "inv": inv, "T": T, "k": k}
+
+    def experts(self, records, state):
+        """This rank's experts on the received records; the fp32 output rows
+        come back in received order."""
+        H, I, E = self.H, self.I, self.epr
+        dev = records.device
+        R = records.shape[0]
+        y_ret = torch.empty((R, H), dtype=torch.float32, device=dev)
+        if R == 0:
+            return y_ret
+        codes = torch.empty((R, H // 2), dtype=torch.uint8, device=dev)
+        sf = torch.empty((R, H // 16), dtype=torch.uint8, device=dev)
+        wts = torch.empty(R, dtype=torch.float32, device=dev)
+        ids = torch.empty(R, dtype=torch.int32, device=dev)
+        fp4_moe_ep_unpack(records, R, H, codes, sf, wts, ids)
+        counts = torch.empty(E, dtype=torch.int32, device=dev)
+        offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+        toffs = torch.empty(E + 1, dtype=torch.int32, device=dev)
+        perm = torch.empty(R, dtype=torch.int32, device=dev)
+        inv = torch.empty(R, dtype=torch.int32, device=dev)
+        fp4_moe_route(ids.view(R, 1), R, 1, E, counts, offsets, toffs, perm, inv,
+                      _u8(fp4_moe_route_scratch_bytes(R, E), dev))
+        cap = moe_rows_cap(R, 1, E)
+        a_c = torch.empty((cap, H // 2), dtype=torch.uint8, device=dev)
+        a_s = _u8(fp4_sf_tiled_bytes(cap, H), dev)
+        fp4_moe_gather(codes, sf, R, 1, H, E, offsets, toffs, perm, a_c, a_s, cap)
+        h_c = torch.empty((cap, I // 2), dtype=torch.uint8, device=dev)
+        h_s = _u8(fp4_sf_tiled_bytes(cap, I), dev)
+        fp4_moe_w13(a_c, a_s, state["g"], self.w, H, I, E, counts, toffs, cap, h_c, h_s)
+        y = torch.empty((R, H), dtype=torch.float32, device=dev)
+        fp4_moe_w2(h_c, h_s, self.w, H, I, E, counts, offsets, toffs, perm, wts, cap, y)
+        fp4_gather_rows(y, H * 4, inv, R, y_ret)  # received row i was routed to row inv[i]
+        return y_ret
+
+    def combine(self, y, state):
+        T, k, H = state["T"], state["k"], self.H
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=y.device)
+        if T:
+            fp4_moe_combine(y, state["inv"], T, k, H, out)
+        return out
+
+
+def moe_layer_ep(x, expert_ids, topk_weights, ops, comm):
+    """One expert-parallel MoE layer step on this rank: this rank's tokens x
+    [T, H] bf16 with their top-k expert ids (global) and weights -> bf16
+    [T, H].  Every rank calls it once per step (the collectives pair up)."""
+    amax = ops.amax(x)
+    comm.all_reduce_max_(amax)
+    records, send_rows, state = ops.dispatch(x, amax, expert_ids, topk_weights)
+    recv_rows = comm.exchange_counts(send_rows)
+    recv = comm.all_to_all(records, send_rows, recv_rows)
+    y_ret = ops.experts(recv, state)
+    y = comm.all_to_all(y_ret, recv_rows, send_rows)
+    return ops.combine(y, state)

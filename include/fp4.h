@@ -134,6 +134,20 @@ fp4_status fp4_quantize(fp4_format fmt, const void *x_bf16, int64_t rows, int64_
  * touched: an MXFP4 tensor's UE8M0 scales serve the widened MXFP8 tensor as
  * they are.  cols % 32 == 0; both pointers 16-byte aligned.  Asynchronous.
  */
+/*
+ * fp4_amax_bf16 -- *amax_bits = max |x| over a bf16 [rows, cols] matrix (row
+ * stride ld elements), as fp32 bits; 0 for rows == 0.  This is pass 1 of the
+ * dynamic NVFP4 quantizer ["DeepSeek-V4.1-Flash-NVFP4" §二: the tensor scale
+ * comes from the tensor's amax], exposed so that several ranks can combine
+ * their amax (an integer max of the bits: amax >= 0) before quantizing with
+ * one shared scale.  cols % 8 == 0; x 16-byte aligned, ld*2 % 16 == 0.
+ * fp4_nv_global_scale -- g[i] = amax(i) / (448*6), one fp32 division, from n
+ * amax values given as fp32 bits: the scale the dynamic quantizer would use.
+ */
+fp4_status fp4_amax_bf16(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld, uint32_t *amax_bits,
+                         fp4_stream_t stream);
+fp4_status fp4_nv_global_scale(const uint32_t *amax_bits, int64_t n, float *g, fp4_stream_t stream);
+
 fp4_status fp4_e2m1_to_e4m3(const uint8_t *codes_e2m1, int64_t rows, int64_t cols, uint8_t *codes_e4m3,
                             fp4_stream_t stream);
 
@@ -407,6 +421,39 @@ fp4_status fp4_moe_w2(const uint8_t *h_codes, const uint8_t *h_sf, const fp4_moe
  * inv < 0 contributes nothing).  H % 16 == 0. */
 fp4_status fp4_moe_combine(const float *y, const int32_t *inv, int64_t T, int32_t topk, int64_t H,
                            void *out_bf16, fp4_stream_t stream);
+
+/*
+ * Expert parallelism ["DeepSeek-V4 architecture" §6.1: experts split across
+ * GPUs, routed rows dispatched to their expert's GPU and the outputs
+ * returned, by all-to-all].  Experts are split into equal contiguous ranges
+ * of `experts_per_rank`; rank r owns experts [r*epr, (r+1)*epr).  After
+ * fp4_moe_route over all experts, the rows bound for rank r are the
+ * contiguous range perm[offsets[r*epr] .. offsets[(r+1)*epr]) of the routed
+ * order, so the send buffer of an all-to-all is the records in routed order.
+ *
+ * A record (fp4_moe_ep_record_bytes(H) = H/2 + H/16 + 16 bytes) holds one
+ * routed row: its NVFP4 codes [H/2], its E4M3 block scales [H/16] in the
+ * canonical layout, its routing weight (fp32; 1.0 if topk_weights is NULL),
+ * its expert's index within the owner's range (int32), and 8 zero bytes.
+ *
+ * fp4_moe_ep_pack -- records[i] for i < R from token perm[i]/topk of x
+ *   (x_codes [T][H/2], x_sf canonical [T][H/16] from fp4_quantize with one
+ *   global scale shared by all ranks), expert_ids/topk_weights [T*topk].
+ * fp4_moe_ep_unpack -- the inverse on the receiving rank: codes [R][H/2],
+ *   sf [R][H/16], weights [R], expert_ids [R] (local indices).
+ * fp4_gather_rows -- dst row i = src row idx[i] for i < n, rows of row_bytes
+ *   (a multiple of 16); used to put expert outputs back in received order.
+ * H % 256 == 0; buffers 16-byte aligned (weights and ids 4-byte).  R, n == 0
+ * launch nothing.  Asynchronous on `stream`.
+ */
+size_t fp4_moe_ep_record_bytes(int64_t H);
+fp4_status fp4_moe_ep_pack(const uint8_t *x_codes, const uint8_t *x_sf, int64_t T, int32_t topk, int64_t H,
+                           const int32_t *expert_ids, const float *topk_weights, const int32_t *perm, int64_t R,
+                           int32_t experts_per_rank, uint8_t *records, fp4_stream_t stream);
+fp4_status fp4_moe_ep_unpack(const uint8_t *records, int64_t R, int64_t H, uint8_t *codes, uint8_t *sf,
+                             float *weights, int32_t *expert_ids, fp4_stream_t stream);
+fp4_status fp4_gather_rows(const void *src, int64_t row_bytes, const int32_t *idx, int64_t n, void *dst,
+                           fp4_stream_t stream);
 
 /* Synchronize `stream`, then read and clear this device's status word
  * (FP4_OK if no device-side error was recorded since the last read). */

@@ -1,0 +1,93 @@
+"""The four compute steps of the expert-parallel layer (amax, dispatch,
+experts, combine) written with the oracle, for running the EP orchestration
+on CPU ranks (gloo).  Records are fp64 rows [dequantized x row | routing
+weight | local expert id]; the arithmetic is the oracle's, row by row, so a
+row's result does not depend on which other rows share its rank."""
+import numpy as np
+import torch
+
+from oracle import formats as F
+from oracle import moe as MO
+from oracle import quant as Q
+
+
+class OracleWeights:
+    """NVFP4 experts quantized by the oracle from seeded fp32 weights."""
+
+    def __init__(self, E, H, I, seed):
+        rng = np.random.default_rng(seed)
+        self.w1, self.w3, self.w2 = [], [], []
+        for _ in range(E):
+            for lst, shape in ((self.w1, (I, H)), (self.w3, (I, H)), (self.w2, (H, I))):
+                w = (rng.standard_normal(shape) * 0.05).astype(np.float32)
+                c, s, g = Q.nvfp4_quantize(w)
+                lst.append(Q.nvfp4_dequantize(c, s, g))
+        self.h_g = np.float32(2e-3)
+
+
+class OracleOps:
+    def __init__(self, weights, H, E, world, rank):
+        self.wt, self.H, self.E = weights, H, E
+        self.world, self.rank = world, rank
+        self.epr = E // world
+
+    def amax(self, x):
+        a = np.float32(np.abs(x.float().numpy()).max()) if x.shape[0] else np.float32(0)
+        return torch.tensor([int(a.view(np.uint32))], dtype=torch.int32)
+
+    def dispatch(self, x, amax, expert_ids, topk_weights):
+        T, H = x.shape
+        k = expert_ids.shape[1]
+        g = np.float32(np.uint32(amax.item()).view(np.float32) / np.float32(2688.0))
+        if T:
+            c, s, _ = Q.nvfp4_quantize(x.float().numpy(), g=g)
+            x_dq = Q.nvfp4_dequantize(c, s, g)
+        else:
+            x_dq = np.zeros((0, H))
+        ids = expert_ids.numpy().astype(np.int64)
+        counts, offsets, perm, inv = MO.route(ids, self.E)
+        send_rows = [int(offsets[(d + 1) * self.epr] - offsets[d * self.epr]) for d in range(self.world)]
+        flat_ids = ids.reshape(-1)
+        w = topk_weights.numpy().reshape(-1).astype(np.float64)
+        rec = np.zeros((T * k, H + 2))
+        for i, j in enumerate(perm):
+            rec[i, :H] = x_dq[j // k]
+            rec[i, H] = w[j]
+            rec[i, H + 1] = flat_ids[j] % self.epr
+        return torch.from_numpy(rec), send_rows, {"inv": inv, "T": T, "k": k}
+
+    def experts(self, records, state):
+        rec = records.numpy()
+        H = self.H
+        y = np.zeros((rec.shape[0], H))
+        e0 = self.rank * self.epr
+        for i in range(rec.shape[0]):
+            e = e0 + int(rec[i, H + 1])
+            r = MO.expert_ffn_ref(rec[i:i + 1, :H], self.wt.w1[e], self.wt.w3[e], self.wt.w2[e], self.wt.h_g)
+            y[i] = rec[i, H] * r["y"][0]
+        return torch.from_numpy(y)
+
+    def combine(self, y, state):
+        if state["T"] == 0:
+            return torch.zeros((0, self.H), dtype=torch.int32)
+        _, bits = MO.combine_ref(y.numpy(), state["inv"])
+        return torch.from_numpy(bits.astype(np.int32))
+
+
+class LocalComm:
+    """A world of one: every exchange is the identity."""
+
+    rank, world = 0, 1
+
+    def all_reduce_max_(self, t):
+        return t
+
+    def exchange_counts(self, send_rows):
+        return list(send_rows)
+
+    def all_to_all(self, send, send_rows, recv_rows):
+        return send
+
+
+def bf16_bits_to_f64(bits):
+    return F.bf16_bits_to_f32(np.asarray(bits, dtype=np.uint16)).astype(np.float64)

@@ -90,6 +90,17 @@ def test_host_validation_without_gpu():
     assert L.fp4_mx_to_nv_codes(A, A, 4, 48, 1, A, A, A, None, 0x400, None) == 3
     assert L.fp4_mx_to_nv_codes(A, A, 4, 64, 1, A + 8, A, A, None, 0x400, None) == 2
     assert L.fp4_mx_to_nv_codes(A, A, 4, 64, 1, A, A, A, A + 4, 0x400, None) == 2
+    # EP records: H % 256, too many rows, misaligned records; row gather: row_bytes % 16
+    assert L.fp4_moe_ep_pack(A, A, 4, 2, 320, A, None, A, 8, 2, A, None) == 3
+    assert L.fp4_moe_ep_pack(A, A, 4, 2, 256, A, None, A, 9, 2, A, None) == 1
+    assert L.fp4_moe_ep_pack(A, A, 4, 2, 256, A, None, A, 8, 2, A + 4, None) == 2
+    assert L.fp4_moe_ep_unpack(A, 8, 256, A, A, A, None, None) == 1
+    assert L.fp4_gather_rows(A, 20, A, 4, A, None) == 3
+    assert L.fp4_amax_bf16(A, 4, 12, 12, A, None) == 3
+    assert L.fp4_moe_ep_record_bytes(7168) == 3584 + 448 + 16
+    # empty EP calls launch nothing and succeed with NULL buffers
+    assert L.fp4_moe_ep_pack(None, None, 0, 2, 256, None, None, None, 0, 2, None, None) == 0
+    assert L.fp4_gather_rows(None, 16, None, 0, None, None) == 0
     # FP4 -> FP8 widening: cols % 32, misaligned output, null input
     assert L.fp4_e2m1_to_e4m3(A, 4, 48, A, None) == 3
     assert L.fp4_e2m1_to_e4m3(A, 4, 64, A + 8, None) == 2

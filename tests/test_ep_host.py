@@ -1,0 +1,93 @@
+"""Expert-parallel orchestration on CPU ranks (gloo): the amax all-reduce,
+the row-count and record all-to-alls and the return of the expert outputs,
+with the compute steps taken by the oracle.  Splitting the batch over two
+ranks -- evenly, unevenly, with a rank that has no tokens, and with a rank
+whose experts receive no rows -- must give exactly the bf16 output of one
+rank holding the whole batch and all the experts."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch.multiprocessing as mp
+
+H, I, E, K = 64, 32, 4, 2
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _batch(T, seed, only_experts):
+    import torch
+
+    import synth
+
+    x = synth.activations_bf16((T, H), seed=seed)
+    ids, w, _ = synth.router(T, E, K, seed=seed + 1)
+    if only_experts is not None:  # every token routed into the given experts
+        ids = torch.stack([torch.full((T,), only_experts[0]), torch.full((T,), only_experts[1])], 1).to(torch.int32)
+    return x, ids, w
+
+
+def _run_rank(rank, world, port, splits, seed, only_experts, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import sys
+
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import datetime
+
+    import torch.distributed as dist
+
+    from fp4_block_scaled_03_b200 import ep
+    from tests.ep_oracle_ops import OracleOps, OracleWeights
+
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        x, ids, w = _batch(sum(splits), seed, only_experts)
+        a = sum(splits[:rank])
+        sl = slice(a, a + splits[rank])
+        ops = OracleOps(OracleWeights(E, H, I, seed=7), H, E, world, rank)
+        out = ep.moe_layer_ep(x[sl], ids[sl], w[sl], ops, ep.TorchComm())
+        q.put((rank, out.numpy()))
+    finally:
+        dist.destroy_process_group()
+
+
+def _reference(T, seed, only_experts):
+    from fp4_block_scaled_03_b200 import ep
+    from tests.ep_oracle_ops import LocalComm, OracleOps, OracleWeights
+
+    x, ids, w = _batch(T, seed, only_experts)
+    return ep.moe_layer_ep(x, ids, w, OracleOps(OracleWeights(E, H, I, seed=7), H, E, 1, 0), LocalComm()).numpy()
+
+
+@pytest.mark.parametrize("splits,only_experts", [([6, 6], None), ([9, 3], None), ([7, 0], None), ([5, 6], (0, 1))])
+def test_two_rank_ep_equals_one_rank(splits, only_experts):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_run_rank, args=(r, 2, port, splits, 3, only_experts, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    got = dict(q.get(timeout=180) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    ref = _reference(sum(splits), 3, only_experts)
+    out = np.concatenate([got[0].reshape(-1, H), got[1].reshape(-1, H)])
+    assert out.shape == ref.shape
+    assert np.array_equal(out, ref)
+    assert np.any(ref != 0)
+
+
+def test_expert_ranges_and_local_ids():
+    from fp4_block_scaled_03_b200 import ep
+
+    assert [ep.expert_range(384, 8, r) for r in (0, 7)] == [(0, 48), (336, 384)]
+    with pytest.raises(ValueError):
+        ep.expert_range(10, 4, 0)

@@ -1,0 +1,215 @@
+"""Expert-parallel layer on the GPU, with G ranks emulated in one process:
+each rank runs fp4_block_scaled_03_b200.ep.moe_layer_ep on its own Python
+thread with its own slice of the experts, and a loopback exchange stands in
+for the all-to-all (the ranks' kernels never wait on one another: they
+share one stream, and every exchange happens on the host between launches).
+The bf16 output of the G ranks, concatenated, must equal the 1-GPU layer's
+on the whole batch bit for bit -- the EP path runs the same kernels on the
+same rows in the same per-expert order (the 1-GPU layer is itself checked
+against the oracle in test_gpu_moe.py)."""
+import threading
+
+import numpy as np
+import pytest
+import torch
+
+from tests import moe_case
+
+pytestmark = pytest.mark.gpu
+
+
+class _Hub:
+    def __init__(self, world):
+        self.world = world
+        self.barrier = threading.Barrier(world, timeout=120)
+        self.slots = [None] * world
+
+
+class _LoopComm:
+    def __init__(self, hub, rank):
+        self.hub, self.rank, self.world = hub, rank, hub.world
+
+    def _exchange(self, obj, take):
+        """Post obj, let every rank compute its result from all posts (on
+        the shared stream, while every post is alive), then release."""
+        self.hub.slots[self.rank] = obj
+        self.hub.barrier.wait()
+        res = take(list(self.hub.slots))
+        self.hub.barrier.wait()
+        return res
+
+    def all_reduce_max_(self, t):
+        def take(posts):
+            m = posts[0].clone()
+            for p in posts[1:]:
+                m = torch.maximum(m, p)
+            return m
+
+        t.copy_(self._exchange(t, take))
+        return t
+
+    def exchange_counts(self, send_rows):
+        return self._exchange(list(send_rows), lambda posts: [posts[s][self.rank] for s in range(self.world)])
+
+    def all_to_all(self, send, send_rows, recv_rows):
+        def take(posts):
+            parts = []
+            for t, rows in posts:
+                o = sum(rows[:self.rank])
+                parts.append(t[o:o + rows[self.rank]])
+            return torch.cat(parts).contiguous()
+
+        out = self._exchange((send, list(send_rows)), take)
+        assert out.shape[0] == sum(recv_rows)
+        return out
+
+
+def _run_ep(c, H, I, E, world, splits):
+    from fp4_block_scaled_03_b200 import ep
+
+    hub = _Hub(world)
+    outs, errs = [None] * world, []
+
+    def rank_main(r):
+        try:
+            a = sum(splits[:r])
+            sl = slice(a, a + splits[r])
+            ops = ep.CudaOps(ep.local_weights(c.weights, E, I, H, world, r), H, I, E, world, r)
+            outs[r] = ep.moe_layer_ep(c.x[sl], c.ids[sl], c.w[sl], ops, _LoopComm(hub, r))
+        except BaseException as exc:  # noqa: BLE001 -- reported below
+            errs.append(exc)
+            hub.barrier.abort()
+
+    th = [threading.Thread(target=rank_main, args=(r,)) for r in range(world)]
+    for t in th:
+        t.start()
+    for t in th:
+        t.join(timeout=300)
+    if errs:
+        raise errs[0]
+    torch.cuda.synchronize()
+    return torch.cat(outs)
+
+
+@pytest.mark.parametrize("world,splits,H,I,E,k,zipf", [
+    (2, [150, 150], 512, 256, 8, 2, 0.0),
+    (4, [300, 100, 0, 200], 1024, 256, 16, 6, 1.1),   # uneven, one rank with no tokens
+    (1, [256], 512, 256, 4, 2, 0.0),
+    (8, [64] * 8, 1024, 512, 32, 6, 1.1),
+])
+def test_ep_equals_single_gpu_layer(world, splits, H, I, E, k, zipf):
+    import fp4_block_scaled_03_b200 as fp4
+
+    T = sum(splits)
+    c = moe_case.build(T, H, I, E, k, seed=T + world, zipf=zipf)
+    ref = fp4.moe_layer(c.x, c.ids, c.w, c.weights, H, I, E)
+    got = _run_ep(c, H, I, E, world, splits)
+    assert fp4.fp4_get_device_status() == 0
+    assert torch.equal(got.view(torch.int16), ref.view(torch.int16))
+
+
+def test_ep_rank_whose_experts_get_no_rows():
+    """All tokens routed to rank 0's experts: rank 1 receives zero records and
+    returns zero rows."""
+    import fp4_block_scaled_03_b200 as fp4
+
+    H, I, E, k, world = 512, 256, 8, 2, 2
+    c = moe_case.build(200, H, I, E, k, seed=5)
+    c.ids = (c.ids % (E // world)).contiguous()  # experts 0..3 only
+    ref = fp4.moe_layer(c.x, c.ids, c.w, c.weights, H, I, E)
+    got = _run_ep(c, H, I, E, world, [120, 80])
+    assert torch.equal(got.view(torch.int16), ref.view(torch.int16))
+
+
+def test_ep_records_round_trip():
+    """fp4_moe_ep_pack then fp4_moe_ep_unpack: codes, scales, weights and
+    local expert ids of every routed row, in routed order."""
+    import fp4_block_scaled_03_b200 as fp4
+
+    T, H, k, E, epr = 37, 768, 3, 12, 4
+    rng = np.random.default_rng(3)
+    codes = torch.from_numpy(rng.integers(0, 256, (T, H // 2), dtype=np.uint8)).cuda()
+    sf = torch.from_numpy(rng.integers(0, 256, (T, H // 16), dtype=np.uint8)).cuda()
+    ids_np = rng.integers(0, E, (T, k)).astype(np.int32)
+    w_np = rng.random((T, k)).astype(np.float32)
+    perm_np = np.argsort(ids_np.reshape(-1), kind="stable").astype(np.int32)
+    R = T * k
+    rb = fp4.fp4_moe_ep_record_bytes(H)
+    assert rb == H // 2 + H // 16 + 16
+    rec = torch.empty((R, rb), dtype=torch.uint8, device="cuda")
+    fp4.fp4_moe_ep_pack(codes, sf, T, k, H, torch.from_numpy(ids_np).cuda(), torch.from_numpy(w_np).cuda(),
+                        torch.from_numpy(perm_np).cuda(), R, epr, rec)
+    oc = torch.empty((R, H // 2), dtype=torch.uint8, device="cuda")
+    osf = torch.empty((R, H // 16), dtype=torch.uint8, device="cuda")
+    ow = torch.empty(R, dtype=torch.float32, device="cuda")
+    oid = torch.empty(R, dtype=torch.int32, device="cuda")
+    fp4.fp4_moe_ep_unpack(rec, R, H, oc, osf, ow, oid)
+    tok = perm_np // k
+    assert np.array_equal(oc.cpu().numpy(), codes.cpu().numpy()[tok])
+    assert np.array_equal(osf.cpu().numpy(), sf.cpu().numpy()[tok])
+    assert np.array_equal(ow.cpu().numpy(), w_np.reshape(-1)[perm_np])
+    assert np.array_equal(oid.cpu().numpy(), ids_np.reshape(-1)[perm_np] % epr)
+    assert np.all(rec.cpu().numpy()[:, -8:] == 0)
+
+
+def test_amax_and_global_scale_match_dynamic_quantizer():
+    """fp4_amax_bf16 + fp4_nv_global_scale give the g the dynamic quantizer
+    computes; empty input gives amax 0."""
+    import fp4_block_scaled_03_b200 as fp4
+    import synth
+
+    x = synth.activations_bf16((333, 1024), seed=9, device="cuda")
+    _, _, g_dyn = fp4.quantize_nv(x)
+    a = torch.empty(1, dtype=torch.int32, device="cuda")
+    fp4.fp4_amax_bf16(x, 333, 1024, 1024, a)
+    ref = np.abs(x.float().cpu().numpy()).max()
+    assert np.uint32(a.item()).view(np.float32) == np.float32(ref)
+    g = torch.empty(1, dtype=torch.float32, device="cuda")
+    fp4.fp4_nv_global_scale(a, 1, g)
+    assert g.item() == g_dyn.item()
+    fp4.fp4_amax_bf16(x, 0, 1024, 1024, a)
+    assert a.item() == 0
+
+
+def test_gather_rows():
+    import fp4_block_scaled_03_b200 as fp4
+
+    rng = np.random.default_rng(1)
+    src = torch.from_numpy(rng.standard_normal((50, 96)).astype(np.float32)).cuda()
+    idx = torch.from_numpy(rng.integers(0, 50, 77).astype(np.int32)).cuda()
+    dst = torch.empty((77, 96), dtype=torch.float32, device="cuda")
+    fp4.fp4_gather_rows(src, 96 * 4, idx, 77, dst)
+    assert torch.equal(dst, src[idx.long()])
+
+
+def test_ep_over_nccl_world_of_one():
+    """The torch.distributed exchange (NCCL: device tensors, all_to_all_single
+    with split sizes, an int32 MAX all-reduce) on a world of one rank: the
+    layer equals the 1-GPU layer bit for bit."""
+    import datetime
+    import socket
+
+    import torch.distributed as dist
+
+    import fp4_block_scaled_03_b200 as fp4
+    from fp4_block_scaled_03_b200 import ep
+
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    store = dist.TCPStore("127.0.0.1", port, 1, is_master=True, timeout=datetime.timedelta(seconds=60))
+    dist.init_process_group("nccl", store=store, rank=0, world_size=1, timeout=datetime.timedelta(seconds=60),
+                            device_id=torch.device("cuda", torch.cuda.current_device()))
+    try:
+        H, I, E, k = 512, 256, 8, 2
+        c = moe_case.build(300, H, I, E, k, seed=41, zipf=1.1)
+        ref = fp4.moe_layer(c.x, c.ids, c.w, c.weights, H, I, E)
+        comm = ep.TorchComm()
+        assert not comm.host_staging
+        ops = ep.CudaOps(ep.local_weights(c.weights, E, I, H, 1, 0), H, I, E, 1, 0)
+        got = ep.moe_layer_ep(c.x, c.ids, c.w, ops, comm)
+        torch.cuda.synchronize()
+        assert torch.equal(got.view(torch.int16), ref.view(torch.int16))
+    finally:
+        dist.destroy_process_group()
