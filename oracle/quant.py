@@ -38,12 +38,12 @@ remapped losslessly and is reported as a range error.
 Lossy-span fallback ("DeepSeek-V4 architecture" §6.3 says the conversion is
 lossless only while the ratio of the scale factors stays under a threshold;
 it gives no rule beyond it).  Reading: a live block whose exact E4M3 power
-2^k would fall below 2^-9 (k < -9) is re-expressed at the smallest power,
-2^-9: each element value val(c) * 2^k (in units of g) becomes the E2M1 code
-nearest to val(c) * 2^(k+9), ties to even, the sign bit kept -- the same
-rounding the NVFP4 quantizer applies -- and the block's scale is 2^-9 if any
-re-encoded magnitude is nonzero, else 0.  Every other block is remapped
-exactly as in the lossless case.
+2^k would fall below 2^-9 (k < -9) is re-quantized from its dequantized
+values, val(c) * 2^e in fp32 (exact), by the NVFP4 rule above at the
+tensor's fixed g, one 16-element half at a time.  Every other block is
+remapped exactly as in the lossless case.  (Under that rule such a block's
+amax_b / (6g) is at most 2^-10, which rounds to the E4M3 code 0: its scales
+become 0 and its codes sign|0.)
 
 MXFP8 (the W4A8 activation format: "DeepSeek-V4 FP4 QAT" §4.3 recommends FP8
 activations against FP4 weights, and §4.2 keeps the power-of-two block scale
@@ -233,11 +233,11 @@ def mx_to_nv(packed, mx_scales, num_tensors=1):
 
 
 def mx_to_nv_lossy(packed, mx_scales, num_tensors=1):
-    """MXFP4 -> NVFP4 remap that re-encodes the blocks below E4M3's range
+    """MXFP4 -> NVFP4 remap that re-quantizes the blocks below E4M3's range
     (the lossy-span fallback above) instead of refusing the tensor.
 
     Returns (codes uint8 [.., cols/2], nv_sf uint8 [.., cols/16],
-    g fp32 [num_tensors], lossy int64 [num_tensors] = re-encoded 32-blocks).
+    g fp32 [num_tensors], lossy int64 [num_tensors] = re-quantized 32-blocks).
     A UE8M0 NaN byte is still an error."""
     packed = np.asarray(packed, dtype=np.uint8)
     mx_scales = np.asarray(mx_scales, dtype=np.uint8)
@@ -259,21 +259,21 @@ def mx_to_nv_lossy(packed, mx_scales, num_tensors=1):
         if not np.any(lt):
             continue
         e_max = int(np.max(e[r0:r0 + rows][lt]))
-        gs[t] = pow2_f32(e_max - 8)
+        g = pow2_f32(e_max - 8)
+        gs[t] = g
         for r in range(r0, r0 + rows):
             for j in range(cols // MX_BLOCK):
                 if not live[r, j]:
                     continue
                 k = int(e[r, j]) - e_max + 8
                 if k >= -9:
-                    sf = e4m3_power_of_two(k)
-                else:
-                    lossy[t] += 1
-                    # exact value in units of g * 2^-9; a power of two this small may
-                    # underflow fp32 to a signed zero, which still rounds to code 0
-                    x = (e2m1_decode(codes[r, j]) * np.ldexp(1.0, k + 9)).astype(np.float32)
-                    codes[r, j] = e2m1_encode(x)
-                    sf = e4m3_power_of_two(-9) if np.any(codes[r, j] & 7) else np.uint8(0)
-                nv_sf[r, 2 * j] = sf
-                nv_sf[r, 2 * j + 1] = sf
+                    nv_sf[r, 2 * j] = nv_sf[r, 2 * j + 1] = e4m3_power_of_two(k)
+                    continue
+                lossy[t] += 1
+                # the block's dequantized values (exact in fp32: at least 2^-128 in
+                # magnitude when nonzero), re-quantized by the NVFP4 rule at g
+                x = (e2m1_decode(codes[r, j]) * np.ldexp(1.0, int(e[r, j]))).astype(np.float32)
+                pc, sf, _ = nvfp4_quantize(x.reshape(1, MX_BLOCK), g=g)
+                codes[r, j] = unpack_nibbles(pc)[0]
+                nv_sf[r, 2 * j:2 * j + 2] = sf[0]
     return pack_nibbles(codes.reshape(total_rows, cols)), nv_sf, gs, lossy
