@@ -367,7 +367,8 @@ def fp4_mx_to_nv_codes(codes, mx_scales, rows, cols, num_tensors, nv_codes, nv_s
 
 def mx_to_nv_codes(codes, mx_scales, num_tensors, tiled=False, allow_lossy=True, out_codes=None):
     """MX -> NV remap that writes the codes too; with allow_lossy, blocks below
-    E4M3's range are re-encoded at 2^-9.  Returns (codes, scales, g, lossy)."""
+    E4M3's range are re-quantized by the NVFP4 rule at the tensor's g (which
+    flushes them to signed zeros).  Returns (codes, scales, g, lossy)."""
     total_rows, half = codes.shape
     rows, cols = total_rows // num_tensors, half * 2
     if tiled:

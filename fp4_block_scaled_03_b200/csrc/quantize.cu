@@ -515,28 +515,15 @@ __device__ __forceinline__ float pow2_f32(int e) {  // exact 2^e, e in [-149, 12
   return __uint_as_float(1u << (e + 149));
 }
 
-// E2M1 magnitude code nearest to val(m) * 2^-d (d >= 1), ties to the even
-// code: the re-encoding of a block below E4M3's smallest power of two.
-// Magnitudes in units of 0.5 are integers (0 1 2 3 4 6 8 12), so the search
-// compares exact integer distances.
-__device__ __forceinline__ uint32_t e2m1_shift_down(uint32_t m, int d) {
-  if (d > 5) return 0;  // val(m) * 2^-6 <= 0.09375: nearest is 0
-  const int half_units[8] = {0, 1, 2, 3, 4, 6, 8, 12};
-  const int v = half_units[m];
-  uint32_t best = 0;
-  int best_dist = v;  // distance to code 0
-  for (uint32_t c = 1; c < 8; ++c) {
-    const int dist = abs(v - (half_units[c] << d));
-    if (dist < best_dist || (dist == best_dist && (c & 1u) == 0)) {
-      best = c;
-      best_dist = dist;
-    }
-  }
-  return best;
+// E2M1 code (sign bit 3) -> its value, exactly.
+__device__ __forceinline__ float e2m1_value(uint32_t c) {
+  const float mag[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+  const float v = mag[c & 7u];
+  return (c & 8u) ? -v : v;
 }
 
 // kCodes: also write the codes to out_codes (which may alias `codes`) and,
-// with kLossy, re-encode the blocks below E4M3's range instead of refusing.
+// with kLossy, re-quantize the blocks below E4M3's range instead of refusing.
 template <bool kTiled, bool kCodes, bool kLossy>
 __global__ void __launch_bounds__(kThreads) mx_to_nv_kernel(const uint8_t *codes, const uint8_t *__restrict__ mx,
                                                             int64_t rows, int64_t cols, uint8_t *__restrict__ nv,
@@ -584,36 +571,36 @@ __global__ void __launch_bounds__(kThreads) mx_to_nv_kernel(const uint8_t *codes
   int n_lossy = 0;
   for (int64_t i = threadIdx.x; i < nb; i += blockDim.x) {
     uint4 c = *reinterpret_cast<const uint4 *>(cb + i * 16);
-    uint32_t code = 0;
+    uint32_t pair = 0;  // the scale bytes of the block's two 16-element halves
     if (block_live(c)) {
       const int k = ((int)sb[i] - 127) - emax + 8;  // exact while k >= -9
-      if (kLossy && k < -9) {  // re-express at 2^-9: every magnitude shrinks by 2^(k+9)
-        uint32_t w[4] = {c.x, c.y, c.z, c.w}, any = 0;
+      if (kLossy && k < -9) {
+        // re-quantize the block's dequantized values, val(c) * 2^e (exact in
+        // fp32), by the NVFP4 block rule at g, one 16-element half at a time
+        const float g = pow2_f32(emax - 8), p2 = pow2_f32((int)sb[i] - 127);
+        const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+        uint32_t o[4], sf2[2];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t o = 0;
+        for (int hh = 0; hh < 2; ++hh) {
+          float x[16];
 #pragma unroll
-          for (int n = 0; n < 8; ++n) {
-            const uint32_t nib = (w[q] >> (4 * n)) & 0xFu;
-            const uint32_t m = e2m1_shift_down(nib & 7u, -9 - k);
-            any |= m;
-            o |= ((nib & 8u) | m) << (4 * n);
-          }
-          w[q] = o;
+          for (int n = 0; n < 16; ++n) x[n] = __fmul_rn(e2m1_value((w[2 * hh + n / 8] >> (4 * (n % 8))) & 0xFu), p2);
+          sf2[hh] = nvfp4_block16(x, g, &o[2 * hh], &o[2 * hh + 1]);
         }
-        c = make_uint4(w[0], w[1], w[2], w[3]);
-        code = any ? 0x01u : 0u;  // 2^-9, E4M3's smallest power of two
+        c = make_uint4(o[0], o[1], o[2], o[3]);
+        pair = sf2[0] | (sf2[1] << 8);
         ++n_lossy;
       } else {
-        code = k >= -6 ? (uint32_t)((k + 7) << 3) : (1u << (k + 9));
+        const uint32_t code = k >= -6 ? (uint32_t)((k + 7) << 3) : (1u << (k + 9));
+        pair = code | (code << 8);
       }
     }
     if (kCodes) *reinterpret_cast<uint4 *>(ocb + i * 16) = c;
     if (kTiled) {  // block i = (row, 32-block j): 16-blocks 2j and 2j+1 are adjacent bytes
       const int64_t r = i / (cols / 32), j = i - r * (cols / 32);
-      *reinterpret_cast<uint16_t *>(ob + sf_tiled_offset(r, 2 * j, cols / 64)) = (uint16_t)(code | (code << 8));
+      *reinterpret_cast<uint16_t *>(ob + sf_tiled_offset(r, 2 * j, cols / 64)) = (uint16_t)pair;
     } else {
-      *reinterpret_cast<uint16_t *>(ob + 2 * i) = (uint16_t)(code | (code << 8));
+      *reinterpret_cast<uint16_t *>(ob + 2 * i) = (uint16_t)pair;
     }
   }
   if (kCodes && lossy_blocks) {

@@ -86,7 +86,7 @@ typedef enum { FP4_OUT_F32 = 0, FP4_OUT_BF16 = 1 } fp4_out_dtype;
 #define FP4_GEMM_B_MXFP8 0x80u       /* fp4_gemm with FP4_GEMM_A_MXFP8: B is MXFP8 too */
 #define FP4_MOE_W4A8 0x100u          /* MoE layer / stages: MXFP4 weights, MXFP8 activations and h */
 #define FP4_MOE_DYNAMIC_H 0x200u     /* MoE layer (NVFP4, row tiles): h scale per expert from this batch */
-#define FP4_MX2NV_ALLOW_LOSSY 0x400u /* fp4_mx_to_nv_codes: re-encode blocks below E4M3's range, never refuse a span */
+#define FP4_MX2NV_ALLOW_LOSSY 0x400u /* fp4_mx_to_nv_codes: re-quantize blocks below E4M3's range, never refuse a span */
 
 /* Human-readable name of a status code (static string). */
 const char *fp4_status_string(fp4_status s);
@@ -180,16 +180,17 @@ fp4_status fp4_mx_to_nv(const uint8_t *codes, const uint8_t *mx_scales, int64_t 
  *   nv_codes      device uint8 [num_tensors*rows][cols/2], 16-byte aligned;
  *                 receives every code.  May equal `codes` (in place).
  *   lossy_blocks  device int64 [num_tensors] or NULL: the number of 32-element
- *                 blocks of each tensor that were re-encoded (0 for a
+ *                 blocks of each tensor that were re-quantized (0 for a
  *                 refused tensor).
  * Without FP4_MX2NV_ALLOW_LOSSY the result is that of fp4_mx_to_nv, codes
  * copied unchanged.  With it, no span is refused: a live block whose exact
- * E4M3 power 2^k lies below 2^-9 (k = e - e_max + 8 < -9) is re-expressed at
- * 2^-9 -- each code becomes the E2M1 code nearest to val(code) * 2^(k+9),
- * ties to the even code, sign bit kept -- and its scale byte is 0x01 (2^-9),
- * or 0 if every re-encoded magnitude is 0.  All other blocks are remapped
- * exactly.  A UE8M0 NaN byte still refuses its tensor (nv_global NaN; its
- * codes and scales are left untouched).  SYNCHRONOUS, like fp4_mx_to_nv;
+ * E4M3 power 2^k lies below 2^-9 (k = e - e_max + 8 < -9) is re-quantized
+ * from its dequantized values val(code) * 2^e by the NVFP4 block rule of
+ * fp4_quantize at the tensor's g = 2^(e_max-8), one 16-element half at a
+ * time (such a block's amax / (6g) is at most 2^-10, so its scales become 0
+ * and its codes sign|0).  All other blocks are remapped exactly.  A UE8M0 NaN
+ * byte still refuses its tensor (nv_global NaN; its codes and scales are
+ * left untouched).  SYNCHRONOUS, like fp4_mx_to_nv;
  * returns FP4_ERR_RANGE if any tensor was refused.
  */
 fp4_status fp4_mx_to_nv_codes(const uint8_t *codes, const uint8_t *mx_scales, int64_t rows, int64_t cols,

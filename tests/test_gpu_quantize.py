@@ -171,7 +171,7 @@ def _wide_span_mx(nt, rows, cols, seed):
 @pytest.mark.parametrize("inplace", [False, True])
 def test_remap_lossy_bit_exact(tiled, inplace):
     """fp4_mx_to_nv_codes with FP4_MX2NV_ALLOW_LOSSY: codes, scales, globals
-    and re-encoded block counts equal the oracle's lossy remap bit for bit
+    and re-quantized block counts equal the oracle's lossy remap bit for bit
     (several tensors, rows not a multiple of 128, spans up to 129 octaves)."""
     fp4 = _lib()
     nt, rows, cols = 3, 96, 192
