@@ -391,6 +391,8 @@ def run_moe(args, world, rank, peaks):
     for i in range(args.steps):
         for j in range(nst - 1):
             stage[j] += evs[i][j].elapsed_time(evs[i][j + 1]) / args.steps
+    per_step = sorted(evs[i][0].elapsed_time(evs[i][nst - 1]) for i in range(args.steps))
+    pct = {f"p{q}": round(per_step[min(len(per_step) - 1, (q * len(per_step)) // 100)], 4) for q in (10, 50, 90)}
     flops = b.flops()
     value = world * flops / (ms * 1e-3) / 1e12
     # FP4 x FP4 runs at 4x the bf16 rate, FP8 x FP4 (W4A8) at the FP8 rate, 2x (the recipe's nominal ratios)
@@ -467,6 +469,24 @@ def run_moe(args, world, rank, peaks):
     d2h = b.T * b.H * 2
     del ws
 
+    # the w13 launch's roofline: the tensor pipe when its FLOPs take longer at
+    # peak than its bytes at the HBM copy rate (prefill), else HBM (decode and
+    # the Flash layer, whose every M tile streams its own expert's weights)
+    t_flops = w13_flops / (fp4_peak * 1e12)
+    t_bytes = w13_bytes / (peaks["hbm"] * 1e9)
+    roof = {"kernel": b.kernel_name("w13") + " (grouped w13 + SwiGLU + requant)"}
+    if t_flops >= t_bytes:
+        roof.update(bound="tensor", achieved=round(w13_tf, 1), peak=round(fp4_peak, 1), unit="TFLOP/s",
+                    frac=round(w13_tf / fp4_peak, 4))
+    else:
+        w13_gbs = w13_bytes / (stage[2] * 1e-3) / 1e9
+        roof.update(bound="hbm", achieved=round(w13_gbs, 1), peak=round(peaks["hbm"], 1), unit="GB/s",
+                    frac=round(w13_gbs / peaks["hbm"], 4), tensor_tflops=round(w13_tf, 1),
+                    tensor_frac=round(w13_tf / fp4_peak, 4))
+    roof.update(traffic=measured_traffic(args.workload, b.kernel_name("w13")), algorithmic_bytes=w13_bytes,
+                frac_of_max_flops_bytes=round(max(t_flops, t_bytes) / (stage[2] * 1e-3), 4),
+                peak_note="tensor pipe: %dx sustained bf16 cuBLAS (nominal %s/bf16 ratio); HBM: copy bandwidth; of %s"
+                          % (ratio, "fp8" if b.w4a8 else "fp4", peaks["src"]))
     line = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -492,15 +512,9 @@ def run_moe(args, world, rank, peaks):
                                "per expert from this batch (two-phase w13)" if b.dynamic_h else
                                "static per expert, calibrated once on the batch"),
                    "padding_frac": round(1.0 - b.R / max(1, b.mma_rows()), 4)},
-        "roofline": {"bound": "tensor", "kernel": b.kernel_name("w13") + " (grouped w13 + SwiGLU + requant)",
-                     "achieved": round(w13_tf, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
-                     "frac": round(w13_tf / fp4_peak, 4), "traffic": measured_traffic(args.workload, b.kernel_name("w13")),
-                     "algorithmic_bytes": w13_bytes,
-                     "frac_of_max_flops_bytes": round(max(w13_flops / (fp4_peak * 1e12), w13_bytes / (peaks["hbm"] * 1e9))
-                                                      / (stage[2] * 1e-3), 4),
-                     "peak_note": "%dx measured sustained bf16 cuBLAS (nominal %s/bf16 ratio), of %s"
-                                  % (ratio, "fp8" if b.w4a8 else "fp4", peaks["src"])},
+        "roofline": roof,
         "stages_ms": {n: round(v, 4) for n, v in zip(["route", "quantize_gather", "w13", "w2", "combine"], stage)},
+        "step_ms_percentiles": pct,
         "w2": {"achieved_tflops": round(w2_tf, 1), "frac": round(w2_tf / fp4_peak, 4),
                "traffic": measured_traffic(args.workload, b.kernel_name("w2"))},
         "quantize": {"achieved_gbs": round(q_gbs, 1), "peak_gbs": peaks["hbm"], "frac": round(q_gbs / peaks["hbm"], 4),
