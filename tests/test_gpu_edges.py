@@ -53,3 +53,17 @@ def test_all_tokens_on_one_expert(tiling):
     c = moe_case.build(1000, 512, 256, 8, 1, seed=3, counts=[0, 0, 1000, 0, 0, 0, 0, 0])
     TM._check_w13(c, tiling)
     TM._check_w2(c, tiling)
+
+
+@pytest.mark.parametrize("tiling", TM.TILINGS)
+def test_layer_one_token_top16_minimal_shape(tiling):
+    """One token sent to all 16 experts (the largest top-k) at the smallest
+    shape the layer takes (H = I = 256): 16 one-row experts."""
+    TM.test_layer_end_to_end(1, 256, 256, 16, 16, 0.0, tiling)
+
+
+@pytest.mark.parametrize("tiling", TM.TILINGS)
+def test_layer_ragged_tiles(tiling):
+    """129 tokens x top-2 over 3 experts: every expert's rows end in a ragged
+    tile (and, for CTA pairs, a ragged 256-row chunk)."""
+    TM.test_layer_end_to_end(129, 256, 512, 3, 2, 0.0, tiling)
