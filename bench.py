@@ -183,7 +183,7 @@ def barrier(world):
 
 # ---------------------------------------------------------------------------
 class MoeBench:
-    def __init__(self, name, seed, pair_tiles=False, dynamic_h=False):
+    def __init__(self, name, seed, pair_tiles=False, dynamic_h=False, weight_seed=None):
         import torch
 
         import fp4_block_scaled_03_b200 as fp4
@@ -201,6 +201,7 @@ class MoeBench:
         self.dynamic_h = dynamic_h and not self.mx and not self.pair
         if self.dynamic_h:
             self.flags |= fp4.FP4_MOE_DYNAMIC_H
+        wseed = seed if weight_seed is None else weight_seed  # the layer's weights (same on every EP rank)
         T, H, I, E, k, zipf, sigma, desc = WORKLOADS[name]
         self.T, self.H, self.I, self.E, self.k, self.desc, self.name = T, H, I, E, k, desc, name
         dev = "cuda"
@@ -217,7 +218,7 @@ class MoeBench:
         for e in range(E):
             for (rows, cols, codes, sf, g, sfb, off) in ((2 * I, H, self.w13_codes, self.w13_sf, self.w13_g, s13, 2),
                                                           (H, I, self.w2_codes, self.w2_sf, self.w2_g, s2, 3)):
-                wb = synth.weights_bf16((rows, cols), sigma, 0.005, 30.0, seed=seed + 1000 * off + e, device=dev)
+                wb = synth.weights_bf16((rows, cols), sigma, 0.005, 30.0, seed=wseed + 1000 * off + e, device=dev)
                 sl = slice(e * rows, (e + 1) * rows)
                 if self.mx:  # MXFP4 weights used as they are
                     cc, ss = fp4.quantize_mx(wb, tiled=True)
@@ -597,6 +598,71 @@ def cpu_baseline_moe(b, n_tokens=1):
 
 
 # ---------------------------------------------------------------------------
+def run_moe_ep(args, world, rank, peaks):
+    """The expert-parallel layer (fp4_block_scaled_03_b200.ep): every rank
+    holds T tokens of its own and E/world experts of one shared layer; rows
+    go to their expert's rank and back by NCCL all-to-all.  Each timed step
+    includes the host's read of the per-rank row counts that the all-to-all
+    needs, so the device time is the step's whole span."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    from fp4_block_scaled_03_b200 import ep
+
+    if not dist.is_initialized():  # a world of one outside torchrun
+        import socket
+
+        sk = socket.socket()
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+        sk.close()
+        store = dist.TCPStore("127.0.0.1", port, 1, is_master=True, timeout=datetime.timedelta(seconds=60))
+        dist.init_process_group("nccl", store=store, rank=0, world_size=1, timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", torch.cuda.current_device()))
+    b = MoeBench(args.workload, seed=rank * 7919, weight_seed=0)
+    if b.mx or b.pair or b.dynamic_h:
+        raise SystemExit("--ep runs the NVFP4 row-tile layer")
+    ops = ep.CudaOps(ep.local_weights(b.wset, b.E, b.I, b.H, world, rank), b.H, b.I, b.E, world, rank)
+    comm = ep.TorchComm()
+    for _ in range(args.warmup):
+        ep.moe_layer_ep(b.x, b.ids, b.w, ops, comm)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        out = ep.moe_layer_ep(b.x, b.ids, b.w, ops, comm)
+    e1.record()
+    torch.cuda.synchronize()
+    dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    assert b.fp4.fp4_get_device_status() == 0 and out.shape == (b.T, b.H)
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+    value = world * b.flops() / (ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e2m1, e4m3/16 scales, fp32 accumulate)",
+        "data": "synthetic (seeded): per-rank tokens, one shared layer of seeded weights",
+        "config": {"workload": b.desc + ", expert-parallel", "tokens_per_rank": b.T, "hidden": b.H,
+                   "intermediate": b.I, "experts": b.E, "experts_per_rank": b.E // world, "topk": b.k,
+                   "parallelism": f"ep{world}", "l2": "inputs larger than L2"},
+        "roofline": None,
+        "note": "layer step through moe_layer_ep: amax all-reduce, quantize, route, record all-to-all, local"
+                " grouped GEMMs, output all-to-all, combine; no per-kernel roofline on this line",
+        "gpu_launches": 16 * args.steps, "clocks": clocks,
+    }
+    dist.destroy_process_group()
+    return line
+
+
 def run_dense(args, world, rank, peaks, mx=False, w4a8=False):
     """Dense 4096^3 GEMM with the activation quantized on the device every
     call: NVFP4 x NVFP4, MXFP4 x MXFP4 (mx), or W4A8 -- MXFP8 activations x
@@ -858,6 +924,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--dynamic-h", action="store_true",
                     help="NVFP4 MoE workloads: per-expert h scale from each batch (two-phase w13)")
+    ap.add_argument("--ep", action="store_true",
+                    help="NVFP4 MoE workloads: the expert-parallel layer over NCCL (experts split over the ranks)")
     ap.add_argument("--pair-tiles", action="store_true",
                     help="MoE workloads: CTA-pair tiles (cta_group::2, tokens on N) for the NVFP4 grouped GEMMs")
     args = ap.parse_args()
@@ -875,6 +943,11 @@ def main():
             import torch.distributed as dist
 
             dist.destroy_process_group()
+        return
+    elif args.workload in WORKLOADS and args.ep:
+        line = run_moe_ep(args, world, rank, peaks)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
         return
     elif args.workload in WORKLOADS:
         line = run_moe(args, world, rank, peaks)

@@ -29,6 +29,7 @@ FP4_GEMM_B_MXFP8 = 0x80
 FP4_MOE_W4A8 = 0x100
 FP4_MOE_DYNAMIC_H = 0x200
 FP4_MX2NV_ALLOW_LOSSY = 0x400
+FP4_MOE_Y_BY_SLOT = 0x800
 FP4_MOE_MX = 0x10
 FP4_MOE_PAIR_TILES = 0x20
 

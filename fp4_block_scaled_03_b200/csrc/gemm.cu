@@ -106,6 +106,7 @@ struct Params {
   const int32_t *perm;
   const float *topk_w;
   float *y;
+  int y_by_slot;  // w2: y row perm[r] (the routed slot) instead of routed row r, stored row by row
   unsigned int *status;
   uint64_t wait_limit;
 };
@@ -375,7 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool row_ok = row < ti.rows_valid;
       // w2: a warp whose 32 rows are all valid writes through TMA (collective
       // per warp); otherwise each valid row is stored by its own thread
-      const bool full_box = (EPI == EPI_W2) && (q * 32 + 32 <= ti.rows_valid);
+      const bool full_box = (EPI == EPI_W2) && !p.y_by_slot && (q * 32 + 32 <= ti.rows_valid);
       if (!row_ok) continue;
       float alpha;  // MXFP4 operands carry no tensor-level scale
       if (MX) alpha = 1.0f;
@@ -478,8 +479,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 4; ++i) d[i] = make_float4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
           }
-        } else if (!full_box) {  // EPI_W2, a warp holding the expert's last rows
-          float *dst = p.y + (int64_t)(ti.out_row0 + row) * p.N + col0;
+        } else if (!full_box) {  // EPI_W2, a warp holding the expert's last rows, or y by slot
+          const int64_t yrow = p.y_by_slot ? (int64_t)p.perm[ti.out_row0 + row] : (int64_t)(ti.out_row0 + row);
+          float *dst = p.y + yrow * p.N + col0;
 #pragma unroll
           for (int i = 0; i < 32; i += 4)
             *reinterpret_cast<float4 *>(dst + i) = make_float4(__fmul_rn(w[i], scale), __fmul_rn(w[i + 1], scale),
@@ -724,6 +726,7 @@ fp4_status fp4_moe_w2(const uint8_t *h_codes, const uint8_t *h_sf, const fp4_moe
   if ((int64_t)E * H > (1LL << 31) - 1 || rows_cap > (1LL << 31) - 1) return FP4_ERR_UNSUPPORTED_SHAPE;
   if (!al16(h_codes) || !al16(h_sf) || !al16(w->w2_codes) || !al16(w->w2_sf) || !al16(y)) return FP4_ERR_ALIGNMENT;
   if (w4a8 && (reinterpret_cast<uintptr_t>(w->w2_codes) & 31u)) return FP4_ERR_ALIGNMENT;
+  if ((flags & FP4_MOE_Y_BY_SLOT) && (flags & FP4_MOE_PAIR_TILES)) return FP4_ERR_INVALID_ARG;
   if (!mx && (flags & FP4_MOE_PAIR_TILES)) {
     if (((rows_cap + 255) / 256 + E) * (H / 256) > (1LL << 31) - 1) return FP4_ERR_UNSUPPORTED_SHAPE;
     return moe_pair_w2(h_codes, h_sf, w, H, I, E, counts, offsets, tile_offsets, perm, topk_weights, rows_cap, y,
@@ -752,6 +755,7 @@ fp4_status fp4_moe_w2(const uint8_t *h_codes, const uint8_t *h_sf, const fp4_moe
   p.E = E; p.counts = counts; p.offsets = offsets; p.tile_offsets = tile_offsets;
   p.w_g = w->w2_g; p.h_g = w->h_g;
   p.perm = perm; p.topk_w = topk_weights; p.y = y;
+  p.y_by_slot = (flags & FP4_MOE_Y_BY_SLOT) ? 1 : 0;
   p.status = ctx->status;
   p.wait_limit = ctx->wait_limit_ns;
   CUtensorMap ty;

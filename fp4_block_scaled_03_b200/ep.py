@@ -15,7 +15,8 @@ layer step on every rank is:
   3. all-to-all of the per-rank row counts, then of the records.
   4. unpack; route the received rows over the local experts (one slot each);
      gather them into expert tiles; grouped w13 (SwiGLU + h requant) and w2
-     (routing weight) on tcgen05; put the outputs back in received order.
+     (routing weight) on tcgen05, w2 writing each output row back at the
+     position its record arrived at.
   5. all-to-all of the fp32 output rows back to their senders: they arrive in
      the sender's routed order, so the fixed-order combine finishes the layer.
 
@@ -32,7 +33,7 @@ ranks."""
 import torch
 import torch.distributed as dist
 
-from . import (FP4_NV, FP4_STATIC_GLOBAL_SCALE, MoeWeightSet, _u8, fp4_amax_bf16, fp4_gather_rows,
+from . import (FP4_MOE_Y_BY_SLOT, FP4_NV, FP4_STATIC_GLOBAL_SCALE, MoeWeightSet, _u8, fp4_amax_bf16,
                fp4_moe_combine, fp4_moe_ep_pack, fp4_moe_ep_record_bytes, fp4_moe_ep_unpack, fp4_moe_gather,
                fp4_moe_route, fp4_moe_route_scratch_bytes, fp4_moe_w13, fp4_moe_w2, fp4_nv_global_scale,
                fp4_quantize, fp4_sf_tiled_bytes, moe_rows_cap)
@@ -58,18 +59,23 @@ def local_weights(w, E, I, H, world, rank):
 
 class TorchComm:
     """The exchange steps over a torch.distributed process group.  NCCL moves
-    device tensors directly; another backend (gloo) gets host copies."""
+    device tensors directly; another backend (gloo) gets host copies.  A
+    world of one exchanges nothing (every step is the identity) unless
+    always_exchange asks for the collectives anyway."""
 
-    def __init__(self, group=None):
+    def __init__(self, group=None, always_exchange=False):
         self.group = group
         self.rank = dist.get_rank(group)
         self.world = dist.get_world_size(group)
         self.host_staging = dist.get_backend(group) != "nccl"
+        self.skip = self.world == 1 and not always_exchange
 
     def _stage(self, t):
         return t.cpu() if self.host_staging and t.is_cuda else t
 
     def all_reduce_max_(self, t):
+        if self.skip:
+            return t
         s = self._stage(t)
         dist.all_reduce(s, op=dist.ReduceOp.MAX, group=self.group)
         if s is not t:
@@ -79,6 +85,8 @@ class TorchComm:
     def all_to_all(self, send, send_rows, recv_rows):
         """Rows send[sum(send_rows[:d]) : +send_rows[d]] go to rank d; the
         result holds recv_rows[s] rows from each rank s, in rank order."""
+        if self.skip:
+            return send
         s = self._stage(send.contiguous())
         recv = s.new_empty((sum(recv_rows),) + tuple(send.shape[1:]))
         dist.all_to_all_single(recv, s, output_split_sizes=list(recv_rows), input_split_sizes=list(send_rows),
@@ -88,6 +96,8 @@ class TorchComm:
     def exchange_counts(self, send_rows):
         """Each rank's row counts for every destination -> the counts every
         source will send here."""
+        if self.skip:
+            return list(send_rows)
         dev = "cuda" if not self.host_staging else "cpu"
         s = torch.tensor(list(send_rows), dtype=torch.int64, device=dev)
         r = torch.empty_like(s)
@@ -164,9 +174,10 @@ class CudaOps:
         h_c = torch.empty((cap, I // 2), dtype=torch.uint8, device=dev)
         h_s = _u8(fp4_sf_tiled_bytes(cap, I), dev)
         fp4_moe_w13(a_c, a_s, state["g"], self.w, H, I, E, counts, toffs, cap, h_c, h_s)
-        y = torch.empty((R, H), dtype=torch.float32, device=dev)
-        fp4_moe_w2(h_c, h_s, self.w, H, I, E, counts, offsets, toffs, perm, wts, cap, y)
-        fp4_gather_rows(y, H * 4, inv, R, y_ret)  # received row i was routed to row inv[i]
+        # one slot per received row, so "slot order" is received order: w2 writes
+        # each output row straight to the position its record arrived at
+        fp4_moe_w2(h_c, h_s, self.w, H, I, E, counts, offsets, toffs, perm, wts, cap, y_ret,
+                   FP4_MOE_Y_BY_SLOT)
         return y_ret
 
     def combine(self, y, state):

@@ -86,6 +86,7 @@ typedef enum { FP4_OUT_F32 = 0, FP4_OUT_BF16 = 1 } fp4_out_dtype;
 #define FP4_GEMM_B_MXFP8 0x80u       /* fp4_gemm with FP4_GEMM_A_MXFP8: B is MXFP8 too */
 #define FP4_MOE_W4A8 0x100u          /* MoE layer / stages: MXFP4 weights, MXFP8 activations and h */
 #define FP4_MOE_DYNAMIC_H 0x200u     /* MoE layer (NVFP4, row tiles): h scale per expert from this batch */
+#define FP4_MOE_Y_BY_SLOT 0x800u     /* fp4_moe_w2: y row perm[r] (the routed slot t*topk+s) for routed row r */
 #define FP4_MX2NV_ALLOW_LOSSY 0x400u /* fp4_mx_to_nv_codes: re-quantize blocks below E4M3's range, never refuse a span */
 
 /* Human-readable name of a status code (static string). */
@@ -410,6 +411,9 @@ fp4_status fp4_moe_h_requant(const float *h_f32, const int32_t *counts, const in
 
 /* Grouped w2 GEMM: y[offsets[e]+i] = w[perm[row]] * h_g[e]*w2_g[e] * (h . W2_e^T)
  * y: fp32 [T*topk][H] in routed order; topk_weights may be NULL.
+ * FP4_MOE_Y_BY_SLOT: routed row r goes to y row perm[r] instead, i.e. y is in
+ * slot order (token t's slot s at row t*topk+s), stored row by row rather
+ * than by TMA boxes; not with FP4_MOE_PAIR_TILES.
  * FP4_MOE_MX: MXFP4 operands, y = w * (h . W2_e^T).  Tiling and
  * FP4_MOE_PAIR_TILES as for fp4_moe_w13. */
 fp4_status fp4_moe_w2(const uint8_t *h_codes, const uint8_t *h_sf, const fp4_moe_weights *w,

@@ -205,11 +205,42 @@ def test_ep_over_nccl_world_of_one():
         H, I, E, k = 512, 256, 8, 2
         c = moe_case.build(300, H, I, E, k, seed=41, zipf=1.1)
         ref = fp4.moe_layer(c.x, c.ids, c.w, c.weights, H, I, E)
-        comm = ep.TorchComm()
-        assert not comm.host_staging
+        comm = ep.TorchComm(always_exchange=True)  # run the NCCL collectives even for one rank
+        assert not comm.host_staging and not comm.skip
         ops = ep.CudaOps(ep.local_weights(c.weights, E, I, H, 1, 0), H, I, E, 1, 0)
         got = ep.moe_layer_ep(c.x, c.ids, c.w, ops, comm)
         torch.cuda.synchronize()
         assert torch.equal(got.view(torch.int16), ref.view(torch.int16))
     finally:
         dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("fmt", ["nv", "mx"])
+def test_w2_y_by_slot_is_the_slot_order_permutation(fmt):
+    """fp4_moe_w2 with FP4_MOE_Y_BY_SLOT writes routed row r's output at row
+    perm[r]: bit for bit the routed-order y permuted into slot order (k = 3,
+    ragged expert tails, rows of both the box-store and row-store paths)."""
+    import fp4_block_scaled_03_b200 as fp4
+    import synth
+    from tests import test_gpu_moe as TM
+
+    T, H, I, E, k = 300, 512, 256, 7, 3
+    c = moe_case.build(T, H, I, E, k, seed=13, fmt=fmt)
+    r = TM._route_gpu(c.ids, T, k, E)
+    cap = fp4.moe_rows_cap(T, k, E)
+    div = 2 if fmt == "mx" else 1
+    h_c = synth.random_codes((cap, I // 2), seed=6, device="cuda")
+    h_s = synth.random_e4m3_scales((fp4.fp4_sf_tiled_bytes(cap, I) // div,), seed=7, lo=0x70, hi=0x80,
+                                   device="cuda") if fmt == "mx" else \
+        synth.random_e4m3_scales((fp4.fp4_sf_tiled_bytes(cap, I),), seed=7, device="cuda")
+    flags = fp4.FP4_MOE_MX if fmt == "mx" else 0
+    y_routed = torch.full((T * k, H), float("nan"), dtype=torch.float32, device="cuda")
+    y_slot = torch.full((T * k, H), float("nan"), dtype=torch.float32, device="cuda")
+    fp4.fp4_moe_w2(h_c, h_s, c.weights, H, I, E, r["counts"], r["offsets"], r["tile_offsets"], r["perm"], c.w, cap,
+                   y_routed, flags)
+    fp4.fp4_moe_w2(h_c, h_s, c.weights, H, I, E, r["counts"], r["offsets"], r["tile_offsets"], r["perm"], c.w, cap,
+                   y_slot, flags | fp4.FP4_MOE_Y_BY_SLOT)
+    assert fp4.fp4_get_device_status() == 0
+    perm = r["perm"].long()
+    assert not torch.isnan(y_routed).any()
+    assert torch.equal(y_slot[perm].view(torch.int32), y_routed.view(torch.int32))
