@@ -106,7 +106,7 @@ struct Params {
   const int32_t *perm;
   const float *topk_w;
   float *y;
-  int y_by_slot;  // w2: y row perm[r] (the routed slot) instead of routed row r, stored row by row
+  int y_by_slot;  // w2: y row perm[r] (the routed slot) instead of routed row r
   unsigned int *status;
   uint64_t wait_limit;
 };
@@ -376,7 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool row_ok = row < ti.rows_valid;
       // w2: a warp whose 32 rows are all valid writes through TMA (collective
       // per warp); otherwise each valid row is stored by its own thread
-      const bool full_box = (EPI == EPI_W2) && !p.y_by_slot && (q * 32 + 32 <= ti.rows_valid);
+      const bool full_box = (EPI == EPI_W2) && (q * 32 + 32 <= ti.rows_valid);
       if (!row_ok) continue;
       float alpha;  // MXFP4 operands carry no tensor-level scale
       if (MX) alpha = 1.0f;
@@ -479,7 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 4; ++i) d[i] = make_float4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
           }
-        } else if (!full_box) {  // EPI_W2, a warp holding the expert's last rows, or y by slot
+        } else if (!full_box) {  // EPI_W2, a warp holding the expert's last rows
           const int64_t yrow = p.y_by_slot ? (int64_t)p.perm[ti.out_row0 + row] : (int64_t)(ti.out_row0 + row);
           float *dst = p.y + yrow * p.N + col0;
 #pragma unroll
@@ -487,7 +487,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             *reinterpret_cast<float4 *>(dst + i) = make_float4(__fmul_rn(w[i], scale), __fmul_rn(w[i + 1], scale),
                                                                __fmul_rn(w[i + 2], scale), __fmul_rn(w[i + 3], scale));
         } else {  // EPI_W2, all 32 rows valid: stage 32 x 8 boxes and store them with TMA
+          // (in slot order each staged row is copied out to its own y row
+          // instead: two lanes per 32-byte row segment, 16 rows per pass)
           uint8_t *stg = smStg + (warp - kFirstEpiWarp) * 1024;
+          int64_t yrow[2] = {0, 0};
+          if (p.y_by_slot) {
+            yrow[0] = p.perm[ti.out_row0 + q * 32 + (lane >> 1)];
+            yrow[1] = p.perm[ti.out_row0 + q * 32 + 16 + (lane >> 1)];
+          }
 #pragma unroll
           for (int bx = 0; bx < 4; ++bx) {
             if (lane == 0) bulk_wait_read_all();  // previous box has left the buffer
@@ -499,11 +506,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                   make_float4(__fmul_rn(w[c], scale), __fmul_rn(w[c + 1], scale), __fmul_rn(w[c + 2], scale),
                               __fmul_rn(w[c + 3], scale));
             }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-              tma_store_2d(&tmY, stg, col0 + 8 * bx, ti.out_row0 + q * 32);
-              bulk_commit();
+            if (!p.y_by_slot) {
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_2d(&tmY, stg, col0 + 8 * bx, ti.out_row0 + q * 32);
+                bulk_commit();
+              }
+            } else {
+              __syncwarp();
+#pragma unroll
+              for (int pass = 0; pass < 2; ++pass) {
+                const int r = pass * 16 + (lane >> 1), ch = lane & 1;
+                const float4 v = *reinterpret_cast<const float4 *>(stg + r * 32 + ((ch ^ ((r >> 2) & 1)) * 16));
+                *reinterpret_cast<float4 *>(p.y + yrow[pass] * p.N + col0 + 8 * bx + 4 * ch) = v;
+              }
+              __syncwarp();  // every lane has read the box before it is overwritten
             }
           }
         }

@@ -412,8 +412,7 @@ fp4_status fp4_moe_h_requant(const float *h_f32, const int32_t *counts, const in
 /* Grouped w2 GEMM: y[offsets[e]+i] = w[perm[row]] * h_g[e]*w2_g[e] * (h . W2_e^T)
  * y: fp32 [T*topk][H] in routed order; topk_weights may be NULL.
  * FP4_MOE_Y_BY_SLOT: routed row r goes to y row perm[r] instead, i.e. y is in
- * slot order (token t's slot s at row t*topk+s), stored row by row rather
- * than by TMA boxes; not with FP4_MOE_PAIR_TILES.
+ * slot order (token t's slot s at row t*topk+s); not with FP4_MOE_PAIR_TILES.
  * FP4_MOE_MX: MXFP4 operands, y = w * (h . W2_e^T).  Tiling and
  * FP4_MOE_PAIR_TILES as for fp4_moe_w13. */
 fp4_status fp4_moe_w2(const uint8_t *h_codes, const uint8_t *h_sf, const fp4_moe_weights *w,
