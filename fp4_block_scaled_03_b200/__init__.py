@@ -118,6 +118,7 @@ _SIGS = {
     "fp4_moe_ep_record_bytes": (_SZ, [_I64]),
     "fp4_moe_ep_pack": (ctypes.c_int, [_P, _P, _I64, _I32, _I64, _P, _P, _P, _I64, _I32, _P, _P]),
     "fp4_moe_ep_unpack": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P, _P, _P]),
+    "fp4_moe_ep_gather": (ctypes.c_int, [_P, _I64, _I64, _I32, _P, _P, _P, _P, _P, _I64, _P]),
     "fp4_gather_rows": (ctypes.c_int, [_P, _I64, _P, _I64, _P, _P]),
     "fp4_get_device_status": (ctypes.c_int, [_P]),
     "fp4_set_wait_limit_ns": (None, [ctypes.c_uint64]),
@@ -260,6 +261,11 @@ def fp4_moe_ep_pack(x_codes, x_sf, T, topk, H, expert_ids, topk_weights, perm, R
 def fp4_moe_ep_unpack(records, R, H, codes, sf, weights, expert_ids):
     _check(lib.fp4_moe_ep_unpack(_ptr(records), R, H, _ptr(codes), _ptr(sf), _ptr(weights), _ptr(expert_ids),
                                  _stream()), "fp4_moe_ep_unpack")
+
+
+def fp4_moe_ep_gather(records, R, H, E, offsets, tile_offsets, perm, a_codes, a_sf, rows_cap):
+    _check(lib.fp4_moe_ep_gather(_ptr(records), R, H, E, _ptr(offsets), _ptr(tile_offsets), _ptr(perm),
+                                 _ptr(a_codes), _ptr(a_sf), rows_cap, _stream()), "fp4_moe_ep_gather")
 
 
 def fp4_gather_rows(src, row_bytes, idx, n, dst):

@@ -19,7 +19,7 @@ namespace {
 
 constexpr int kWarps = 8;  // warps per CTA
 
-int64_t record_bytes(int64_t H) { return H / 2 + H / 16 + 16; }
+__host__ __device__ __forceinline__ int64_t record_bytes(int64_t H) { return H / 2 + H / 16 + 16; }
 
 int grid_rows(int64_t n) {
   int dev = 0, sms = 148;
@@ -60,13 +60,43 @@ __global__ void __launch_bounds__(32 * kWarps)
   const int64_t nc = H / 32, ns = H / 256, nr = nc + ns + 1;
   for (int64_t i = blockIdx.x * (int64_t)kWarps + (threadIdx.x >> 5); i < R; i += (int64_t)gridDim.x * kWarps) {
     const uint4 *in = rec + i * nr;
-    for (int64_t c = lane; c < nc; c += 32) codes[i * nc + c] = in[c];
-    for (int64_t c = lane; c < ns; c += 32) sf[i * ns + c] = in[nc + c];
+    if (codes)
+      for (int64_t c = lane; c < nc; c += 32) codes[i * nc + c] = in[c];
+    if (sf)
+      for (int64_t c = lane; c < ns; c += 32) sf[i * ns + c] = in[nc + c];
     if (lane == 0) {
       const uint4 tail = in[nc + ns];
       w[i] = __uint_as_float(tail.x);
       ids[i] = (int32_t)tail.y;
     }
+  }
+}
+
+// Received records -> expert-contiguous, 128-padded rows of codes and tiled
+// scales, as fp4_moe_gather does from canonical x (here the source rows are
+// records, read in place).  One warp per routed row.
+__global__ void __launch_bounds__(32 * kWarps)
+    ep_gather_kernel(const uint8_t *__restrict__ rec, int64_t H, int32_t E, const int32_t *__restrict__ offsets,
+                     const int32_t *__restrict__ tile_offsets, const int32_t *__restrict__ perm,
+                     uint8_t *__restrict__ a_codes, uint8_t *__restrict__ a_sf) {
+  const int lane = threadIdx.x & 31;
+  const int32_t nvalid = offsets[E];
+  const int64_t rb = record_bytes(H), nvec = H / 32, nwords = H / 64;
+  for (int64_t r = blockIdx.x * (int64_t)kWarps + (threadIdx.x >> 5); r < nvalid; r += (int64_t)gridDim.x * kWarps) {
+    int lo = 0, hi = E;  // the expert whose routed range holds r: offsets[e] <= r < offsets[e+1]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (offsets[mid] <= r) lo = mid; else hi = mid;
+    }
+    const int e = lo;
+    const int64_t dst = (int64_t)tile_offsets[e] * 128 + (r - offsets[e]);
+    const uint8_t *src = rec + (int64_t)perm[r] * rb;
+    const uint4 *cs = reinterpret_cast<const uint4 *>(src);
+    uint4 *out = reinterpret_cast<uint4 *>(a_codes + dst * (H / 2));
+    for (int64_t v = lane; v < nvec; v += 32) out[v] = cs[v];
+    const uint32_t *ss = reinterpret_cast<const uint32_t *>(src + H / 2);
+    const int64_t line = ((dst >> 7) * nwords) * 512 + (dst & 31) * 16 + ((dst >> 5) & 3) * 4;
+    for (int64_t w = lane; w < nwords; w += 32) *reinterpret_cast<uint32_t *>(a_sf + line + w * 512) = ss[w];
   }
 }
 
@@ -114,7 +144,7 @@ fp4_status fp4_moe_ep_unpack(const uint8_t *records, int64_t R, int64_t H, uint8
   if (R < 0 || H <= 0) return FP4_ERR_INVALID_ARG;
   if (H % 256) return FP4_ERR_UNSUPPORTED_SHAPE;
   if (R == 0) return FP4_OK;
-  if (!records || !codes || !sf || !weights || !expert_ids) return FP4_ERR_INVALID_ARG;
+  if (!records || !weights || !expert_ids) return FP4_ERR_INVALID_ARG;
   if (!al16(records) || !al16(codes) || !al16(sf) || (reinterpret_cast<uintptr_t>(weights) & 3u) ||
       (reinterpret_cast<uintptr_t>(expert_ids) & 3u))
     return FP4_ERR_ALIGNMENT;
@@ -122,6 +152,21 @@ fp4_status fp4_moe_ep_unpack(const uint8_t *records, int64_t R, int64_t H, uint8
   ep_unpack_kernel<<<grid_rows(R), 32 * kWarps, 0, s>>>(reinterpret_cast<const uint4 *>(records), R, H,
                                                        reinterpret_cast<uint4 *>(codes), reinterpret_cast<uint4 *>(sf),
                                                        weights, expert_ids);
+  FP4_HOST_CHECK(cudaGetLastError());
+  return FP4_OK;
+}
+
+fp4_status fp4_moe_ep_gather(const uint8_t *records, int64_t R, int64_t H, int32_t E, const int32_t *offsets,
+                             const int32_t *tile_offsets, const int32_t *perm, uint8_t *a_codes, uint8_t *a_sf,
+                             int64_t rows_cap, fp4_stream_t stream) {
+  if (R < 0 || H <= 0 || E < 1 || E > 4096) return FP4_ERR_INVALID_ARG;
+  if (H % 256) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (R == 0) return FP4_OK;
+  if (!records || !offsets || !tile_offsets || !perm || !a_codes || !a_sf) return FP4_ERR_INVALID_ARG;
+  if (rows_cap < R + 127LL * E) return FP4_ERR_WORKSPACE;
+  if (!al16(records) || !al16(a_codes) || (reinterpret_cast<uintptr_t>(a_sf) & 3u)) return FP4_ERR_ALIGNMENT;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  ep_gather_kernel<<<grid_rows(R), 32 * kWarps, 0, s>>>(records, H, E, offsets, tile_offsets, perm, a_codes, a_sf);
   FP4_HOST_CHECK(cudaGetLastError());
   return FP4_OK;
 }

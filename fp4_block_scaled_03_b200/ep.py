@@ -13,8 +13,8 @@ layer step on every rank is:
      pack them as fixed-size records (codes, scales, routing weight, local
      expert id: fp4_moe_ep_pack).
   3. all-to-all of the per-rank row counts, then of the records.
-  4. unpack; route the received rows over the local experts (one slot each);
-     gather them into expert tiles; grouped w13 (SwiGLU + h requant) and w2
+  4. route the received rows over the local experts (one slot each); gather
+     them from the records into expert tiles; grouped w13 (SwiGLU + h requant) and w2
      (routing weight) on tcgen05, w2 writing each output row back at the
      position its record arrived at.
   5. all-to-all of the fp32 output rows back to their senders: they arrive in
@@ -34,7 +34,7 @@ import torch
 import torch.distributed as dist
 
 from . import (FP4_MOE_Y_BY_SLOT, FP4_NV, FP4_STATIC_GLOBAL_SCALE, MoeWeightSet, _u8, fp4_amax_bf16,
-               fp4_moe_combine, fp4_moe_ep_pack, fp4_moe_ep_record_bytes, fp4_moe_ep_unpack, fp4_moe_gather,
+               fp4_moe_combine, fp4_moe_ep_gather, fp4_moe_ep_pack, fp4_moe_ep_record_bytes, fp4_moe_ep_unpack,
                fp4_moe_route, fp4_moe_route_scratch_bytes, fp4_moe_w13, fp4_moe_w2, fp4_nv_global_scale,
                fp4_quantize, fp4_sf_tiled_bytes, moe_rows_cap)
 
@@ -155,11 +155,9 @@ class CudaOps:
         y_ret = torch.empty((R, H), dtype=torch.float32, device=dev)
         if R == 0:
             return y_ret
-        codes = torch.empty((R, H // 2), dtype=torch.uint8, device=dev)
-        sf = torch.empty((R, H // 16), dtype=torch.uint8, device=dev)
         wts = torch.empty(R, dtype=torch.float32, device=dev)
         ids = torch.empty(R, dtype=torch.int32, device=dev)
-        fp4_moe_ep_unpack(records, R, H, codes, sf, wts, ids)
+        fp4_moe_ep_unpack(records, R, H, None, None, wts, ids)  # the rows stay in the records
         counts = torch.empty(E, dtype=torch.int32, device=dev)
         offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
         toffs = torch.empty(E + 1, dtype=torch.int32, device=dev)
@@ -170,7 +168,7 @@ class CudaOps:
         cap = moe_rows_cap(R, 1, E)
         a_c = torch.empty((cap, H // 2), dtype=torch.uint8, device=dev)
         a_s = _u8(fp4_sf_tiled_bytes(cap, H), dev)
-        fp4_moe_gather(codes, sf, R, 1, H, E, offsets, toffs, perm, a_c, a_s, cap)
+        fp4_moe_ep_gather(records, R, H, E, offsets, toffs, perm, a_c, a_s, cap)
         h_c = torch.empty((cap, I // 2), dtype=torch.uint8, device=dev)
         h_s = _u8(fp4_sf_tiled_bytes(cap, I), dev)
         fp4_moe_w13(a_c, a_s, state["g"], self.w, H, I, E, counts, toffs, cap, h_c, h_s)

@@ -444,7 +444,12 @@ fp4_status fp4_moe_combine(const float *y, const int32_t *inv, int64_t T, int32_
  *   (x_codes [T][H/2], x_sf canonical [T][H/16] from fp4_quantize with one
  *   global scale shared by all ranks), expert_ids/topk_weights [T*topk].
  * fp4_moe_ep_unpack -- the inverse on the receiving rank: codes [R][H/2],
- *   sf [R][H/16], weights [R], expert_ids [R] (local indices).
+ *   sf [R][H/16], weights [R], expert_ids [R] (local indices); codes and sf
+ *   may be NULL (only the weights and ids are written).
+ * fp4_moe_ep_gather -- fp4_moe_gather with the received records as the
+ *   source rows (read in place, routed over the local experts with one slot
+ *   per record): a_codes [rows_cap][H/2] and tiled a_sf for [rows_cap, H],
+ *   rows_cap >= R + 127*E.
  * fp4_gather_rows -- dst row i = src row idx[i] for i < n, rows of row_bytes
  *   (a multiple of 16); used to put expert outputs back in received order.
  * H % 256 == 0; buffers 16-byte aligned (weights and ids 4-byte).  R, n == 0
@@ -456,6 +461,9 @@ fp4_status fp4_moe_ep_pack(const uint8_t *x_codes, const uint8_t *x_sf, int64_t 
                            int32_t experts_per_rank, uint8_t *records, fp4_stream_t stream);
 fp4_status fp4_moe_ep_unpack(const uint8_t *records, int64_t R, int64_t H, uint8_t *codes, uint8_t *sf,
                              float *weights, int32_t *expert_ids, fp4_stream_t stream);
+fp4_status fp4_moe_ep_gather(const uint8_t *records, int64_t R, int64_t H, int32_t E, const int32_t *offsets,
+                             const int32_t *tile_offsets, const int32_t *perm, uint8_t *a_codes, uint8_t *a_sf,
+                             int64_t rows_cap, fp4_stream_t stream);
 fp4_status fp4_gather_rows(const void *src, int64_t row_bytes, const int32_t *idx, int64_t n, void *dst,
                            fp4_stream_t stream);
 

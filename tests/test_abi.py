@@ -96,6 +96,8 @@ def test_host_validation_without_gpu():
     assert L.fp4_moe_ep_pack(A, A, 4, 2, 256, A, None, A, 8, 2, A + 4, None) == 2
     assert L.fp4_moe_ep_unpack(A, 8, 256, A, A, A, None, None) == 1
     assert L.fp4_gather_rows(A, 20, A, 4, A, None) == 3
+    assert L.fp4_moe_ep_gather(A, 8, 320, 2, A, A, A, A, A, 1 << 20, None) == 3
+    assert L.fp4_moe_ep_gather(A, 8, 256, 2, A, A, A, A, A, 16, None) == 6
     assert L.fp4_amax_bf16(A, 4, 12, 12, A, None) == 3
     assert L.fp4_moe_ep_record_bytes(7168) == 3584 + 448 + 16
     # empty EP calls launch nothing and succeed with NULL buffers

@@ -244,3 +244,39 @@ def test_w2_y_by_slot_is_the_slot_order_permutation(fmt):
     perm = r["perm"].long()
     assert not torch.isnan(y_routed).any()
     assert torch.equal(y_slot[perm].view(torch.int32), y_routed.view(torch.int32))
+
+
+def test_ep_gather_from_records_equals_unpack_then_gather():
+    """fp4_moe_ep_gather reads the received records in place and fills the
+    expert tiles exactly as fp4_moe_ep_unpack followed by fp4_moe_gather
+    does (both buffers start zeroed, so padding rows compare too)."""
+    import fp4_block_scaled_03_b200 as fp4
+    from tests import test_gpu_moe as TM
+
+    R, H, E = 531, 1024, 6
+    rng = np.random.default_rng(17)
+    rb = fp4.fp4_moe_ep_record_bytes(H)
+    rec_np = rng.integers(0, 256, (R, rb), dtype=np.uint8)
+    rec_np[:, H // 2 + H // 16 + 4:H // 2 + H // 16 + 8] = 0
+    ids_np = rng.integers(0, E, R).astype(np.int32)
+    rec_np[:, H // 2 + H // 16 + 4:H // 2 + H // 16 + 8] = ids_np.view(np.uint8).reshape(R, 4)
+    rec = torch.from_numpy(rec_np).cuda()
+    w = torch.empty(R, dtype=torch.float32, device="cuda")
+    ids = torch.empty(R, dtype=torch.int32, device="cuda")
+    codes = torch.empty((R, H // 2), dtype=torch.uint8, device="cuda")
+    sf = torch.empty((R, H // 16), dtype=torch.uint8, device="cuda")
+    fp4.fp4_moe_ep_unpack(rec, R, H, codes, sf, w, ids)
+    assert np.array_equal(ids.cpu().numpy(), ids_np)
+    r = TM._route_gpu(ids.view(R, 1), R, 1, E)
+    cap = fp4.moe_rows_cap(R, 1, E)
+    outs = []
+    for via_records in (True, False):
+        a_c = torch.zeros((cap, H // 2), dtype=torch.uint8, device="cuda")
+        a_s = torch.zeros(fp4.fp4_sf_tiled_bytes(cap, H), dtype=torch.uint8, device="cuda")
+        if via_records:
+            fp4.fp4_moe_ep_gather(rec, R, H, E, r["offsets"], r["tile_offsets"], r["perm"], a_c, a_s, cap)
+        else:
+            fp4.fp4_moe_gather(codes, sf, R, 1, H, E, r["offsets"], r["tile_offsets"], r["perm"], a_c, a_s, cap)
+        outs.append((a_c, a_s))
+    assert fp4.fp4_get_device_status() == 0
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
