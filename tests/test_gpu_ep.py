@@ -280,3 +280,25 @@ def test_ep_gather_from_records_equals_unpack_then_gather():
         outs.append((a_c, a_s))
     assert fp4.fp4_get_device_status() == 0
     assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_ep_full_size_pro_layer_equals_single_gpu(world):
+    """The Pro-shaped layer at full size (16384 tokens, 384 experts, H 7168,
+    I 2048, top-6, Zipf 1.1), built as the bench builds it: split over
+    `world` emulated ranks, the expert-parallel output equals the 1-GPU
+    layer's bf16 output bit for bit (the 1-GPU layer is checked against the
+    oracle on sampled tokens in test_gpu_fullsize.py)."""
+    import bench
+
+    b = bench.MoeBench("pro", seed=0)
+    b.step()
+    torch.cuda.synchronize()
+    assert b.fp4.fp4_get_device_status() == 0
+
+    class _Case:
+        x, ids, w, weights = b.x, b.ids, b.w, b.wset
+
+    got = _run_ep(_Case, b.H, b.I, b.E, world, [b.T // world] * world)
+    assert b.fp4.fp4_get_device_status() == 0
+    assert torch.equal(got.view(torch.int16), b.out.view(torch.int16))
