@@ -48,6 +48,8 @@ WORKLOADS = {
                   "Flash-shaped MoE layer in W4A8: MXFP4 weights (UE8M0/32) x MXFP8 activations and h (E4M3, UE8M0/32)"),
     "pro64": (4096, 7168, 2048, 64, 6, 1.1, 0.01,
               "Pro-shaped expert matrices, 64 experts, 4096 tokens, top-6, Zipf 1.1 (profiling size)"),
+    "pro128k": (131072, 7168, 2048, 384, 6, 1.1, 0.01,
+                "Pro-shaped MoE layer at 131072 tokens (786432 routed rows; the largest token count quantized)"),
 }
 
 METRIC = "NVFP4 W4A4 grouped-MoE GEMM TFLOPS (% FP4 peak); quantize GB/s (% HBM)"

@@ -29,7 +29,8 @@ def _h_tol(xr, w1, w3, gate, up, h):
         4e-7 * np.abs(h) + 1e-30
 
 
-@pytest.mark.parametrize("workload,tokens", [("pro", [0, 9999]), ("decode", [63]), ("flash", [17]), ("flashmx", [5])])
+@pytest.mark.parametrize("workload,tokens", [("pro", [0, 9999]), ("decode", [63]), ("flash", [17]), ("flashmx", [5]),
+                                             ("pro128k", [131071])])
 def test_layer_full_size_sampled_tokens(workload, tokens):
     import bench
 
