@@ -486,6 +486,10 @@ def run_moe(args, world, rank, peaks):
         roof.update(bound="hbm", achieved=round(w13_gbs, 1), peak=round(peaks["hbm"], 1), unit="GB/s",
                     frac=round(w13_gbs / peaks["hbm"], 4), tensor_tflops=round(w13_tf, 1),
                     tensor_frac=round(w13_tf / fp4_peak, 4))
+    # the same launch counted over every MMA row, padding rows included: the
+    # kernel's tensor-pipe rate, as opposed to the useful work it delivers
+    roof.update(mma_rows_tflops=round(w13_tf * b.mma_rows() / max(1, b.R), 1),
+                mma_rows_frac=round(w13_tf * b.mma_rows() / max(1, b.R) / fp4_peak, 4))
     roof.update(traffic=measured_traffic(args.workload, b.kernel_name("w13")), algorithmic_bytes=w13_bytes,
                 frac_of_max_flops_bytes=round(max(t_flops, t_bytes) / (stage[2] * 1e-3), 4),
                 peak_note="tensor pipe: %dx sustained bf16 cuBLAS (nominal %s/bf16 ratio); HBM: copy bandwidth; of %s"
