@@ -327,10 +327,14 @@ class MoeBench:
         ev(5)
 
     def launches_per_step(self):
-        """Kernels one step launches: 3 routing; quantize + gather (NVFP4:
-        tensor amax, fused quantize-gather, scale transpose; MX / W4A8: one);
-        w13 (+ the h requant with a dynamic h scale); w2; combine."""
-        return 3 + (1 if self.mx else 3) + 1 + (1 if self.dynamic_h else 0) + 1 + 1
+        """Kernels one step launches: routing (one kernel up to 1024 routed
+        rows, else count, scan and scatter); quantize + gather (NVFP4: tensor
+        amax, fused quantize-gather, and above 4096 routed rows the scale
+        transpose; MX / W4A8: one); w13 (+ the h requant with a dynamic h
+        scale); w2; combine."""
+        route = 1 if self.R <= 1024 else 3
+        qg = 1 if self.mx else (2 if self.R <= 4096 else 3)
+        return route + qg + 1 + (1 if self.dynamic_h else 0) + 1 + 1
 
     def mma_rows(self):
         """Routed rows the grouped GEMMs run through the tensor cores: each

@@ -14,6 +14,7 @@ namespace fp4 {
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int64_t kDirectRows = 4096;  // routed rows up to which the gather writes tiled scales in place
 
 int grid_for(int64_t work_items, int per_cta = kThreads) {
   int dev = 0, sms = 148;
@@ -165,13 +166,17 @@ __device__ __forceinline__ void gather_destinations(const int32_t *__restrict__ 
 }
 
 // NVFP4: a lane's K step is 64 elements (four 16-element blocks).
+// kDirect = false: scale words go row-major to sf_rows [rows][H/64]
+// (coalesced); sf_rows_to_tiled_kernel then writes the tiled layout one
+// whole 512-byte tile at a time.  kDirect (small batches, where a launch
+// costs more than the scattered stores): each word goes straight to its
+// place in the tiled layout a_sf.
+template <bool kDirect>
 __global__ void __launch_bounds__(128) nvfp4_quantize_gather_kernel(
     const uint16_t *__restrict__ x, int64_t T, int64_t H, int32_t topk, int32_t E,
     const int32_t *__restrict__ offsets, const int32_t *__restrict__ tile_offsets, const int32_t *__restrict__ inv,
-    uint8_t *__restrict__ a_codes, uint32_t *__restrict__ sf_rows, const unsigned int *__restrict__ amax_bits,
-    float *__restrict__ g_out) {
-  // scale words go row-major to sf_rows [rows][H/64] (coalesced); sf_rows_to_tiled_kernel
-  // then writes the tiled layout one whole 512-byte tile at a time
+    uint8_t *__restrict__ a_codes, uint32_t *__restrict__ sf_rows, uint8_t *__restrict__ a_sf,
+    const unsigned int *__restrict__ amax_bits, float *__restrict__ g_out) {
   const float g = __fdiv_rn(__uint_as_float(*amax_bits), 2688.0f);
   if (blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
   const int lane = threadIdx.x & 31;
@@ -213,7 +218,11 @@ __global__ void __launch_bounds__(128) nvfp4_quantize_gather_kernel(
         uint4 *out = reinterpret_cast<uint4 *>(a_codes + d * (H / 2) + kw * 32);
         out[0] = make_uint4(code[0], code[1], code[2], code[3]);
         out[1] = make_uint4(code[4], code[5], code[6], code[7]);
-        sf_rows[d * n_ksteps + kw] = sfw;
+        if (kDirect)  // the word of K step kw of row d: bytes 4 consecutive 16-blocks
+          *reinterpret_cast<uint32_t *>(a_sf + ((d >> 7) * n_ksteps + kw) * 512 + (d & 31) * 16 + ((d >> 5) & 3) * 4) =
+              sfw;
+        else
+          sf_rows[d * n_ksteps + kw] = sfw;
       }
 #pragma unroll
       for (int q = 0; q < 8; ++q) v[q] = vn[q];
@@ -840,8 +849,14 @@ fp4_status fp4_moe_quantize_gather(const void *x_bf16, int64_t T, int32_t topk, 
   const int64_t need = (T + 3) / 4;  // four rows (warps) per CTA
   const int64_t grid = need < (int64_t)sms * 16 ? need : (int64_t)sms * 16;
   uint32_t *sf_rows = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(workspace) + 256);
-  nvfp4_quantize_gather_kernel<<<(unsigned)grid, 128, 0, s>>>(x, T, H, topk, E, offsets, tile_offsets, inv, a_codes,
-                                                               sf_rows, amax, global_scale);
+  if (T * topk <= kDirectRows) {  // small batch: tiled scale words written in place, no transpose launch
+    nvfp4_quantize_gather_kernel<true><<<(unsigned)grid, 128, 0, s>>>(x, T, H, topk, E, offsets, tile_offsets, inv,
+                                                                      a_codes, sf_rows, a_sf, amax, global_scale);
+    FP4_HOST_CHECK(cudaGetLastError());
+    return FP4_OK;
+  }
+  nvfp4_quantize_gather_kernel<false><<<(unsigned)grid, 128, 0, s>>>(x, T, H, topk, E, offsets, tile_offsets, inv,
+                                                                     a_codes, sf_rows, a_sf, amax, global_scale);
   FP4_HOST_CHECK(cudaGetLastError());
   const int64_t jobs = (rows_cap / 128) * ((H / 64 + 31) / 32);  // an upper bound; the kernel stops at the routed rows
   const int64_t tgrid = jobs < (int64_t)sms * 8 ? (jobs > 0 ? jobs : 1) : (int64_t)sms * 8;

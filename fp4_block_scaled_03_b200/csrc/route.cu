@@ -144,6 +144,85 @@ __global__ void route_scatter_kernel(const int32_t *__restrict__ ids, int64_t R,
   }
 }
 
+// Routing of at most one chunk (R <= kChunk) in one CTA: the three passes
+// above back to back through shared memory -- histogram (warp 0, slot order),
+// exclusive prefixes over experts of rows and 128-row tiles (all threads),
+// stable scatter (warp 0) -- one launch instead of three for decode-sized
+// batches.  Same outputs as the three-kernel path; R = 0 writes zero tables.
+__global__ void __launch_bounds__(1024) route_small_kernel(const int32_t *__restrict__ ids, int64_t R, int32_t E,
+                                                           int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
+                                                           int32_t *__restrict__ tile_offsets,
+                                                           int32_t *__restrict__ perm, int32_t *__restrict__ inv,
+                                                           unsigned int *__restrict__ status) {
+  extern __shared__ int32_t sm[];  // cnt[E] | run[E] | rows[blockDim] | tiles[blockDim]
+  int32_t *cnt = sm, *run = sm + E, *s_rows = sm + 2 * E, *s_tiles = s_rows + blockDim.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  if (warp == 0) {
+    for (int64_t f0 = 0; f0 < R; f0 += 32) {  // uniform over the warp
+      const int64_t f = f0 + lane;
+      int id = f < R ? ids[f] : -1;
+      if (f < R && (id < 0 || id >= E)) {
+        record_status(status, FP4_ERR_BAD_EXPERT);
+        id = -1;
+      }
+      const uint32_t grp = __match_any_sync(0xffffffffu, id);
+      if (id >= 0 && (grp & lanemask_lt()) == 0) cnt[id] += __popc(grp);
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+  const int per = (E + (int)blockDim.x - 1) / (int)blockDim.x, e0 = (int)threadIdx.x * per;
+  int32_t local_rows = 0, local_tiles = 0;
+  for (int e = e0; e < e0 + per && e < E; ++e) {
+    local_rows += cnt[e];
+    local_tiles += (cnt[e] + 127) / 128;
+  }
+  s_rows[threadIdx.x] = local_rows;
+  s_tiles[threadIdx.x] = local_tiles;
+  __syncthreads();
+  for (int o = 1; o < (int)blockDim.x; o <<= 1) {  // inclusive Hillis-Steele scan over threads
+    const int32_t a = (int)threadIdx.x >= o ? s_rows[threadIdx.x - o] : 0;
+    const int32_t b = (int)threadIdx.x >= o ? s_tiles[threadIdx.x - o] : 0;
+    __syncthreads();
+    s_rows[threadIdx.x] += a;
+    s_tiles[threadIdx.x] += b;
+    __syncthreads();
+  }
+  int32_t row_base = s_rows[threadIdx.x] - local_rows, tile_base = s_tiles[threadIdx.x] - local_tiles;
+  for (int e = e0; e < e0 + per && e < E; ++e) {
+    counts[e] = cnt[e];
+    offsets[e] = row_base;
+    tile_offsets[e] = tile_base;
+    run[e] = row_base;
+    row_base += cnt[e];
+    tile_base += (cnt[e] + 127) / 128;
+  }
+  if (threadIdx.x == blockDim.x - 1) {
+    offsets[E] = s_rows[threadIdx.x];
+    tile_offsets[E] = s_tiles[threadIdx.x];
+  }
+  __syncthreads();
+  if (warp == 0) {
+    for (int64_t f0 = 0; f0 < R; f0 += 32) {
+      const int64_t f = f0 + lane;
+      int id = f < R ? ids[f] : -1;
+      if (id < 0 || id >= E) id = -1;
+      const uint32_t grp = __match_any_sync(0xffffffffu, id);
+      int32_t pos = -1;
+      if (id >= 0) pos = run[id] + __popc(grp & lanemask_lt());
+      __syncwarp();
+      if (id >= 0 && (grp & lanemask_lt()) == 0) run[id] += __popc(grp);
+      __syncwarp();
+      if (f < R) {
+        inv[f] = pos;
+        if (pos >= 0) perm[pos] = (int32_t)f;
+      }
+    }
+  }
+}
+
 __device__ __forceinline__ int find_expert(const int32_t *__restrict__ offsets, int E, int32_t r) {
   // largest e with offsets[e] <= r < offsets[e+1]  (upper_bound(offsets, r) - 1)
   int lo = 0, hi = E;  // offsets[lo] <= r < offsets[hi]
@@ -323,6 +402,12 @@ fp4_status fp4_moe_route(const int32_t *expert_ids, int64_t T, int32_t topk, int
   const int nchunks = (int)((R + kChunk - 1) / kChunk);
   int32_t *cc = static_cast<int32_t *>(scratch);
   const size_t esm = (size_t)E * 4;
+  if (nchunks <= 1) {  // one chunk or none: the single-CTA path
+    route_small_kernel<<<1, 1024, (size_t)(2 * E + 2 * 1024) * 4, s>>>(expert_ids, R, E, counts, offsets,
+                                                                       tile_offsets, perm, inv, ctx->status);
+    FP4_HOST_CHECK(cudaGetLastError());
+    return FP4_OK;
+  }
   if (nchunks > 0) {
     route_count_kernel<<<nchunks, 32, esm, s>>>(expert_ids, R, E, cc, ctx->status);
     FP4_HOST_CHECK(cudaGetLastError());
