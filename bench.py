@@ -667,7 +667,9 @@ def run_moe_ep(args, world, rank, peaks):
         "roofline": None,
         "note": "layer step through moe_layer_ep: amax all-reduce, quantize, route, record all-to-all, local"
                 " grouped GEMMs, output all-to-all, combine; no per-kernel roofline on this line",
-        "gpu_launches": 16 * args.steps, "clocks": clocks,
+        # amax, global scale, quantize, pack, unpack (weights and ids), records gather, w13, w2, combine,
+        # and two routings (one kernel up to 1024 rows, else three; the local one taken at this rank's R)
+        "gpu_launches": (9 + 2 * (1 if b.R <= 1024 else 3)) * args.steps, "clocks": clocks,
     }
     dist.destroy_process_group()
     return line
