@@ -474,6 +474,29 @@ def run_moe(args, world, rank, peaks):
     assert fp4.fp4_get_device_status() == 0
     h2d = b.T * b.H * 2 + b.R * 4 + b.R * 4
     d2h = b.T * b.H * 2
+
+    graph = None
+    if args.graph:  # the layer call captured once in a CUDA graph, replayed per step (inputs resident)
+        out_g = torch.empty((b.T, b.H), dtype=torch.bfloat16, device="cuda")
+        fp4.fp4_moe_grouped_gemm(b.x, b.ids, b.w, b.T, b.k, b.wset, b.H, b.I, b.E, out_g, ws, b.flags)
+        torch.cuda.synchronize()
+        cg = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(cg):
+            fp4.fp4_moe_grouped_gemm(b.x, b.ids, b.w, b.T, b.k, b.wset, b.H, b.I, b.E, out_g, ws, b.flags)
+        for _ in range(args.warmup):
+            cg.replay()
+        torch.cuda.synchronize()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record()
+        for _ in range(args.steps):
+            cg.replay()
+        g1.record()
+        torch.cuda.synchronize()
+        g_ms = max_over_ranks(g0.elapsed_time(g1) / args.steps, world)
+        assert fp4.fp4_get_device_status() == 0
+        graph = {"ms_per_step": round(g_ms, 4), "value": round(world * flops / (g_ms * 1e-3) / 1e12, 2),
+                 "unit": "TFLOP/s", "how": "fp4_moe_grouped_gemm captured once in a CUDA graph, replayed per step"}
+        del cg, out_g
     del ws
 
     # the w13 launch's roofline: the tensor pipe when its FLOPs take longer at
@@ -541,6 +564,8 @@ def run_moe(args, world, rank, peaks):
         "gpu_launches": b.launches_per_step() * args.steps,
         "clocks": clocks,
     }
+    if graph is not None:
+        line["graph"] = graph
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_moe(b)
     return line
@@ -936,6 +961,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--dynamic-h", action="store_true",
                     help="NVFP4 MoE workloads: per-expert h scale from each batch (two-phase w13)")
+    ap.add_argument("--graph", action="store_true",
+                    help="MoE workloads: also time the layer call replayed from a CUDA graph")
     ap.add_argument("--ep", action="store_true",
                     help="NVFP4 MoE workloads: the expert-parallel layer over NCCL (experts split over the ranks)")
     ap.add_argument("--pair-tiles", action="store_true",

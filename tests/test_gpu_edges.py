@@ -67,3 +67,40 @@ def test_layer_ragged_tiles(tiling):
     """129 tokens x top-2 over 3 experts: every expert's rows end in a ragged
     tile (and, for CTA pairs, a ragged 256-row chunk)."""
     TM.test_layer_end_to_end(129, 256, 512, 3, 2, 0.0, tiling)
+
+
+@pytest.mark.parametrize("T,E,k", [(64, 384, 6), (1000, 16, 6)])
+def test_layer_cuda_graph_replay(T, E, k):
+    """The whole layer call captured in a CUDA graph (after one eager call
+    has set up the library's per-device state): a replay gives the eager
+    output bit for bit, and after new inputs are copied into the captured
+    buffers a replay gives the eager output for those inputs.  T = 64 takes
+    the small-batch routing and gather paths, T = 1000 the chunked ones."""
+    import fp4_block_scaled_03_b200 as fp4
+    import synth
+
+    H, I = 512, 256
+    c = moe_case.build(T, H, I, E, k, seed=T + 3)
+    ws = torch.empty(fp4.fp4_moe_workspace_size_flags(T, k, H, I, E, 0), dtype=torch.uint8, device="cuda")
+    out = torch.empty((T, H), dtype=torch.bfloat16, device="cuda")
+    fp4.moe_layer(c.x, c.ids, c.w, c.weights, H, I, E, workspace=ws, out=out)
+    torch.cuda.synchronize()
+    ref = out.clone()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        fp4.moe_layer(c.x, c.ids, c.w, c.weights, H, I, E, workspace=ws, out=out)
+    out.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert fp4.fp4_get_device_status() == 0
+    assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+    x2 = synth.activations_bf16((T, H), seed=T + 99, device="cuda")
+    ids2, w2, _ = synth.router(T, E, k, seed=T + 98, device="cuda")
+    c.x.copy_(x2)
+    c.ids.copy_(ids2)
+    c.w.copy_(w2)
+    graph.replay()
+    torch.cuda.synchronize()
+    ref2 = fp4.moe_layer(x2, ids2, w2, c.weights, H, I, E)
+    assert torch.equal(out.view(torch.int16), ref2.view(torch.int16))
+    del graph
