@@ -98,6 +98,8 @@ _SIGS = {
     ),
     "fp4_moe_route_scratch_bytes": (_SZ, [_I64, _I32]),
     "fp4_moe_topk": (ctypes.c_int, [_P, _I64, _I32, _I32, _P, _P, _P]),
+    "fp4_moe_router_route": (ctypes.c_int, [_P, _I64, _I64, _P, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ,
+                                            _P]),
     "fp4_moe_route": (ctypes.c_int, [_P, _I64, _I32, _I32, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "fp4_moe_route_noalloc": (ctypes.c_int, [_P, _I64, _I32, _I32, _P, _P, _P, _P, _P, _P]),
     "fp4_moe_gather": (ctypes.c_int, [_P, _P, _I64, _I32, _I64, _I32, _P, _P, _P, _P, _P, _I64, _P]),
@@ -182,6 +184,14 @@ def fp4_gemm(a_codes, a_sf, a_g, b_codes, b_sf, b_g, c, c_dtype, M, N, K, flags=
 def fp4_moe_topk(logits, T, E, topk, expert_ids, topk_weights):
     _check(lib.fp4_moe_topk(_ptr(logits), T, E, topk, _ptr(expert_ids), _ptr(topk_weights), _stream()),
            "fp4_moe_topk")
+
+
+def fp4_moe_router_route(x, T, H, gate_w, E, topk, logits, expert_ids, topk_weights, counts, offsets, tile_offsets,
+                         perm, inv, scratch):
+    _check(lib.fp4_moe_router_route(_ptr(x), T, H, _ptr(gate_w), E, topk, _ptr(logits), _ptr(expert_ids),
+                                    _ptr(topk_weights), _ptr(counts), _ptr(offsets), _ptr(tile_offsets), _ptr(perm),
+                                    _ptr(inv), _ptr(scratch), scratch.numel() * scratch.element_size(), _stream()),
+           "fp4_moe_router_route")
 
 
 def fp4_moe_route(expert_ids, T, topk, E, counts, offsets, tile_offsets, perm, inv, scratch):

@@ -299,8 +299,12 @@ __global__ void combine_kernel(const float *__restrict__ y, const int32_t *__res
 // Router top-k: one warp per token.  Each of k rounds takes the warp-wide
 // largest remaining logit (ties to the lower expert id); the weights are the
 // softmax of the k chosen logits, fp32, summed in slot order.
+// With chunk_counts (zeroed, [nchunks][E]), each chosen slot also counts
+// into its routing chunk's histogram: the count pass of the routing, done
+// while the ids are in registers.
 __global__ void topk_softmax_kernel(const float *__restrict__ logits, int64_t T, int32_t E, int32_t k,
-                                    int32_t *__restrict__ ids, float *__restrict__ weights) {
+                                    int32_t *__restrict__ ids, float *__restrict__ weights,
+                                    int32_t *__restrict__ chunk_counts) {
   const int lane = threadIdx.x & 31;
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
   for (int64_t t = blockIdx.x * (int64_t)(blockDim.x / 32) + (threadIdx.x >> 5); t < T; t += warps) {
@@ -334,6 +338,7 @@ __global__ void topk_softmax_kernel(const float *__restrict__ logits, int64_t T,
       for (int s = 0; s < k; ++s) {
         ids[t * k + s] = chosen[s];
         weights[t * k + s] = __fdiv_rn(e[s], sum);
+        if (chunk_counts) atomicAdd(chunk_counts + ((t * k + s) / kChunk) * E + chosen[s], 1);
       }
     }
   }
@@ -430,7 +435,7 @@ fp4_status fp4_moe_topk(const float *logits, int64_t T, int32_t E, int32_t topk,
   int64_t grid = (T + 7) / 8;
   const int64_t cap = (int64_t)sm_count() * 16;
   if (grid > cap) grid = cap;
-  topk_softmax_kernel<<<(unsigned)grid, 256, 0, s>>>(logits, T, E, topk, expert_ids, topk_weights);
+  topk_softmax_kernel<<<(unsigned)grid, 256, 0, s>>>(logits, T, E, topk, expert_ids, topk_weights, nullptr);
   FP4_HOST_CHECK(cudaGetLastError());
   return FP4_OK;
 }
@@ -444,6 +449,43 @@ fp4_status fp4_moe_router(const void *x_bf16, int64_t T, int64_t H, const void *
   const fp4_status st = fp4_gemm_bf16(x_bf16, gate_w_bf16, logits, T, E, H, stream);
   if (st != FP4_OK) return st;
   return fp4_moe_topk(logits, T, E, topk, expert_ids, topk_weights, stream);
+}
+
+fp4_status fp4_moe_router_route(const void *x_bf16, int64_t T, int64_t H, const void *gate_w_bf16, int32_t E,
+                                int32_t topk, float *logits, int32_t *expert_ids, float *topk_weights, int32_t *counts,
+                                int32_t *offsets, int32_t *tile_offsets, int32_t *perm, int32_t *inv, void *scratch,
+                                size_t scratch_bytes, fp4_stream_t stream) {
+  if (T < 0 || H < 64 || H % 64 || E < 8 || E % 8 || E > 4096 || topk < 1 || topk > 16 || topk > E)
+    return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (!counts || !offsets || !tile_offsets || !scratch) return FP4_ERR_INVALID_ARG;
+  const int64_t R = T * topk;
+  if (R > 2147483647LL / 2) return FP4_ERR_UNSUPPORTED_SHAPE;
+  if (T > 0 && (!x_bf16 || !gate_w_bf16 || !logits || !expert_ids || !topk_weights || !perm || !inv))
+    return FP4_ERR_INVALID_ARG;
+  if (scratch_bytes < fp4_moe_route_scratch_bytes(R, E)) return FP4_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(scratch) & 3u)) return FP4_ERR_ALIGNMENT;
+  const int nchunks = (int)((R + kChunk - 1) / kChunk);
+  if (nchunks <= 1) {  // one chunk or none: the router, then the single-CTA routing
+    fp4_status st = fp4_moe_router(x_bf16, T, H, gate_w_bf16, E, topk, logits, expert_ids, topk_weights, stream);
+    if (st != FP4_OK) return st;
+    return fp4_moe_route(expert_ids, T, topk, E, counts, offsets, tile_offsets, perm, inv, scratch, scratch_bytes,
+                         stream);
+  }
+  const fp4_status st = fp4_gemm_bf16(x_bf16, gate_w_bf16, logits, T, E, H, stream);
+  if (st != FP4_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int32_t *cc = static_cast<int32_t *>(scratch);
+  FP4_HOST_CHECK(cudaMemsetAsync(cc, 0, (size_t)nchunks * E * 4, s));
+  int64_t grid = (T + 7) / 8;
+  const int64_t cap = (int64_t)sm_count() * 16;
+  if (grid > cap) grid = cap;
+  topk_softmax_kernel<<<(unsigned)grid, 256, 0, s>>>(logits, T, E, topk, expert_ids, topk_weights, cc);
+  FP4_HOST_CHECK(cudaGetLastError());
+  route_scan_kernel<<<1, 1024, 2 * 1024 * 4, s>>>(cc, nchunks, E, counts, offsets, tile_offsets);
+  FP4_HOST_CHECK(cudaGetLastError());
+  route_scatter_kernel<<<nchunks, 32, (size_t)E * 4, s>>>(expert_ids, R, E, cc, perm, inv);
+  FP4_HOST_CHECK(cudaGetLastError());
+  return FP4_OK;
 }
 
 fp4_status fp4_moe_gather(const uint8_t *x_codes, const uint8_t *x_sf, int64_t T, int32_t topk, int64_t H,

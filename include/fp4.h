@@ -318,6 +318,22 @@ fp4_status fp4_moe_router(const void *x_bf16, int64_t T, int64_t H, const void *
 fp4_status fp4_moe_topk(const float *logits, int64_t T, int32_t E, int32_t topk, int32_t *expert_ids,
                         float *topk_weights, fp4_stream_t stream);
 
+/*
+ * fp4_moe_router_route -- fp4_moe_router followed by fp4_moe_route over the
+ * ids it picks, with the routing's count pass fused into the top-k kernel
+ * ["DeepSeek-V4 FP4 QAT" §3.1; each chosen (token, slot) is counted into its
+ * routing chunk's per-expert histogram while the ids are in registers].
+ * Outputs: logits, expert_ids, topk_weights as fp4_moe_router; counts,
+ * offsets, tile_offsets, perm, inv as fp4_moe_route (bit for bit the same
+ * tables as the two calls).  scratch as for fp4_moe_route
+ * (fp4_moe_route_scratch_bytes(T*topk, E) bytes, 4-byte aligned).
+ * Shapes: H % 64 == 0; E % 8 == 0, 8 <= E <= 4096; 1 <= topk <= min(16, E).
+ */
+fp4_status fp4_moe_router_route(const void *x_bf16, int64_t T, int64_t H, const void *gate_w_bf16, int32_t E,
+                                int32_t topk, float *logits, int32_t *expert_ids, float *topk_weights, int32_t *counts,
+                                int32_t *offsets, int32_t *tile_offsets, int32_t *perm, int32_t *inv, void *scratch,
+                                size_t scratch_bytes, fp4_stream_t stream);
+
 /* Routing tables written by fp4_moe_route (all device int32):
  *   counts[E]          rows per expert
  *   offsets[E+1]       exclusive prefix of counts (row index in routed order)

@@ -100,6 +100,9 @@ def test_host_validation_without_gpu():
     assert L.fp4_moe_ep_gather(A, 8, 256, 2, A, A, A, A, A, 16, None) == 6
     assert L.fp4_amax_bf16(A, 4, 12, 12, A, None) == 3
     assert L.fp4_moe_ep_record_bytes(7168) == 3584 + 448 + 16
+    # fused router + routing: E % 8, too little scratch
+    assert L.fp4_moe_router_route(A, 64, 512, A, 12, 2, A, A, A, A, A, A, A, A, A, 1 << 20, None) == 3
+    assert L.fp4_moe_router_route(A, 4096, 512, A, 384, 6, A, A, A, A, A, A, A, A, A, 16, None) == 6
     # empty EP calls launch nothing and succeed with NULL buffers
     assert L.fp4_moe_ep_pack(None, None, 0, 2, 256, None, None, None, 0, 2, None, None) == 0
     assert L.fp4_gather_rows(None, 16, None, 0, None, None) == 0

@@ -67,3 +67,36 @@ def test_router_gate_and_topk(T, H, E, k):
         if rest:
             tol = 2 * G.FP32_REL_TOL * bound[t].max()
             assert min(L[t, list(sel)]) >= max(L[t, rest]) - tol
+
+
+@pytest.mark.parametrize("T,H,E,k", [(16384, 1024, 384, 6), (3000, 512, 64, 8), (100, 512, 64, 6), (0, 512, 64, 6)])
+def test_router_route_fused_equals_router_then_route(T, H, E, k):
+    """fp4_moe_router_route (the routing's count pass done by the top-k
+    kernel) gives the same ids, weights, logits and routing tables, bit for
+    bit, as fp4_moe_router followed by fp4_moe_route."""
+    fp4 = _lib()
+    x = synth.activations_bf16((max(T, 1), H), seed=T + 1, device="cuda")[:T]
+    wg = synth.weights_bf16((E, H), 0.02, 0.0, 1.0, seed=E + 2, device="cuda")
+    R = T * k
+    scratch = torch.empty(max(fp4.fp4_moe_route_scratch_bytes(R, E), 4), dtype=torch.uint8, device="cuda")
+
+    def tables():
+        return dict(logits=torch.full((max(T, 1), E), -7.0, device="cuda"),
+                    ids=torch.full((max(T, 1), k), -7, dtype=torch.int32, device="cuda"),
+                    w=torch.full((max(T, 1), k), -7.0, device="cuda"),
+                    counts=torch.full((E,), -7, dtype=torch.int32, device="cuda"),
+                    offsets=torch.full((E + 1,), -7, dtype=torch.int32, device="cuda"),
+                    toffs=torch.full((E + 1,), -7, dtype=torch.int32, device="cuda"),
+                    perm=torch.full((max(R, 1),), -7, dtype=torch.int32, device="cuda"),
+                    inv=torch.full((max(R, 1),), -7, dtype=torch.int32, device="cuda"))
+
+    a, b = tables(), tables()
+    fp4.fp4_moe_router_route(x, T, H, wg, E, k, a["logits"], a["ids"], a["w"], a["counts"], a["offsets"], a["toffs"],
+                             a["perm"], a["inv"], scratch)
+    fp4.fp4_moe_router(x, T, H, wg, E, k, b["logits"], b["ids"], b["w"])
+    fp4.fp4_moe_route(b["ids"], T, k, E, b["counts"], b["offsets"], b["toffs"], b["perm"], b["inv"], scratch)
+    assert fp4.fp4_get_device_status() == 0
+    for name in a:
+        assert torch.equal(a[name], b[name]), name
+    if T:
+        assert int(a["offsets"][E]) == R
