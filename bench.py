@@ -604,6 +604,11 @@ def cpu_baseline_moe(b, n_tokens=1):
             return Q.nvfp4_dequantize(c, sf, gg[0])
         return Q.nvfp4_dequantize(*Q.nvfp4_quantize(w))
 
+    # one host thread, stated as such: the oracle's time is its elementwise
+    # numpy quantizers (single-threaded); its small matmuls get no extra BLAS threads
+    from threadpoolctl import threadpool_limits
+
+    limits = threadpool_limits(limits=1)
     t0 = time.perf_counter()
     if b.w4a8:
         x_dq = Q.mxfp8_dequantize(*Q.mxfp8_quantize(xs))
@@ -625,9 +630,10 @@ def cpu_baseline_moe(b, n_tokens=1):
                 r = MO.expert_ffn_ref(x_dq[t:t + 1], w1d, w3d, w2d, hg[e])
             out[t] += wts[t, s] * r["y"][0]
     dt = time.perf_counter() - t0
+    limits.restore_original_limits()
     flops = 2.0 * 3 * b.H * b.I * b.k * n_tokens
-    return {"value": round(flops / dt / 1e12, 9), "unit": "TFLOP/s", "cores": len(os.sched_getaffinity(0)),
-            "kind": "oracle",
+    return {"value": round(flops / dt / 1e12, 9), "unit": "TFLOP/s", "cores": 1,
+            "host_cores_available": len(os.sched_getaffinity(0)), "kind": "oracle",
             "sample": f"{n_tokens} token(s) x top-{b.k} experts of the same layer, including the oracle's own"
                       f" quantize/dequantize of the {len(experts)} touched experts' weights: {dt:.1f} s"}
 
@@ -942,12 +948,15 @@ def cpu_dense_sample(rows=64):
     from oracle import gemm as G
     from oracle import quant as Q
 
+    from threadpoolctl import threadpool_info
+
     t0 = time.perf_counter()
     a = synth.activations_bf16((rows, 4096), seed=0).float().numpy()
     b = synth.weights_bf16((4096, 4096), 0.02, 0.005, 30.0, seed=1).float().numpy()
     G.nvfp4_gemm_ref(*Q.nvfp4_quantize(a), *Q.nvfp4_quantize(b))
     dt = time.perf_counter() - t0
-    return {"value": 2.0 * rows * 4096 * 4096 / dt / 1e12, "unit": "TFLOP/s", "cores": len(os.sched_getaffinity(0)),
+    blas = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])  # the fp64 matmul's BLAS threads
+    return {"value": 2.0 * rows * 4096 * 4096 / dt / 1e12, "unit": "TFLOP/s", "cores": blas,
             "kind": "oracle", "sample": f"{rows} rows of the 4096^3 GEMM, {dt:.1f} s"}
 
 
