@@ -608,6 +608,7 @@ def cpu_baseline_moe(b, n_tokens=1):
     # numpy quantizers (single-threaded); its small matmuls get no extra BLAS threads
     from threadpoolctl import threadpool_limits
 
+    _ = np.ones((2, 2)) @ np.ones((2, 2))  # load BLAS first: threadpoolctl only sees loaded libraries
     limits = threadpool_limits(limits=1)
     t0 = time.perf_counter()
     if b.w4a8:
