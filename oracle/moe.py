@@ -3,6 +3,12 @@ re-quantize -> w2), combine.
 
 TEST INFRASTRUCTURE ONLY (see ``oracle/__init__``).
 
+Parity unpinned: expert_ffn_ref, expert_ffn_ref_mx and expert_ffn_ref_w4a8.
+The pages print no worked example of an expert or a layer, so these are
+checked only as compositions of pinned parts (the quantizers, the fp64
+matmul, SiLU's closed forms).  route, topk_softmax and combine_ref are
+pinned (library stable sort, brute force, hand-worked sums).
+
 Sources: "DeepSeek-V4 FP4 QAT" page §3.1 (simplified MoE forward: each token
 goes to its top-k experts, the expert outputs are summed); "DeepSeek-V4
 architecture" §2.1 (Pro: 384 routed experts, 6 active) and §5.1 (SwiGLU
