@@ -30,9 +30,9 @@ Modules:
 Parity pins: every function here is checked by ``tests/test_oracle_*.py``
 against something other than itself (the pages' table, a library cast,
 exhaustive brute force, closed-form integer GEMMs, invariants).  The
-exhaustive 2^32 sweeps live in ``oracle/sweep.c``.  One exception: the
-expert FFN (``moe.expert_ffn_ref`` and its MXFP4 / W4A8 variants) is
-parity unpinned -- the pages print no worked example of a layer, so it is
-checked only as the composition of its pinned parts (the quantizers, the
-GEMM, the SiLU closed forms).
+exhaustive 2^32 sweeps live in ``oracle/sweep.c``.  The pages print no
+worked example of an expert; the expert FFN (``moe.expert_ffn_ref`` and its
+MXFP4 / W4A8 variants) is pinned by a case worked by hand
+(``tests/golden/expert_ffn_hand.txt``) where SiLU and every re-quantization
+are exact, so a swapped gate/up, a missing SiLU or a transposed W2 fails.
 """

@@ -3,11 +3,12 @@ re-quantize -> w2), combine.
 
 TEST INFRASTRUCTURE ONLY (see ``oracle/__init__``).
 
-Parity unpinned: expert_ffn_ref, expert_ffn_ref_mx and expert_ffn_ref_w4a8.
-The pages print no worked example of an expert or a layer, so these are
-checked only as compositions of pinned parts (the quantizers, the fp64
-matmul, SiLU's closed forms).  route, topk_softmax and combine_ref are
-pinned (library stable sort, brute force, hand-worked sums).
+Pins: the pages print no worked example of an expert or a layer.
+expert_ffn_ref, expert_ffn_ref_mx and expert_ffn_ref_w4a8 are pinned by a
+case worked by hand (tests/golden/expert_ffn_hand.txt): gates of +-100 (or
++-128) make SiLU exact in fp64 and every re-quantization lossless, so y is
+a sum of small integers.  route, topk_softmax and combine_ref are pinned by
+a library stable sort, brute force and hand-worked sums.
 
 Sources: "DeepSeek-V4 FP4 QAT" page §3.1 (simplified MoE forward: each token
 goes to its top-k experts, the expert outputs are summed); "DeepSeek-V4

@@ -131,3 +131,42 @@ def test_topk_softmax_brute_force_and_ties():
     # softmax of the chosen logits, closed form for one row
     sel = z[5, ids[5]].astype(np.float64)
     np.testing.assert_allclose(w[5], np.exp(sel) / np.exp(sel).sum(), rtol=1e-14)
+
+
+def _ffn_hand_case(P, I):
+    """The inputs of golden/expert_ffn_hand.txt (construction only)."""
+    H = 4
+    x = np.zeros((1, H))
+    x[0, 0] = 1.0
+    u = np.array([1, 2, 3, 4, 6], dtype=np.float64)[np.arange(I) % 5]
+    w1 = np.zeros((I, H))
+    w1[:, 0] = np.where(np.arange(I) % 2 == 0, P, -P)
+    w3 = np.zeros((I, H))
+    w3[:, 0] = u
+    w2 = ((np.arange(I)[None, :] + 2 * np.arange(H)[:, None]) % 3 - 1).astype(np.float64)
+    return x, w1, w3, w2
+
+
+def _ffn_golden(variant):
+    import os
+
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "expert_ffn_hand.txt")
+    rows = {l.split()[0]: [float(v) for v in l.split()[1:]] for l in open(path) if l.strip() and not l.startswith("#")}
+    return np.array(rows[variant])
+
+
+def test_expert_ffn_hand_worked_nv():
+    """The whole NVFP4 expert FFN on a case worked by hand
+    (golden/expert_ffn_hand.txt): SiLU on the gate rows only, the up rows as
+    the multiplier, h re-quantized losslessly with the static scale, y = h W2^T.
+    A swapped gate/up, a missing SiLU or a transposed W2 all change y."""
+    x, w1, w3, w2 = _ffn_hand_case(100.0, 16)
+    r = M.expert_ffn_ref(x, w1, w3, w2, np.float32(25.0 / 64.0))
+    assert np.array_equal(r["y"][0], _ffn_golden("nv"))
+    assert np.all(F.unpack_nibbles(r["h_codes"])[0, 1::2] == 8)  # the negative-gate rows: signed zeros
+
+
+def test_expert_ffn_hand_worked_mx():
+    x, w1, w3, w2 = _ffn_hand_case(128.0, 32)
+    r = M.expert_ffn_ref_mx(x, w1, w3, w2)
+    assert np.array_equal(r["y"][0], _ffn_golden("mx"))

@@ -150,3 +150,14 @@ def test_expert_ffn_w4a8_requantizes_h_to_mxfp8():
     err = np.abs(r["h_dq"] - r["h"].astype(np.float32))
     assert np.all(err <= 64.0 * np.exp2(X))
     np.testing.assert_allclose(r["y"], r["h_dq"] @ w2.T, rtol=1e-15)
+
+
+def test_expert_ffn_hand_worked_w4a8():
+    """The W4A8 expert FFN (MXFP8 h) on the hand-worked case of
+    golden/expert_ffn_hand.txt."""
+    from oracle import moe as M
+    from tests.test_oracle_gemm_moe import _ffn_golden, _ffn_hand_case
+
+    x, w1, w3, w2 = _ffn_hand_case(128.0, 32)
+    r = M.expert_ffn_ref_w4a8(x, w1, w3, w2)
+    assert np.array_equal(r["y"][0], _ffn_golden("w4a8"))
