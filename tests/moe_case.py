@@ -119,7 +119,25 @@ def oracle_token_rows(x_dq_rows, experts_w, slot_weights, g_h, fmt, h_tol_fn):
             gate, up = xr @ w1.T, xr @ w3.T
             h = MO.swiglu(gate, up)
             tol = h_tol_fn(xr, w1, w3, gate, up, h)
-            blk = 32 if fmt == "mx" else 16
+            blk = 32 if fmt in ("mx", "w4a8") else 16
+            if fmt == "w4a8":  # MXFP8 h: one E4M3 byte per element, magnitude in bits 0-6
+                hc, hs = Q.mxfp8_quantize(h.astype(np.float32))
+                h_dq = Q.mxfp8_dequantize(hc, hs)
+                lo_c, lo_s = Q.mxfp8_quantize((h - tol).astype(np.float32))
+                hi_c, hi_s = Q.mxfp8_quantize((h + tol).astype(np.float32))
+                mid = hc & 0x7F
+                unstable = ~((lo_s == hs) & (hi_s == hs) & ((lo_c & 0x7F) == mid).reshape(1, -1, blk).all(2) &
+                             ((hi_c & 0x7F) == mid).reshape(1, -1, blk).all(2))
+                # a different decision in the band moves an element by at most the
+                # block's largest coded magnitude: 448 x 2^X <= 2 amax
+                amax_hi = (np.abs(h) + tol).reshape(1, -1, blk).max(2)
+                dh = np.repeat(np.where(unstable, 2.0 * amax_hi, 0.0), blk, axis=1)
+                wt = float(slot_weights[t, s])
+                y = wt * (h_dq @ w2.T)
+                ref[t] += y[0]
+                sum_abs[t] += np.abs(y[0])
+                slack[t] += (abs(wt) * (dh @ np.abs(w2).T) + G.FP32_REL_TOL * abs(wt) * (np.abs(h_dq) @ np.abs(w2).T))[0]
+                continue
             if fmt == "mx":
                 hc, hs = Q.mxfp4_quantize(h.astype(np.float32))
                 h_dq = Q.mxfp4_dequantize(hc, hs)

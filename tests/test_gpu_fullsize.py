@@ -30,7 +30,7 @@ def _h_tol(xr, w1, w3, gate, up, h):
 
 
 @pytest.mark.parametrize("workload,tokens", [("pro", [0, 9999]), ("decode", [63]), ("flash", [17]), ("flashmx", [5]),
-                                             ("pro128k", [131071])])
+                                             ("flashw4a8", [2049]), ("pro128k", [131071])])
 def test_layer_full_size_sampled_tokens(workload, tokens):
     import bench
 
@@ -40,7 +40,9 @@ def test_layer_full_size_sampled_tokens(workload, tokens):
     assert b.fp4.fp4_get_device_status() == 0
     T, H, I, E, k, zipf, sigma, _ = bench.WORKLOADS[workload]
     xf = b.x.float().cpu().numpy()
-    if b.mx:
+    if b.w4a8:
+        x_dq = Q.mxfp8_dequantize(*Q.mxfp8_quantize(xf[tokens]))
+    elif b.mx:
         x_dq = Q.mxfp4_dequantize(*Q.mxfp4_quantize(xf[tokens]))
     else:
         g = Q.nv_global_scale(xf)
@@ -68,7 +70,8 @@ def test_layer_full_size_sampled_tokens(workload, tokens):
     cache = {}
     experts_w = [[cache.setdefault(int(e), oracle_weights(int(e))) for e in row] for row in ids]
     g_h = None if b.mx else [[hg[int(e)] for e in row] for row in ids]
-    ref, slack, sum_abs = moe_case.oracle_token_rows(x_dq, experts_w, wts, g_h, "mx" if b.mx else "nv", _h_tol)
+    fmt = "w4a8" if b.w4a8 else "mx" if b.mx else "nv"
+    ref, slack, sum_abs = moe_case.oracle_token_rows(x_dq, experts_w, wts, g_h, fmt, _h_tol)
     got_bits = bf16_bits(b.out)[tokens]
     got = F.bf16_bits_to_f32(got_bits).astype(np.float64)
     ulps = bf16_ulps_apart(got_bits, F.f64_to_bf16_rne(ref))
