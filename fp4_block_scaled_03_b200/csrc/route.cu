@@ -299,6 +299,66 @@ __global__ void combine_kernel(const float *__restrict__ y, const int32_t *__res
 // Router top-k: one warp per token.  Each of k rounds takes the warp-wide
 // largest remaining logit (ties to the lower expert id); the weights are the
 // softmax of the k chosen logits, fp32, summed in slot order.
+// Top-k for E <= 32 * kPerLane: each lane keeps its logits e = lane + 32j in
+// registers; a pass takes the warp's (largest value, lowest id) by shuffles
+// and marks the winner taken in the owning lane's bitmask.  Same choices, in
+// the same order, as the general kernel below.
+template <int kPerLane>
+__global__ void topk_softmax_reg_kernel(const float *__restrict__ logits, int64_t T, int32_t E, int32_t k,
+                                        int32_t *__restrict__ ids, float *__restrict__ weights,
+                                        int32_t *__restrict__ chunk_counts) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
+  for (int64_t t = blockIdx.x * (int64_t)(blockDim.x / 32) + (threadIdx.x >> 5); t < T; t += warps) {
+    const float *z = logits + t * E;
+    float v[kPerLane];
+#pragma unroll
+    for (int j = 0; j < kPerLane; ++j) {
+      const int e = lane + 32 * j;
+      v[j] = e < E ? z[e] : -INFINITY;
+    }
+    int chosen[16];
+    float val[16];
+    uint32_t taken = 0;  // bit j: this lane's e = lane + 32j already chosen
+    for (int s = 0; s < k; ++s) {
+      float best = -INFINITY;
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int j = 0; j < kPerLane; ++j) {
+        const int e = lane + 32 * j;
+        if (e < E && !((taken >> j) & 1u) && (v[j] > best || (v[j] == best && e < bi))) {
+          best = v[j];
+          bi = e;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, best, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (ov > best || (ov == best && oi < bi)) {
+          best = ov;
+          bi = oi;
+        }
+      }
+      chosen[s] = bi;
+      val[s] = best;
+      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+    }
+    if (lane == 0) {
+      float ex[16], sum = 0.0f;
+      for (int s = 0; s < k; ++s) {
+        ex[s] = expf(__fsub_rn(val[s], val[0]));
+        sum = __fadd_rn(sum, ex[s]);
+      }
+      for (int s = 0; s < k; ++s) {
+        ids[t * k + s] = chosen[s];
+        weights[t * k + s] = __fdiv_rn(ex[s], sum);
+        if (chunk_counts) atomicAdd(chunk_counts + ((t * k + s) / kChunk) * E + chosen[s], 1);
+      }
+    }
+  }
+}
+
 // With chunk_counts (zeroed, [nchunks][E]), each chosen slot also counts
 // into its routing chunk's histogram: the count pass of the routing, done
 // while the ids are in registers.
@@ -435,7 +495,10 @@ fp4_status fp4_moe_topk(const float *logits, int64_t T, int32_t E, int32_t topk,
   int64_t grid = (T + 7) / 8;
   const int64_t cap = (int64_t)sm_count() * 16;
   if (grid > cap) grid = cap;
-  topk_softmax_kernel<<<(unsigned)grid, 256, 0, s>>>(logits, T, E, topk, expert_ids, topk_weights, nullptr);
+  if (E <= 32 * 16)
+    topk_softmax_reg_kernel<16><<<(unsigned)grid, 256, 0, s>>>(logits, T, E, topk, expert_ids, topk_weights, nullptr);
+  else
+    topk_softmax_kernel<<<(unsigned)grid, 256, 0, s>>>(logits, T, E, topk, expert_ids, topk_weights, nullptr);
   FP4_HOST_CHECK(cudaGetLastError());
   return FP4_OK;
 }
@@ -479,7 +542,10 @@ fp4_status fp4_moe_router_route(const void *x_bf16, int64_t T, int64_t H, const 
   int64_t grid = (T + 7) / 8;
   const int64_t cap = (int64_t)sm_count() * 16;
   if (grid > cap) grid = cap;
-  topk_softmax_kernel<<<(unsigned)grid, 256, 0, s>>>(logits, T, E, topk, expert_ids, topk_weights, cc);
+  if (E <= 32 * 16)
+    topk_softmax_reg_kernel<16><<<(unsigned)grid, 256, 0, s>>>(logits, T, E, topk, expert_ids, topk_weights, cc);
+  else
+    topk_softmax_kernel<<<(unsigned)grid, 256, 0, s>>>(logits, T, E, topk, expert_ids, topk_weights, cc);
   FP4_HOST_CHECK(cudaGetLastError());
   route_scan_kernel<<<1, 1024, 2 * 1024 * 4, s>>>(cc, nchunks, E, counts, offsets, tile_offsets);
   FP4_HOST_CHECK(cudaGetLastError());

@@ -346,7 +346,8 @@ def _unstable_blocks(h, tol, g):
     return ~same
 
 
-@pytest.mark.parametrize("T,E,k,grid", [(4096, 384, 6, None), (777, 256, 8, None), (300, 64, 6, 0.25), (5, 16, 16, None)])
+@pytest.mark.parametrize("T,E,k,grid", [(4096, 384, 6, None), (777, 256, 8, None), (300, 64, 6, 0.25), (5, 16, 16, None),
+                                        (200, 1000, 6, 0.5), (100, 512, 16, 0.25)])
 def test_topk_softmax(T, E, k, grid):
     """Router top-k: ids bit-exact against the oracle's stable sort (ties to
     the lower id, forced by rounding logits to a coarse grid); weights within
