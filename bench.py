@@ -848,7 +848,7 @@ def run_router(args, world, rank, peaks):
         "data": "synthetic (seeded)",
         "config": {"workload": "Router at the Pro shape: 16384 tokens x hidden 7168 -> 384 expert logits, top-6",
                    "l2": "flushed (256 MB write) before each timed step"},
-        "roofline": {"bound": "tensor", "kernel": "fp4_gemm_kernel<256, f32, bf16>",
+        "roofline": {"bound": "tensor", "kernel": "fp4_gemm_kernel<192, f32, bf16>" if E % 192 == 0 and E % 256 else "fp4_gemm_kernel<256, f32, bf16>",
                      "achieved": round(flops / (gms * 1e-3) / 1e12, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
                      "frac": round(flops / (gms * 1e-3) / 1e12 / peak, 4), "traffic": None,
                      "peak_note": "measured burst bf16 cuBLAS, of " + peaks["src"]},

@@ -66,7 +66,7 @@ struct Cfg {
   static constexpr int SF_SLOT_COLS = 16 + 16 * HALVES;  // SFA: 4 K-words x 4; SFB: 4 x 4*HALVES
   static constexpr int SF_COL0 = 256;                     // slot s at SF_COL0 + s * SF_SLOT_COLS
   static constexpr int SMEM_BYTES = kStages * STAGE_BYTES + STG_BYTES + 1024 /*align*/ + 256 /*barriers*/;
-  static_assert(BN == 256, "the early-release epilogue splits 256 columns into two halves");
+  static_assert(BN == 256 || (BN == 192 && EPI == 0), "256-column tiles (192 for fp32-out bf16 GEMMs)");
   static_assert(SF_COL0 + kStages * SF_SLOT_COLS <= TMEM_COLS, "tmem");
   static_assert((3 * kStages + 4) * 8 <= 256, "barriers");
   static_assert(STAGE_BYTES % 1024 == 0, "stage buffers stay 1024-byte aligned");
@@ -636,10 +636,13 @@ fp4_status fp4_gemm_bf16(const void *a_bf16, const void *b_bf16, float *c, int64
   if (!ctx) return FP4_ERR_CUDA;
   CUtensorMap ta, tb;  // bf16 rows viewed as bytes: 128-byte swizzle rows of 64 elements
   if (!make_code_map(&ta, a_bf16, (uint64_t)M, (uint64_t)K * 2, BM)) return FP4_ERR_CUDA;
-  if (!make_code_map(&tb, b_bf16, (uint64_t)N, (uint64_t)K * 2, kBN)) return FP4_ERR_CUDA;
+  // 192-column tiles when they cover N exactly and 256-column ones would not
+  // (a 384-expert router: two full tiles instead of one and a half)
+  const int bn = (N % 192 == 0 && N % 256 != 0) ? 192 : kBN;
+  if (!make_code_map(&tb, b_bf16, (uint64_t)N, (uint64_t)K * 2, bn)) return FP4_ERR_CUDA;
   Params p = {};
   p.M = (int)M; p.N = (int)N; p.K = (int)K;
-  p.n_tiles = (int)((N + kBN - 1) / kBN);
+  p.n_tiles = (int)((N + bn - 1) / bn);
   p.m_tiles = (int)((M + BM - 1) / BM);
   p.k_stages = (int)(K / 64);
   p.kw = (int)(K / 16);  // MMA K steps of 16 elements
@@ -649,6 +652,7 @@ fp4_status fp4_gemm_bf16(const void *a_bf16, const void *b_bf16, float *c, int64
   const int64_t tiles = (int64_t)p.m_tiles * p.n_tiles;
   if (tiles > 2147483647LL) return FP4_ERR_UNSUPPORTED_SHAPE;
   const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
+  if (bn == 192) return launch<192, EPI_F32, 3>(ta, tb, tb, p, grid, reinterpret_cast<cudaStream_t>(stream));
   return launch<kBN, EPI_F32, 3>(ta, tb, tb, p, grid, reinterpret_cast<cudaStream_t>(stream));
 }
 
